@@ -1,0 +1,321 @@
+"""Python binding of libep.so, the B200 MoE token-routing library.
+
+Argument marshalling only: every function below checks dtypes and shapes,
+allocates missing outputs with torch (device memory is plumbing), passes raw
+pointers and the current CUDA stream to the C entry point of the same name,
+and raises on a non-zero return.  All computation runs in the CUDA kernels of
+``csrc/``; there is no CPU fallback -- importing this package without the built
+library, or calling it without a CUDA device, raises.
+
+Layouts and semantics are those of ``include/ep.h``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libep.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -c 'import __graft_entry__ as g; g.build()'` "
+        "or `python combine_get_dispatch_06_b200/build.py`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_Z = ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/ep.h
+_SIGS = {
+    "ep_status_string": (ctypes.c_char_p, [_I]),
+    "ep_version": (_I, []),
+    "ep_set_wait_timeout_ns": (_I, [ctypes.c_longlong]),
+    "ep_set_debug_flags": (_I, [ctypes.c_uint]),
+    "ep_get_dispatch_layout": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
+    "ep_dispatch_workspace_bytes": (_Z, [_I, _I, _I]),
+    "ep_dispatch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                         _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P]),
+    "ep_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "ep_ll_workspace_bytes": (_Z, [_I, _I, _I]),
+    "ep_ll_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
+                            _P, _Z, _P, _P]),
+    "ep_ll_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EP_OK, EP_ERR_INVALID_ARG, EP_ERR_CUDA, EP_ERR_UNSUPPORTED = 0, 1, 2, 3
+EP_STATUS_BAD_EXPERT = 1
+EP_STATUS_CAPACITY = 2
+EP_STATUS_WAIT_TIMEOUT = 4
+EP_STATUS_BAD_POSITION = 8
+EP_DEBUG_SUPPRESS_PUBLISH = 1
+
+
+class EPError(RuntimeError):
+    pass
+
+
+def _check(rc: int, what: str):
+    if rc != EP_OK:
+        raise EPError(f"{what}: {_lib.ep_status_string(rc).decode()} ({rc})")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise EPError("all tensors passed to libep must be CUDA tensors")
+    if not t.is_contiguous():
+        raise EPError("all tensors passed to libep must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _need(t: torch.Tensor, dtype, shape, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise EPError(f"{name}: expected {dtype} {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def ep_version() -> int:
+    return _lib.ep_version()
+
+
+def ep_status_string(code: int) -> str:
+    return _lib.ep_status_string(code).decode()
+
+
+def ep_set_wait_timeout_ns(ns: int) -> None:
+    _check(_lib.ep_set_wait_timeout_ns(int(ns)), "ep_set_wait_timeout_ns")
+
+
+def ep_set_debug_flags(flags: int) -> None:
+    _check(_lib.ep_set_debug_flags(int(flags)), "ep_set_debug_flags")
+
+
+def new_status(device=None) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+# ---------------------------------------------------------------------------
+# A1
+# ---------------------------------------------------------------------------
+
+def ep_get_dispatch_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, *,
+                           num_tokens_per_rank=None, num_tokens_per_expert=None,
+                           is_token_in_rank=None, status=None, stream=None):
+    """topk_idx int64 [S, T, K] (or [T, K] for one source rank) ->
+    (num_tokens_per_rank int32 [S, R], num_tokens_per_expert int32 [S, E],
+    is_token_in_rank bool [S, T, R])."""
+    squeeze = topk_idx.dim() == 2
+    idx = topk_idx.unsqueeze(0) if squeeze else topk_idx
+    S, T, K = idx.shape
+    R, E = num_ranks, num_experts
+    dev = idx.device
+    if squeeze:  # outputs given in the single-rank shapes
+        if num_tokens_per_rank is not None and num_tokens_per_rank.dim() == 1:
+            num_tokens_per_rank = num_tokens_per_rank.unsqueeze(0)
+        if num_tokens_per_expert is not None and num_tokens_per_expert.dim() == 1:
+            num_tokens_per_expert = num_tokens_per_expert.unsqueeze(0)
+        if is_token_in_rank is not None and is_token_in_rank.dim() == 2:
+            is_token_in_rank = is_token_in_rank.unsqueeze(0)
+    if num_tokens_per_rank is None:
+        num_tokens_per_rank = torch.empty((S, R), dtype=torch.int32, device=dev)
+    if num_tokens_per_expert is None:
+        num_tokens_per_expert = torch.empty((S, E), dtype=torch.int32, device=dev)
+    if is_token_in_rank is None:
+        is_token_in_rank = torch.empty((S, T, R), dtype=torch.bool, device=dev)
+    _need(idx, torch.int64, (S, T, K), "topk_idx")
+    _need(num_tokens_per_rank, torch.int32, (S, R), "num_tokens_per_rank")
+    _need(num_tokens_per_expert, torch.int32, (S, E), "num_tokens_per_expert")
+    _need(is_token_in_rank, torch.bool, (S, T, R), "is_token_in_rank")
+    rc = _lib.ep_get_dispatch_layout(
+        _ptr(idx), S, T, K, E, R, _ptr(num_tokens_per_rank), _ptr(num_tokens_per_expert),
+        _ptr(is_token_in_rank), _ptr(status), _stream(stream))
+    _check(rc, "ep_get_dispatch_layout")
+    if squeeze:
+        return num_tokens_per_rank[0], num_tokens_per_expert[0], is_token_in_rank[0]
+    return num_tokens_per_rank, num_tokens_per_expert, is_token_in_rank
+
+
+# ---------------------------------------------------------------------------
+# A2 + A3
+# ---------------------------------------------------------------------------
+
+def ep_dispatch_workspace_bytes(num_ranks: int, num_tokens: int, num_experts: int) -> int:
+    return int(_lib.ep_dispatch_workspace_bytes(num_ranks, num_tokens, num_experts))
+
+
+def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor],
+                topk_weights: Optional[torch.Tensor], num_experts: int, *,
+                is_token_in_rank: Optional[torch.Tensor] = None, expert_alignment: int = 1,
+                capacity: Optional[int] = None, out: Optional[dict] = None,
+                with_metadata: bool = True, workspace: Optional[torch.Tensor] = None,
+                status=None, stream=None) -> dict:
+    """x bf16 [R, T, H] -> dict of recv_x, recv_topk_idx, recv_topk_weights,
+    recv_src_idx, rank_prefix_matrix, recv_count, num_recv_tokens_per_expert,
+    send_pos (see ep.h).  Outputs given in ``out`` are reused."""
+    R, T, H = x.shape
+    dev = x.device
+    _need(x, torch.bfloat16, (R, T, H), "x")
+    K = topk_idx.shape[2] if topk_idx is not None else 0
+    E = num_experts
+    cap = R * T if capacity is None else int(capacity)
+    o = dict(out or {})
+
+    def get(name, shape, dtype):
+        if o.get(name) is None:
+            o[name] = torch.empty(shape, dtype=dtype, device=dev)
+        _need(o[name], dtype, shape, name)
+        return o[name]
+
+    get("recv_x", (R, cap, H), torch.bfloat16)
+    get("recv_src_idx", (R, cap), torch.int32)
+    get("rank_prefix_matrix", (R, R), torch.int32)
+    get("recv_count", (R,), torch.int32)
+    get("send_pos", (R, T, R), torch.int32)
+    meta = with_metadata and topk_idx is not None
+    if meta:
+        get("recv_topk_idx", (R, cap, K), torch.int64)
+        get("num_recv_tokens_per_expert", (R, E // R), torch.int32)
+        if topk_weights is not None:
+            get("recv_topk_weights", (R, cap, K), torch.float32)
+    if topk_idx is not None:
+        _need(topk_idx, torch.int64, (R, T, K), "topk_idx")
+    if topk_weights is not None:
+        _need(topk_weights, torch.float32, (R, T, K), "topk_weights")
+    if is_token_in_rank is not None:
+        _need(is_token_in_rank, torch.bool, (R, T, R), "is_token_in_rank")
+    need = ep_dispatch_workspace_bytes(R, T, E if topk_idx is not None else 0)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    rc = _lib.ep_dispatch(
+        _ptr(x), _ptr(topk_idx), _ptr(topk_weights), _ptr(is_token_in_rank), R, T, H, K, E,
+        int(expert_alignment), cap, _ptr(o["recv_x"]), _ptr(o.get("recv_topk_idx") if meta else None),
+        _ptr(o.get("recv_topk_weights") if meta else None), _ptr(o["recv_src_idx"]),
+        _ptr(o["rank_prefix_matrix"]), _ptr(o["recv_count"]),
+        _ptr(o.get("num_recv_tokens_per_expert") if meta else None), _ptr(o["send_pos"]),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+    _check(rc, "ep_dispatch")
+    return o
+
+
+# ---------------------------------------------------------------------------
+# A4
+# ---------------------------------------------------------------------------
+
+def ep_combine(y: torch.Tensor, send_pos: torch.Tensor,
+               recv_topk_weights: Optional[torch.Tensor] = None, *,
+               combined_x: Optional[torch.Tensor] = None,
+               combined_topk_weights: Optional[torch.Tensor] = None,
+               status=None, stream=None):
+    """y bf16 [R, cap, H], send_pos int32 [R, T, R] ->
+    (combined_x bf16 [R, T, H], combined_topk_weights fp32 [R, T, K] or None)."""
+    R, cap, H = y.shape
+    T = send_pos.shape[1]
+    dev = y.device
+    _need(y, torch.bfloat16, (R, cap, H), "y")
+    _need(send_pos, torch.int32, (R, T, R), "send_pos")
+    K = 0
+    if recv_topk_weights is not None:
+        K = recv_topk_weights.shape[2]
+        _need(recv_topk_weights, torch.float32, (R, cap, K), "recv_topk_weights")
+        if combined_topk_weights is None:
+            combined_topk_weights = torch.empty((R, T, K), dtype=torch.float32, device=dev)
+    if combined_x is None:
+        combined_x = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
+    _need(combined_x, torch.bfloat16, (R, T, H), "combined_x")
+    rc = _lib.ep_combine(
+        _ptr(y), _ptr(recv_topk_weights), _ptr(send_pos), R, T, H, K, cap, _ptr(combined_x),
+        _ptr(combined_topk_weights if recv_topk_weights is not None else None), _ptr(status),
+        _stream(stream))
+    _check(rc, "ep_combine")
+    return combined_x, (combined_topk_weights if recv_topk_weights is not None else None)
+
+
+# ---------------------------------------------------------------------------
+# A5 + A6
+# ---------------------------------------------------------------------------
+
+def ep_ll_workspace_bytes(num_ranks: int, num_tokens: int, num_experts: int) -> int:
+    return int(_lib.ep_ll_workspace_bytes(num_ranks, num_tokens, num_experts))
+
+
+def ep_ll_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int, *,
+                   use_fp8: bool = True, out: Optional[dict] = None,
+                   workspace: Optional[torch.Tensor] = None, status=None, stream=None) -> dict:
+    """x bf16 [R, T, H] -> dict of recv_x (uint8 e4m3 or bf16 [R, E_l, R*T, H]),
+    recv_scales (fp32 [R, E_l, R*T, H/128] or None), recv_count, recv_src_info,
+    layout_range, ll_pos."""
+    R, T, H = x.shape
+    K = topk_idx.shape[2]
+    E = num_experts
+    El = E // R
+    dev = x.device
+    _need(x, torch.bfloat16, (R, T, H), "x")
+    _need(topk_idx, torch.int64, (R, T, K), "topk_idx")
+    o = dict(out or {})
+
+    def get(name, shape, dtype):
+        if o.get(name) is None:
+            o[name] = torch.empty(shape, dtype=dtype, device=dev)
+        _need(o[name], dtype, shape, name)
+        return o[name]
+
+    get("recv_x", (R, El, R * T, H), torch.uint8 if use_fp8 else torch.bfloat16)
+    if use_fp8:
+        get("recv_scales", (R, El, R * T, H // 128), torch.float32)
+    else:
+        o["recv_scales"] = None
+    get("recv_count", (R, El), torch.int32)
+    get("recv_src_info", (R, El, R * T), torch.int32)
+    get("layout_range", (R, El, R, 2), torch.int32)
+    get("ll_pos", (R, T, K), torch.int32)
+    need = ep_ll_workspace_bytes(R, T, E)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    rc = _lib.ep_ll_dispatch(
+        _ptr(x), _ptr(topk_idx), R, T, H, K, E, 1 if use_fp8 else 0, _ptr(o["recv_x"]),
+        _ptr(o["recv_scales"]), _ptr(o["recv_count"]), _ptr(o["recv_src_info"]),
+        _ptr(o["layout_range"]), _ptr(o["ll_pos"]), _ptr(workspace), workspace.numel(),
+        _ptr(status), _stream(stream))
+    _check(rc, "ep_ll_dispatch")
+    return o
+
+
+def ep_ll_combine(y: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                  ll_pos: torch.Tensor, *, out: Optional[torch.Tensor] = None, status=None,
+                  stream=None) -> torch.Tensor:
+    """y bf16 [R, E_l, R*T, H] -> out bf16 [R, T, H]."""
+    R, El, cap, H = y.shape
+    T = topk_idx.shape[1]
+    K = topk_idx.shape[2]
+    E = R * El
+    _need(y, torch.bfloat16, (R, El, R * T, H), "y")
+    _need(topk_idx, torch.int64, (R, T, K), "topk_idx")
+    _need(topk_weights, torch.float32, (R, T, K), "topk_weights")
+    _need(ll_pos, torch.int32, (R, T, K), "ll_pos")
+    if out is None:
+        out = torch.empty((R, T, H), dtype=torch.bfloat16, device=y.device)
+    _need(out, torch.bfloat16, (R, T, H), "out")
+    rc = _lib.ep_ll_combine(_ptr(y), _ptr(topk_idx), _ptr(topk_weights), _ptr(ll_pos), R, T, H,
+                            K, E, _ptr(out), _ptr(status), _stream(stream))
+    _check(rc, "ep_ll_combine")
+    return out

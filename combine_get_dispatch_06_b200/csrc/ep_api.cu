@@ -1,0 +1,106 @@
+// ep_api.cu -- host-side helpers of the C ABI: status text, version, the
+// process-wide limits of the bounded device waits, device properties.
+#include <atomic>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "ep_common.cuh"
+
+namespace ep {
+
+namespace {
+std::atomic<unsigned long long> g_timeout_ns{1000000000ull};
+std::atomic<unsigned> g_flags{0u};
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices] = {0};
+std::mutex g_sms_mu;
+}  // namespace
+
+WaitConfig wait_config() {
+  WaitConfig c;
+  c.timeout_ns = g_timeout_ns.load(std::memory_order_relaxed);
+  c.flags = g_flags.load(std::memory_order_relaxed);
+  return c;
+}
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(g_sms_mu);
+  if (g_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sms[dev] = n;
+  }
+  return g_sms[dev];
+}
+
+int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+namespace {
+std::mutex g_attr_mu;
+std::map<std::pair<const void *, int>, size_t> g_smem_set;
+std::map<std::tuple<const void *, int, int, size_t>, int> g_occ;
+}  // namespace
+
+int ensure_dynamic_smem(const void *func, size_t bytes) {
+  if (bytes <= 48 * 1024) return EP_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return EP_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  size_t &cur = g_smem_set[{func, dev}];
+  if (cur >= bytes) return EP_OK;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(bytes)) != cudaSuccess)
+    return EP_ERR_CUDA;
+  cur = bytes;
+  return EP_OK;
+}
+
+int ctas_per_sm(const void *func, int threads, size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  auto key = std::make_tuple(func, dev, threads, smem);
+  auto it = g_occ.find(key);
+  if (it != g_occ.end()) return it->second;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, func, threads, smem) != cudaSuccess ||
+      n < 1)
+    n = 1;
+  g_occ[key] = n;
+  return n;
+}
+
+}  // namespace ep
+
+extern "C" {
+
+EP_API const char *ep_status_string(int code) {
+  switch (code) {
+    case EP_OK: return "ok";
+    case EP_ERR_INVALID_ARG: return "invalid argument";
+    case EP_ERR_CUDA: return "CUDA launch error";
+    case EP_ERR_UNSUPPORTED: return "unsupported shape";
+    default: return "unknown status";
+  }
+}
+
+EP_API int ep_version(void) { return 100; }
+
+EP_API int ep_set_wait_timeout_ns(long long ns) {
+  if (ns < 0) return EP_ERR_INVALID_ARG;
+  ep::g_timeout_ns.store(static_cast<unsigned long long>(ns), std::memory_order_relaxed);
+  return EP_OK;
+}
+
+EP_API int ep_set_debug_flags(unsigned flags) {
+  ep::g_flags.store(flags, std::memory_order_relaxed);
+  return EP_OK;
+}
+
+}  // extern "C"

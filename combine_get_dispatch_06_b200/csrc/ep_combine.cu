@@ -1,0 +1,140 @@
+// ep_combine.cu -- A4: combine (gather-reduce of the dispatched copies).
+//
+// Semantics (DeepEP legacy-test analysis page, combine call and its check
+// (combined_x - bias) / is_token_in_rank.sum(1) == x): every source token
+// gets back the sum of the rows its destinations return, summed in fp32 in
+// ascending destination rank, then rounded once to bf16 (nearest even).
+//
+// One warp per source token.  The warp reads send_pos[s][t][0..R), compacts
+// the valid (d, row) pairs in ascending d into shared memory with a ballot,
+// then each lane owns 16-byte chunks (8 channels) of the hidden row: it issues
+// the loads of two chunks from up to 8 rows at once (16 loads in flight per
+// lane), accumulates in fp32 in list order and writes 16 bytes back.
+// HBM-bound: N*H*2 bytes read, R*T*H*2 bytes written.
+#include <algorithm>
+
+#include "ep_common.cuh"
+
+namespace ep {
+namespace {
+
+constexpr int kCombineWarps = 8;
+constexpr int kCombineBatch = 8;
+
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 &v) {
+  acc[0] += bf16lo(v.x);
+  acc[1] += bf16hi(v.x);
+  acc[2] += bf16lo(v.y);
+  acc[3] += bf16hi(v.y);
+  acc[4] += bf16lo(v.z);
+  acc[5] += bf16hi(v.z);
+  acc[6] += bf16lo(v.w);
+  acc[7] += bf16hi(v.w);
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float (&a)[8]) {
+  uint4 r;
+  r.x = pack_bf16x2(a[0], a[1]);
+  r.y = pack_bf16x2(a[2], a[3]);
+  r.z = pack_bf16x2(a[4], a[5]);
+  r.w = pack_bf16x2(a[6], a[7]);
+  return r;
+}
+
+__global__ void __launch_bounds__(kCombineWarps * 32)
+    combine_kernel(const uint8_t *__restrict__ y, const float *__restrict__ recv_w,
+                   const int32_t *__restrict__ send_pos, int R, long num_tok, int H, int K,
+                   int cap, uint8_t *__restrict__ out, float *__restrict__ out_w,
+                   int32_t *status) {
+  extern __shared__ __align__(16) int64_t s_rows[];  // [warps][R] row indices d*cap + pos
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  int64_t *rows = s_rows + static_cast<size_t>(warp) * R;
+  const uint32_t lt = lanemask_lt();
+  const int nvec = H >> 3;
+  const long row_bytes = static_cast<long>(H) * 2;
+
+  for (long u = static_cast<long>(blockIdx.x) * kCombineWarps + warp; u < num_tok;
+       u += static_cast<long>(gridDim.x) * kCombineWarps) {
+    int n = 0;
+    bool bad = false;
+    for (int d0 = 0; d0 < R; d0 += 32) {
+      const int d = d0 + lane;
+      int pos = -1;
+      if (d < R) pos = __ldg(send_pos + u * R + d);
+      bad |= (pos < -1 || pos >= cap);
+      const bool take = pos >= 0 && pos < cap;
+      const uint32_t bal = __ballot_sync(0xffffffffu, take);
+      if (take) rows[n + __popc(bal & lt)] = static_cast<int64_t>(d) * cap + pos;
+      n += __popc(bal);
+    }
+    if (bad) report(status, EP_STATUS_BAD_POSITION);
+    __syncwarp();
+
+    uint8_t *orow = out + u * row_bytes;
+    for (int c = lane; c < nvec; c += 64) {
+      const bool two = c + 32 < nvec;
+      float a0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float a1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int i = 0; i < n; i += kCombineBatch) {
+        uint4 v0[kCombineBatch], v1[kCombineBatch];
+#pragma unroll
+        for (int b = 0; b < kCombineBatch; ++b) {
+          if (i + b < n) {
+            const uint8_t *r = y + rows[i + b] * row_bytes;
+            v0[b] = ld_stream_v4(r + static_cast<long>(c) * 16);
+            if (two) v1[b] = ld_stream_v4(r + static_cast<long>(c + 32) * 16);
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < kCombineBatch; ++b) {
+          if (i + b < n) {
+            add_bf16x8(a0, v0[b]);
+            if (two) add_bf16x8(a1, v1[b]);
+          }
+        }
+      }
+      st_stream_v4(orow + static_cast<long>(c) * 16, pack_bf16x8(a0));
+      if (two) st_stream_v4(orow + static_cast<long>(c + 32) * 16, pack_bf16x8(a1));
+    }
+    if (out_w != nullptr && lane < K) {
+      float a = 0.f;
+      for (int i = 0; i < n; ++i) a += __ldg(recv_w + rows[i] * K + lane);
+      out_w[u * K + lane] = a;
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace
+}  // namespace ep
+
+extern "C" EP_API int ep_combine(const void *y, const float *recv_topk_weights,
+                                 const int32_t *send_pos, int num_ranks, int num_tokens,
+                                 int hidden, int num_topk, int capacity, void *combined_x,
+                                 float *combined_topk_weights, int32_t *status,
+                                 cudaStream_t stream) {
+  using namespace ep;
+  const int R = num_ranks, T = num_tokens, H = hidden, K = num_topk, cap = capacity;
+  if (R < 1 || R > kMaxRanks || T < 0 || H < 8 || H % 8 != 0 || cap < 0) return EP_ERR_INVALID_ARG;
+  if (combined_topk_weights != nullptr &&
+      (recv_topk_weights == nullptr || K < 1 || K > kMaxTopk))
+    return EP_ERR_INVALID_ARG;
+  if (T == 0) return EP_OK;
+  if (y == nullptr || send_pos == nullptr || combined_x == nullptr) return EP_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(y) & 15u) || (reinterpret_cast<uintptr_t>(combined_x) & 15u))
+    return EP_ERR_INVALID_ARG;
+  const long num_tok = static_cast<long>(R) * T;
+  const int threads = kCombineWarps * 32;
+  const size_t smem = static_cast<size_t>(kCombineWarps) * R * sizeof(int64_t);
+  const void *fn = reinterpret_cast<const void *>(combine_kernel);
+  if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
+  const long want = (num_tok + kCombineWarps - 1) / kCombineWarps;
+  const long grid =
+      std::min<long>(want, static_cast<long>(ctas_per_sm(fn, threads, smem)) * num_sms());
+  combine_kernel<<<static_cast<unsigned>(grid), threads, smem, stream>>>(
+      static_cast<const uint8_t *>(y), combined_topk_weights ? recv_topk_weights : nullptr,
+      send_pos, R, num_tok, H, K, cap, static_cast<uint8_t *>(combined_x), combined_topk_weights,
+      status);
+  return launch_status();
+}

@@ -1,0 +1,409 @@
+// ep_dispatch.cu -- A2 + A3: rank prefix matrix, positions, dispatch scatter.
+//
+// Semantics (DeepEP "Python 接口" page, Dispatch API; legacy-test analysis
+// page, intranode handle tuple and check_data): the copy of token (s, t) to
+// rank d lands at row send_pos[s][t][d] of d's receive buffer, rows ordered by
+// source rank then token.  That row number is the exclusive prefix, over the
+// flattened (s, t) order, of is_token_in_rank[.][.][d]; its value at the end
+// of source rank s is the rank prefix matrix P[s][d].
+//
+// Two kernels:
+//   dispatch_scan_kernel  one CTA per 128-token tile: routing bits -> warp
+//                         ballots -> per-rank tile counts -> decoupled
+//                         look-back -> send_pos, recv_src_idx, received
+//                         top-k metadata, P, recv_count; expert counts are
+//                         reduced with shared + global atomics and finalised
+//                         by the last CTA.  Small (a few MB of traffic).
+//   dispatch_copy_kernel  the data movement: each token row is read ONCE from
+//                         HBM into shared memory by a bulk (TMA) copy and
+//                         written to each destination by bulk shared->global
+//                         copies, S stages deep.  HBM-bound: R*T*H*2 bytes
+//                         read, N*H*2 bytes written (N = number of copies).
+#include <algorithm>
+
+#include "ep_scan.cuh"
+
+namespace ep {
+namespace {
+
+constexpr int kMaskWords = (kMaxRanks + 31) / 32;
+
+struct DispatchScanParams {
+  const int64_t *topk_idx;
+  const float *topk_w;
+  const uint8_t *in_rank;
+  int R, T, K, E, El, cap, align, tiles_per_src, num_tiles, W;
+  int32_t *send_pos;
+  int32_t *recv_src_idx;
+  int64_t *recv_idx;
+  float *recv_w;
+  int32_t *P;
+  int32_t *recv_count;
+  int32_t *nrte;
+  ScanHeader *head;
+  int32_t *expert_cnt;
+  uint64_t *desc;
+  int32_t *status;
+  unsigned long long timeout_ns;
+  unsigned flags;
+};
+
+__global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanParams p) {
+  __shared__ int s_tile;
+  __shared__ int s_last;
+  __shared__ uint32_t s_mask[kScanTile * kMaskWords];
+  __shared__ int s_woff[kScanWarps][kMaxRanks];
+  __shared__ int s_excl[kMaxRanks];
+  __shared__ int s_ehist[kMaxExperts];
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const bool count_experts = p.nrte != nullptr;
+
+  if (tid == 0) s_tile = static_cast<int>(atomicAdd(&p.head->ticket, 1u));
+  if (count_experts)
+    for (int e = tid; e < p.E; e += kScanTile) s_ehist[e] = 0;
+  __syncthreads();
+
+  const int tile = s_tile;
+  const int s = tile / p.tiles_per_src;
+  const int t = (tile % p.tiles_per_src) * kScanTile + tid;
+  const bool valid = t < p.T;
+  const size_t st = static_cast<size_t>(s) * p.T + t;
+
+  // ---- routing bits of this token --------------------------------------
+  uint32_t *my_mask = s_mask + tid * p.W;
+  for (int w = 0; w < p.W; ++w) my_mask[w] = 0u;
+  if (valid) {
+    if (p.in_rank != nullptr) {
+      const uint8_t *ir = p.in_rank + st * p.R;
+      for (int d = 0; d < p.R; ++d)
+        if (ir[d]) my_mask[d >> 5] |= 1u << (d & 31);
+    }
+    if (p.topk_idx != nullptr && (p.in_rank == nullptr || count_experts)) {
+      const int64_t *row = p.topk_idx + st * p.K;
+      bool bad = false;
+      for (int k = 0; k < p.K; ++k) {
+        const int64_t e = row[k];
+        if (e == -1) continue;
+        if (e < -1 || e >= p.E) {
+          bad = true;
+          continue;
+        }
+        if (p.in_rank == nullptr) {
+          const int d = static_cast<int>(e) / p.El;
+          my_mask[d >> 5] |= 1u << (d & 31);
+        }
+        if (count_experts) atomicAdd(&s_ehist[static_cast<int>(e)], 1);
+      }
+      if (bad) report(p.status, EP_STATUS_BAD_EXPERT);
+    }
+  }
+  __syncthreads();
+
+  // ---- pass 1: per-warp count of tokens going to each rank ---------------
+  for (int d0 = 0; d0 < p.R; d0 += 32) {
+    const uint32_t word = my_mask[d0 >> 5];
+    const int nb = min(32, p.R - d0);
+    for (int b = 0; b < nb; ++b) {
+      const uint32_t bal = __ballot_sync(0xffffffffu, (word >> b) & 1u);
+      if (lane == 0) s_woff[warp][d0 + b] = __popc(bal);
+    }
+  }
+  __syncthreads();
+
+  // ---- tile totals, look-back, rank prefix matrix -----------------------
+  const bool publish = (p.flags & EP_DEBUG_SUPPRESS_PUBLISH) == 0;
+  const bool last_of_src = (tile % p.tiles_per_src) == p.tiles_per_src - 1;
+  for (int d = tid; d < p.R; d += kScanTile) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kScanWarps; ++w) {
+      const int c = s_woff[w][d];
+      s_woff[w][d] = run;
+      run += c;
+    }
+    const uint32_t excl =
+        lookback_column(p.desc, tile, p.R, d, static_cast<uint32_t>(run), publish, p.timeout_ns,
+                        p.status);
+    s_excl[d] = static_cast<int>(excl);
+    if (last_of_src) {
+      p.P[static_cast<size_t>(s) * p.R + d] = static_cast<int>(excl) + run;
+      if (tile == p.num_tiles - 1) p.recv_count[d] = static_cast<int>(excl) + run;
+    }
+  }
+  __syncthreads();
+
+  // ---- pass 2: positions, handle and received metadata -------------------
+  const uint32_t lt = lanemask_lt();
+  bool overflow = false;
+  for (int d0 = 0; d0 < p.R; d0 += 32) {
+    const uint32_t word = my_mask[d0 >> 5];
+    const int nb = min(32, p.R - d0);
+    for (int b = 0; b < nb; ++b) {
+      const int d = d0 + b;
+      const bool has = (word >> b) & 1u;
+      const uint32_t bal = __ballot_sync(0xffffffffu, has);
+      if (!valid) continue;
+      const int pos = has ? s_excl[d] + s_woff[warp][d] + __popc(bal & lt) : -1;
+      p.send_pos[st * p.R + d] = pos;
+      if (!has) continue;
+      if (pos < 0 || pos >= p.cap) {  // pos < 0 only after a timed-out look-back
+        overflow = true;
+        continue;
+      }
+      const size_t row = static_cast<size_t>(d) * p.cap + pos;
+      p.recv_src_idx[row] = t;
+      if (p.topk_idx != nullptr && (p.recv_idx != nullptr || p.recv_w != nullptr)) {
+        const int64_t *irow = p.topk_idx + st * p.K;
+        for (int k = 0; k < p.K; ++k) {
+          const int64_t e = irow[k];
+          const bool local = e >= 0 && e < p.E && static_cast<int>(e) / p.El == d;
+          if (p.recv_idx != nullptr)
+            p.recv_idx[row * p.K + k] = local ? e - static_cast<int64_t>(d) * p.El : -1;
+          if (p.recv_w != nullptr) p.recv_w[row * p.K + k] = local ? p.topk_w[st * p.K + k] : 0.0f;
+        }
+      }
+    }
+  }
+  if (overflow) report(p.status, EP_STATUS_CAPACITY);
+
+  // ---- expert counts -> num_recv_tokens_per_expert ----------------------
+  if (count_experts)
+    for (int e = tid; e < p.E; e += kScanTile) {
+      const int c = s_ehist[e];
+      if (c != 0) atomicAdd(&p.expert_cnt[e], c);
+    }
+  if (elect_last_cta(&p.head->done, static_cast<uint32_t>(p.num_tiles), &s_last) &&
+      count_experts) {
+    for (int e = tid; e < p.E; e += kScanTile) {
+      int n = __ldcg(&p.expert_cnt[e]);
+      if (p.align > 1) n = (n + p.align - 1) / p.align * p.align;
+      p.nrte[e] = n;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Row scatter.  One thread per destination rank (blockDim = 32 * ceil(R/32)),
+// thread 0 also drives the loads.  Items are (token, chunk) pairs; CTA b owns
+// tokens b, b + grid, b + 2*grid, ...  Stage i % S holds item i.  Loads run
+// S - 1 items ahead; before a stage is reloaded every thread waits until its
+// own bulk stores from that stage have finished reading shared memory.
+// ---------------------------------------------------------------------------
+
+constexpr int kCopyStages = 4;
+constexpr int kCopyChunkMax = 16384;
+
+template <int S>
+__global__ void __launch_bounds__(kMaxRanks)
+    dispatch_copy_kernel(const uint8_t *__restrict__ x, const int32_t *__restrict__ send_pos,
+                         uint8_t *__restrict__ recv_x, int R, long num_tok, int row_bytes,
+                         int chunk_bytes, int nchunks, int stage_stride, int cap,
+                         int32_t *status, unsigned long long timeout_ns) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+  uint8_t *buf = smem + 128;
+  const int tid = threadIdx.x;
+  const int d = tid;
+
+  const long ntok_cta =
+      static_cast<long>(blockIdx.x) < num_tok ? (num_tok - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const long nitems = ntok_cta * nchunks;
+
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  auto token_of = [&](long i) -> long {
+    return static_cast<long>(blockIdx.x) + (i / nchunks) * static_cast<long>(gridDim.x);
+  };
+  auto issue_load = [&](long i, int stg) {
+    const long u = token_of(i);
+    const int off = static_cast<int>(i % nchunks) * chunk_bytes;
+    const int nb = min(chunk_bytes, row_bytes - off);
+    mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(nb));
+    bulk_g2s(buf + stg * stage_stride, x + u * row_bytes + off, static_cast<uint32_t>(nb),
+             &bars[stg]);
+  };
+  auto load_pos = [&](long i) -> int {
+    return d < R ? __ldg(send_pos + token_of(i) * R + d) : -1;
+  };
+
+  int sp[S];
+#pragma unroll
+  for (int k = 0; k < S; ++k) sp[k] = -1;
+#pragma unroll
+  for (int k = 0; k < S - 1; ++k) {
+    if (k < nitems) {
+      if (tid == 0) issue_load(k, k);
+      sp[k] = load_pos(k);
+    }
+  }
+
+  bool all_ok = true;
+  long stop = nitems;  // first item whose load may still be in flight on failure
+  for (long base = 0; base < nitems && all_ok; base += S) {
+    const uint32_t parity = static_cast<uint32_t>((base / S) & 1);
+#pragma unroll
+    for (int st = 0; st < S; ++st) {
+      const long i = base + st;
+      if (i >= nitems) break;
+      const bool ok = mbar_wait_bounded(&bars[st], parity, timeout_ns);
+      const int chunk = static_cast<int>(i % nchunks);
+      if (ok && sp[st] >= 0) {  // sp < 0: no copy to this rank
+        if (sp[st] < cap) {
+          const int off = chunk * chunk_bytes;
+          const int nb = min(chunk_bytes, row_bytes - off);
+          bulk_s2g(recv_x + (static_cast<long>(d) * cap + sp[st]) * row_bytes + off,
+                   buf + st * stage_stride, static_cast<uint32_t>(nb));
+        } else if (chunk == 0) {
+          report(status, EP_STATUS_CAPACITY);
+        }
+      }
+      bulk_commit();
+      bulk_wait_read<1>();
+      all_ok = __syncthreads_and(ok) != 0;
+      if (!all_ok) {
+        stop = i;
+        break;
+      }
+      const long j = i + S - 1;
+      const int ps = (st + S - 1) % S;
+      if (j < nitems) {
+        if (tid == 0) issue_load(j, ps);
+        sp[ps] = load_pos(j);
+      }
+    }
+  }
+  bulk_wait_all<0>();
+  if (!all_ok) {
+    report(status, EP_STATUS_WAIT_TIMEOUT);
+    if (tid == 0) {
+      // drain loads still in flight before the CTA's shared memory goes away
+      const long end = min(nitems, stop + S - 1);
+      for (long k = stop; k < end; ++k)
+        (void)mbar_wait_bounded(&bars[k % S], static_cast<uint32_t>((k / S) & 1), timeout_ns);
+    }
+  }
+}
+
+}  // namespace
+}  // namespace ep
+
+extern "C" EP_API size_t ep_dispatch_workspace_bytes(int num_ranks, int num_tokens,
+                                                     int num_experts) {
+  using namespace ep;
+  if (num_ranks < 1 || num_tokens < 0 || num_experts < 0) return 0;
+  const long tiles = static_cast<long>(num_ranks) * ((num_tokens + kScanTile - 1) / kScanTile);
+  return scan_workspace_bytes(tiles, num_ranks, num_experts);
+}
+
+extern "C" EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
+                                  const float *topk_weights, const uint8_t *is_token_in_rank,
+                                  int num_ranks, int num_tokens, int hidden, int num_topk,
+                                  int num_experts, int expert_alignment, int capacity,
+                                  void *recv_x, int64_t *recv_topk_idx, float *recv_topk_weights,
+                                  int32_t *recv_src_idx, int32_t *rank_prefix_matrix,
+                                  int32_t *recv_count, int32_t *num_recv_tokens_per_expert,
+                                  int32_t *send_pos, void *workspace, size_t workspace_bytes,
+                                  int32_t *status, cudaStream_t stream) {
+  using namespace ep;
+  const int R = num_ranks, T = num_tokens, H = hidden, K = num_topk, E = num_experts;
+  const int cap = capacity;
+  if (R < 1 || R > kMaxRanks || T < 0 || H < 8 || H % 8 != 0 || cap < 0 || expert_alignment < 1)
+    return EP_ERR_INVALID_ARG;
+  if (rank_prefix_matrix == nullptr || recv_count == nullptr) return EP_ERR_INVALID_ARG;
+  if (T == 0) {  // nothing to route; an empty tensor's pointers may be NULL
+    if (num_recv_tokens_per_expert != nullptr &&
+        (E < 1 || E > kMaxExperts || E % R != 0))
+      return EP_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(rank_prefix_matrix, 0, sizeof(int32_t) * R * R, stream) != cudaSuccess ||
+        cudaMemsetAsync(recv_count, 0, sizeof(int32_t) * R, stream) != cudaSuccess)
+      return EP_ERR_CUDA;
+    if (num_recv_tokens_per_expert != nullptr &&
+        cudaMemsetAsync(num_recv_tokens_per_expert, 0, sizeof(int32_t) * E, stream) !=
+            cudaSuccess)
+      return EP_ERR_CUDA;
+    return EP_OK;
+  }
+  if (topk_idx == nullptr && is_token_in_rank == nullptr) return EP_ERR_INVALID_ARG;
+  if (topk_idx != nullptr &&
+      (K < 1 || K > kMaxTopk || E < 1 || E > kMaxExperts || E % R != 0))
+    return EP_ERR_INVALID_ARG;
+  if ((recv_topk_idx != nullptr || num_recv_tokens_per_expert != nullptr) && topk_idx == nullptr)
+    return EP_ERR_INVALID_ARG;
+  if (recv_topk_weights != nullptr && (topk_idx == nullptr || topk_weights == nullptr))
+    return EP_ERR_INVALID_ARG;
+  const int El = topk_idx != nullptr ? E / R : 1;
+  if (send_pos == nullptr || recv_src_idx == nullptr || x == nullptr ||
+      (cap > 0 && recv_x == nullptr))
+    return EP_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(recv_x) & 15u))
+    return EP_ERR_INVALID_ARG;
+  const int Ectr = topk_idx != nullptr ? E : 0;
+  const size_t need = ep_dispatch_workspace_bytes(R, T, Ectr);
+  if (workspace == nullptr || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 15u))
+    return EP_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return EP_ERR_CUDA;
+
+  const int tiles_per_src = (T + kScanTile - 1) / kScanTile;
+  const long num_tiles = static_cast<long>(R) * tiles_per_src;
+  if (num_tiles > 0x7fffffffL || static_cast<long>(R) * T > 0x7fffffffL)
+    return EP_ERR_UNSUPPORTED;
+
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  DispatchScanParams p;
+  p.topk_idx = topk_idx;
+  p.topk_w = topk_weights;
+  p.in_rank = is_token_in_rank;
+  p.R = R;
+  p.T = T;
+  p.K = K;
+  p.E = E;
+  p.El = El;
+  p.cap = cap;
+  p.align = expert_alignment;
+  p.tiles_per_src = tiles_per_src;
+  p.num_tiles = static_cast<int>(num_tiles);
+  p.W = (R + 31) / 32;
+  p.send_pos = send_pos;
+  p.recv_src_idx = recv_src_idx;
+  p.recv_idx = recv_topk_idx;
+  p.recv_w = recv_topk_weights;
+  p.P = rank_prefix_matrix;
+  p.recv_count = recv_count;
+  p.nrte = num_recv_tokens_per_expert;
+  p.head = reinterpret_cast<ScanHeader *>(ws);
+  p.expert_cnt = reinterpret_cast<int32_t *>(ws + sizeof(ScanHeader));
+  p.desc = reinterpret_cast<uint64_t *>(ws + sizeof(ScanHeader) +
+                                        static_cast<size_t>((Ectr + 3) & ~3) * 4);
+  p.status = status;
+  const WaitConfig wc = wait_config();
+  p.timeout_ns = wc.timeout_ns;
+  p.flags = wc.flags;
+  dispatch_scan_kernel<<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
+  if (launch_status() != EP_OK) return EP_ERR_CUDA;
+
+  if (cap == 0) return EP_OK;
+  const int row_bytes = H * 2;
+  const int nchunks = (row_bytes + kCopyChunkMax - 1) / kCopyChunkMax;
+  const int chunk_bytes = ((row_bytes + nchunks - 1) / nchunks + 15) & ~15;
+  const int stage_stride = (chunk_bytes + 127) & ~127;
+  const size_t smem = 128 + static_cast<size_t>(kCopyStages) * stage_stride;
+  const int threads = 32 * ((R + 31) / 32);
+  const void *fn = reinterpret_cast<const void *>(dispatch_copy_kernel<kCopyStages>);
+  if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
+  const long num_tok = static_cast<long>(R) * T;
+  const long grid = std::min<long>(num_tok, static_cast<long>(ctas_per_sm(fn, threads, smem)) *
+                                                num_sms());
+  dispatch_copy_kernel<kCopyStages><<<static_cast<unsigned>(grid), threads, smem, stream>>>(
+      static_cast<const uint8_t *>(x), send_pos, static_cast<uint8_t *>(recv_x), R, num_tok,
+      row_bytes, chunk_bytes, nchunks, stage_stride, cap, status, wc.timeout_ns);
+  return launch_status();
+}

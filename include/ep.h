@@ -1,0 +1,254 @@
+/*
+ * ep.h -- C ABI of the B200 MoE token-routing library (libep.so).
+ *
+ * The library computes the data-parallel hot path of expert-parallel token
+ * routing as the DeepEP pages describe it, with all R ranks simulated inside
+ * one GPU's HBM: every "rank" is a slice of one allocation, and a copy to a
+ * rank is a store into that rank's slice.  There is no inter-GPU transfer.
+ *
+ * General rules (all entry points):
+ *   - Every pointer argument is DEVICE memory owned by the caller, except
+ *     where a comment says "host".  The library never allocates device memory
+ *     and never frees what it is given.  Scratch memory ("workspace") is sized
+ *     by ep_*_workspace_bytes() and passed in by the caller; the library clears
+ *     it on the stream at the start of each call.
+ *   - Every call is asynchronous on `stream` and never synchronises the host.
+ *     The caller orders calls with events.  Calls are stateless and may run
+ *     concurrently if they use distinct output and workspace buffers.
+ *   - The return value is a host-side status (EP_OK ... EP_ERR_UNSUPPORTED).
+ *     Argument checks happen before anything is launched; on an error nothing
+ *     is launched and no output is touched.
+ *   - Errors the GPU detects (a bad expert id, a receive buffer too small, a
+ *     bounded wait that ran out) are never trapped.  The kernels skip the
+ *     offending access and OR an EP_STATUS_* bit into the optional device word
+ *     `status` (int32), which the caller zeroes beforehand and reads after its
+ *     own synchronisation.  A NULL `status` discards these reports.
+ *   - Layouts are row-major and contiguous.  "[R, T, H]" means R*T*H elements,
+ *     the last index fastest.  bf16 data is passed as raw 16-bit patterns
+ *     (void*), e4m3 data as bytes.
+ *
+ * Notation: R ranks (every rank is a source and a destination), T tokens per
+ * source rank, H hidden size, K top-k slots per token, E experts in total,
+ * E_l = E / R experts per rank (expert e lives on rank e / E_l, local id
+ * e % E_l), cap = rows per destination rank in the normal receive buffer.
+ *
+ * Limits (from the get_dispatch_layout specification: 1 <= K <= 16,
+ * 1 <= E <= 512 with E % R == 0, R <= 384): calls outside them return
+ * EP_ERR_INVALID_ARG.
+ */
+#ifndef EP_H_
+#define EP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define EP_API __attribute__((visibility("default")))
+#else
+#define EP_API
+#endif
+
+/* Host-side return codes. */
+#define EP_OK               0  /* launched                                   */
+#define EP_ERR_INVALID_ARG  1  /* a size, pointer or alignment check failed  */
+#define EP_ERR_CUDA         2  /* the CUDA runtime reported a launch error   */
+#define EP_ERR_UNSUPPORTED  3  /* valid call, shape this build cannot run    */
+
+/* Device-side status bits, OR-ed into `status`. */
+#define EP_STATUS_BAD_EXPERT       1  /* a top-k id outside [-1, E); slot ignored      */
+#define EP_STATUS_CAPACITY         2  /* a copy's row >= cap; copy not written         */
+#define EP_STATUS_WAIT_TIMEOUT     4  /* a bounded wait ran out; results are invalid   */
+#define EP_STATUS_BAD_POSITION     8  /* a send_pos / ll_pos entry outside its buffer  */
+
+/* Debug flags for ep_set_debug_flags(). */
+#define EP_DEBUG_SUPPRESS_PUBLISH  1u /* scan tiles publish nothing, so every tile but
+                                         the first waits until its limit runs out:
+                                         exercises EP_STATUS_WAIT_TIMEOUT            */
+
+/* Text for a host return code. */
+EP_API const char *ep_status_string(int code);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+EP_API int ep_version(void);
+
+/* Process-wide limit of every bounded device wait, in nanoseconds of
+ * %globaltimer (default 1e9, i.e. one second).  Applies to launches issued
+ * after the call.  Returns EP_ERR_INVALID_ARG for a negative value. */
+EP_API int ep_set_wait_timeout_ns(long long ns);
+
+/* Process-wide debug flags (EP_DEBUG_*); 0 restores normal operation. */
+EP_API int ep_set_debug_flags(unsigned flags);
+
+/*
+ * A1: get_dispatch_layout.
+ * Passage: the get_dispatch_layout API (GET_DISPATCH_LAYOUT_API page,
+ * "Parameters" and "Return Values"; DeepEP "Python 接口" page, Dispatch API
+ * inputs num_tokens_per_rank, is_token_in_rank, num_tokens_per_expert).
+ *
+ *   topk_idx               in  int64 [S, T, K]; -1 marks an unselected slot
+ *   num_src_ranks (S)      source ranks whose tokens are in topk_idx (S >= 1;
+ *                          S = 1 is the pages' single-rank call)
+ *   num_tokens (T) >= 0, num_topk (K), num_experts (E), num_ranks (R)
+ *   num_tokens_per_rank    out int32 [S, R]: tokens of s with >= 1 expert on d
+ *   num_tokens_per_expert  out int32 [S, E]: slots of s that select e
+ *   is_token_in_rank       out uint8 [S, T, R]: 1 if (s,t) goes to d, else 0
+ *
+ * A repeated expert in one token counts twice in num_tokens_per_expert and
+ * once in is_token_in_rank.  Ids outside [-1, E) are ignored and reported as
+ * EP_STATUS_BAD_EXPERT.
+ */
+EP_API int ep_get_dispatch_layout(const int64_t *topk_idx, int num_src_ranks,
+                                  int num_tokens, int num_topk, int num_experts,
+                                  int num_ranks, int32_t *num_tokens_per_rank,
+                                  int32_t *num_tokens_per_expert,
+                                  uint8_t *is_token_in_rank, int32_t *status,
+                                  cudaStream_t stream);
+
+/* Workspace bytes ep_dispatch needs for R ranks, T tokens and E experts. */
+EP_API size_t ep_dispatch_workspace_bytes(int num_ranks, int num_tokens,
+                                          int num_experts);
+
+/*
+ * A2 + A3: rank prefix matrix, positions, and the dispatch scatter.
+ * Passage: Buffer.dispatch (DeepEP "Python 接口" page, Dispatch API inputs
+ * and outputs; intranode handle tuple and check_data's inclusive
+ * recv_gbl_rank_prefix_sum walk on the DeepEP legacy-test analysis page).
+ *
+ * Inputs:
+ *   x                  bf16 [R, T, H], H % 8 == 0, 16-byte aligned
+ *   topk_idx           int64 [R, T, K] or NULL (then is_token_in_rank is
+ *                      required and no metadata or expert counts are written)
+ *   topk_weights       fp32 [R, T, K] or NULL
+ *   is_token_in_rank   uint8 [R, T, R] or NULL.  If given it decides which
+ *                      ranks receive each token (topk_idx then only fills the
+ *                      received metadata); if NULL the routing is computed
+ *                      from topk_idx (rank of each valid slot's expert).
+ *   expert_alignment   >= 1; capacity (cap) >= 0 rows per destination rank
+ *                      (cap = R*T can never overflow)
+ * Outputs (rows of destination d are numbered by source rank, then token):
+ *   recv_x             bf16 [R, cap, H]: row p of d = x of the p-th token
+ *                      d receives.  Rows >= recv_count[d] are not touched.
+ *   recv_topk_idx      int64 [R, cap, K] or NULL: local expert id (e - d*E_l)
+ *                      for slots whose expert lives on d, else -1
+ *   recv_topk_weights  fp32 [R, cap, K] or NULL: the weight for local slots,
+ *                      else 0.0 (needs topk_weights)
+ *   recv_src_idx       int32 [R, cap]: source token index t of each row
+ *   rank_prefix_matrix int32 [R, R]: P[s][d] = tokens ranks 0..s send to d
+ *   recv_count         int32 [R]: P[R-1][d]
+ *   num_recv_tokens_per_expert int32 [R, E_l] or NULL: slots received per
+ *                      local expert, rounded up to expert_alignment (needs
+ *                      topk_idx)
+ *   send_pos           int32 [R, T, R]: row of (s,t) inside d, or -1.
+ *                      (rank_prefix_matrix, recv_src_idx, is_token_in_rank,
+ *                      send_pos and recv_count form the dispatch handle.)
+ *   workspace          ep_dispatch_workspace_bytes(R, T, E) bytes, any content
+ * A copy whose row is >= cap is not written and sets EP_STATUS_CAPACITY;
+ * send_pos still holds its row.
+ */
+EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
+                       const float *topk_weights,
+                       const uint8_t *is_token_in_rank, int num_ranks,
+                       int num_tokens, int hidden, int num_topk,
+                       int num_experts, int expert_alignment, int capacity,
+                       void *recv_x, int64_t *recv_topk_idx,
+                       float *recv_topk_weights, int32_t *recv_src_idx,
+                       int32_t *rank_prefix_matrix, int32_t *recv_count,
+                       int32_t *num_recv_tokens_per_expert, int32_t *send_pos,
+                       void *workspace, size_t workspace_bytes,
+                       int32_t *status, cudaStream_t stream);
+
+/*
+ * A4: combine (gather-reduce).
+ * Passage: Buffer.combine (DeepEP legacy-test analysis page, combine_args and
+ * the check that (combined_x - bias) / is_token_in_rank.sum(1) equals x).
+ *
+ *   y                      bf16 [R, cap, H], the experts' outputs, row for row
+ *                          as ep_dispatch laid out recv_x (identity experts:
+ *                          y = recv_x); H % 8 == 0, 16-byte aligned
+ *   recv_topk_weights      fp32 [R, cap, K] or NULL
+ *   send_pos               int32 [R, T, R] from ep_dispatch
+ *   combined_x             out bf16 [R, T, H]:
+ *                          bf16_rne( sum over d ascending with send_pos >= 0
+ *                          of float(y[d][send_pos]) ), fp32 accumulation from
+ *                          +0.0; a token with no destination gives +0.0
+ *   combined_topk_weights  out fp32 [R, T, K] or NULL: the same ascending sum
+ *                          of recv_topk_weights (needs recv_topk_weights)
+ * A send_pos entry outside [-1, cap) is skipped and sets
+ * EP_STATUS_BAD_POSITION.
+ */
+EP_API int ep_combine(const void *y, const float *recv_topk_weights,
+                      const int32_t *send_pos, int num_ranks, int num_tokens,
+                      int hidden, int num_topk, int capacity, void *combined_x,
+                      float *combined_topk_weights, int32_t *status,
+                      cudaStream_t stream);
+
+/* Workspace bytes ep_ll_dispatch needs for R ranks, T tokens, E experts. */
+EP_API size_t ep_ll_workspace_bytes(int num_ranks, int num_tokens,
+                                    int num_experts);
+
+/*
+ * A5: low-latency dispatch with fused FP8 quantisation.
+ * Passage: Buffer.low_latency_dispatch (DeepEP legacy-test analysis page, the
+ * low_latency_dispatch call, its handle (recv_src_info, recv_layout_range)
+ * and its per-expert count and per-source-rank checks; FP8 input described on
+ * the "Python 接口" page as e4m3 values with fp32 scales per 128 channels).
+ *
+ * Each (token, expert) pair gets one row of that expert's slab; rows are
+ * ordered by source rank, then token.  Slabs hold R*T rows, so they never
+ * overflow.
+ *   x              bf16 [R, T, H]; H % 128 == 0 for FP8, H % 8 == 0 for bf16
+ *   topk_idx       int64 [R, T, K]
+ *   use_fp8        1: recv_x is e4m3 [R, E_l, R*T, H] and recv_scales fp32
+ *                  [R, E_l, R*T, H/128] with, per 128-channel block,
+ *                  amax' = max(max|x|, 1e-4), q = e4m3_rne_satfinite(x *
+ *                  (448 / amax')), scale = amax' / 448;
+ *                  0: recv_x is bf16 [R, E_l, R*T, H], recv_scales unused
+ *   recv_count     out int32 [R, E_l]: rows of each local expert
+ *   recv_src_info  out int32 [R, E_l, R*T]: source token index of each row
+ *   layout_range   out int32 [R, E_l, R, 2]: (first row, rows) per source rank
+ *   ll_pos         out int32 [R, T, K]: slab row of each slot, -1 if the slot
+ *                  is unselected or invalid (a repeated expert in a token
+ *                  shares its first slot's row)
+ *   workspace      ep_ll_workspace_bytes(R, T, E) bytes, any content
+ */
+EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
+                          int num_ranks, int num_tokens, int hidden,
+                          int num_topk, int num_experts, int use_fp8,
+                          void *recv_x, float *recv_scales,
+                          int32_t *recv_count, int32_t *recv_src_info,
+                          int32_t *layout_range, int32_t *ll_pos,
+                          void *workspace, size_t workspace_bytes,
+                          int32_t *status, cudaStream_t stream);
+
+/*
+ * A6: low-latency combine with top-k weights.
+ * Passage: Buffer.low_latency_combine (DeepEP legacy-test analysis page, the
+ * low_latency_combine call and the check that the result equals x times the
+ * sum of the top-k weights with unselected slots masked to 0).
+ *
+ *   y              bf16 [R, E_l, R*T, H], the experts' outputs laid out as
+ *                  ep_ll_dispatch laid out its slabs; H % 8 == 0
+ *   topk_idx, topk_weights  int64 / fp32 [R, T, K]
+ *   ll_pos         int32 [R, T, K] from ep_ll_dispatch
+ *   out            bf16 [R, T, H]: bf16_rne(acc), acc = +0.0 then, for k
+ *                  ascending over valid slots, acc = fmaf(float(y[e][ll_pos]),
+ *                  w[k], acc)
+ * A slot with a valid expert but ll_pos outside [0, R*T) is skipped and sets
+ * EP_STATUS_BAD_POSITION.
+ */
+EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
+                         const float *topk_weights, const int32_t *ll_pos,
+                         int num_ranks, int num_tokens, int hidden,
+                         int num_topk, int num_experts, void *out,
+                         int32_t *status, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_H_ */

@@ -299,6 +299,7 @@ def ll_combine(y, topk_idx, topk_weights, ll_pos, tokens=None) -> np.ndarray:
     R, El, cap, H = yy.shape
     T = idx.shape[1]
     K = idx.shape[2]
+    assert idx.shape[0] == R and cap == R * T, "y must be [R, E_l, R*T, H] for topk_idx [R, T, K]"
     out = np.zeros((R, T, H), np.uint16)
     tk, nt = _tokens(tokens)
     lib().orc_ll_combine(_ptr(yy), _ptr(idx), _ptr(w), _ptr(pos), R, T, H, K, R * El,

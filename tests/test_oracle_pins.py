@@ -248,10 +248,24 @@ def test_combine_identity_closed_form(name):
     idx, wts, x = inp["topk_idx"], inp["topk_weights"], inp["x"]
     res = oracle.normal_path(x, idx, wts, w.E)
     n_dest = res["is_token_in_rank"].sum(axis=2).astype(np.float64)
-    expect = f2b((n_dest[..., None] * b2f(x).astype(np.float64)).astype(np.float32))
+    # n * x is exact in fp32; the sum starts from +0.0, so -0.0 inputs give +0.0
+    expect = f2b((n_dest[..., None] * b2f(x).astype(np.float64) + 0.0).astype(np.float32))
     np.testing.assert_array_equal(res["combined_x"], expect)
     masked = np.where((idx >= 0) & (idx < w.E), wts, np.float32(0.0))
     np.testing.assert_array_equal(res["combined_topk_weights"], masked)
+
+
+def test_combine_signed_zero():
+    # one token to two ranks, payload -0.0 everywhere: the fp32 sum from +0.0
+    # gives +0.0 (IEEE: +0 + -0 = +0 under round to nearest)
+    idx = np.array([[[0, 1]]], np.int64)          # R=1 would keep one copy; use R=2
+    idx = np.array([[[0, 2]], [[-1, -1]]], np.int64)
+    x = np.full((2, 1, 8), 0x8000, np.uint16)    # -0.0
+    w = np.ones((2, 1, 2), np.float32)
+    res = oracle.normal_path(x, idx, w, 4)
+    assert res["recv_count"].tolist() == [1, 1]
+    assert (res["combined_x"][0, 0] == 0x0000).all()
+    assert (res["combined_x"][1, 0] == 0x0000).all()
 
 
 def test_combine_random_y_error_bound():
