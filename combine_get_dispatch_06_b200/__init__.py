@@ -41,6 +41,8 @@ _SIGS = {
     "ep_dispatch_workspace_bytes": (_Z, [_I, _I, _I]),
     "ep_dispatch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                          _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P]),
+    "ep_dispatch_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                 _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "ep_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "ep_ll_workspace_bytes": (_Z, [_I, _I, _I]),
     "ep_ll_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
@@ -214,6 +216,45 @@ def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor],
         _ptr(o.get("num_recv_tokens_per_expert") if meta else None), _ptr(o["send_pos"]),
         _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
     _check(rc, "ep_dispatch")
+    return o
+
+
+def ep_dispatch_noalloc(x: torch.Tensor, topk_idx: Optional[torch.Tensor],
+                        topk_weights: Optional[torch.Tensor], num_experts: int, *,
+                        is_token_in_rank: Optional[torch.Tensor] = None,
+                        expert_alignment: int = 1, capacity: Optional[int] = None,
+                        out: Optional[dict] = None, status=None, stream=None) -> dict:
+    """ep_dispatch for callers that cannot allocate device memory when they call
+    (their memory belongs to another allocator, or cudaMalloc is too slow for
+    their loop): the scratch is a static 2 MiB array inside the library.  All
+    outputs must be passed in ``out``; nothing is allocated here.  Calls that
+    overlap on the GPU share that array and race."""
+    R, T, H = x.shape
+    _need(x, torch.bfloat16, (R, T, H), "x")
+    K = topk_idx.shape[2] if topk_idx is not None else 0
+    E = num_experts
+    cap = R * T if capacity is None else int(capacity)
+    o = dict(out or {})
+    shapes = {"recv_x": ((R, cap, H), torch.bfloat16), "recv_src_idx": ((R, cap), torch.int32),
+              "rank_prefix_matrix": ((R, R), torch.int32), "recv_count": ((R,), torch.int32),
+              "send_pos": ((R, T, R), torch.int32)}
+    if topk_idx is not None:
+        shapes["recv_topk_idx"] = ((R, cap, K), torch.int64)
+        shapes["num_recv_tokens_per_expert"] = ((R, E // R), torch.int32)
+        if topk_weights is not None:
+            shapes["recv_topk_weights"] = ((R, cap, K), torch.float32)
+    for name, (shape, dtype) in shapes.items():
+        if o.get(name) is None:
+            raise EPError(f"ep_dispatch_noalloc allocates nothing: pass out[{name!r}]")
+        _need(o[name], dtype, shape, name)
+    rc = _lib.ep_dispatch_noalloc(
+        _ptr(x), _ptr(topk_idx), _ptr(topk_weights), _ptr(is_token_in_rank), R, T, H, K, E,
+        int(expert_alignment), cap, _ptr(o["recv_x"]), _ptr(o.get("recv_topk_idx")),
+        _ptr(o.get("recv_topk_weights")), _ptr(o["recv_src_idx"]),
+        _ptr(o["rank_prefix_matrix"]), _ptr(o["recv_count"]),
+        _ptr(o.get("num_recv_tokens_per_expert")), _ptr(o["send_pos"]), _ptr(status),
+        _stream(stream))
+    _check(rc, "ep_dispatch_noalloc")
     return o
 
 

@@ -20,6 +20,7 @@
 //                         copies, S stages deep.  HBM-bound: R*T*H*2 bytes
 //                         read, N*H*2 bytes written (N = number of copies).
 #include <algorithm>
+#include <mutex>
 
 #include "ep_scan.cuh"
 
@@ -406,4 +407,71 @@ extern "C" EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
       static_cast<const uint8_t *>(x), send_pos, static_cast<uint8_t *>(recv_x), R, num_tok,
       row_bytes, chunk_bytes, nchunks, stage_stride, cap, status, wc.timeout_ns);
   return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// ep_dispatch_noalloc: ep_dispatch with its scratch in a static device array.
+//
+// Some callers cannot hand the library a workspace: a host program whose
+// device memory is owned by another allocator (a raw cudaMalloc next to that
+// pool fails or fragments it), or a latency-critical loop that cannot afford
+// cudaMalloc/cudaFree, which may synchronise the device.  For them this entry
+// point keeps the look-back scratch in a file-scope __device__ array of
+// kNoAllocScratchBytes, which every GPU that loads this library holds until
+// the process exits.  It allocates nothing and calls nothing that allocates.
+//
+// Set-up: the first call on a device (with that device current) looks up the
+// array's device address with cudaGetSymbolAddress and caches it; make that
+// first call before any stream capture.  The array is shared by every call on
+// a device and keeps the last call's contents; ep_dispatch clears the part it
+// uses on the stream before its kernels run, so calls on one stream are safe,
+// but calls that overlap on the GPU (other streams, other threads) race on it.
+// ---------------------------------------------------------------------------
+
+namespace ep {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 2u << 20;  // 2 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+void *g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device, or nullptr.
+void *noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return nullptr;
+    g_noalloc_ptr[dev] = p;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+}  // namespace ep
+
+extern "C" EP_API int ep_dispatch_noalloc(
+    const void *x, const int64_t *topk_idx, const float *topk_weights,
+    const uint8_t *is_token_in_rank, int num_ranks, int num_tokens, int hidden, int num_topk,
+    int num_experts, int expert_alignment, int capacity, void *recv_x, int64_t *recv_topk_idx,
+    float *recv_topk_weights, int32_t *recv_src_idx, int32_t *rank_prefix_matrix,
+    int32_t *recv_count, int32_t *num_recv_tokens_per_expert, int32_t *send_pos,
+    int32_t *status, cudaStream_t stream) {
+  using namespace ep;
+  if (num_ranks < 1 || num_tokens < 0 || num_experts < 0) return EP_ERR_INVALID_ARG;
+  const size_t need =
+      ep_dispatch_workspace_bytes(num_ranks, num_tokens, topk_idx != nullptr ? num_experts : 0);
+  if (need > kNoAllocScratchBytes) return EP_ERR_UNSUPPORTED;  // beyond the static scratch
+  void *scratch = noalloc_scratch();
+  if (scratch == nullptr) return EP_ERR_CUDA;
+  return ep_dispatch(x, topk_idx, topk_weights, is_token_in_rank, num_ranks, num_tokens, hidden,
+                     num_topk, num_experts, expert_alignment, capacity, recv_x, recv_topk_idx,
+                     recv_topk_weights, recv_src_idx, rank_prefix_matrix, recv_count,
+                     num_recv_tokens_per_expert, send_pos, scratch, kNoAllocScratchBytes,
+                     status, stream);
 }

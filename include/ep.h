@@ -163,6 +163,39 @@ EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
                        int32_t *status, cudaStream_t stream);
 
 /*
+ * ep_dispatch without a workspace argument.  The routing method has no
+ * counterpart of this call: it exists for callers that cannot allocate device
+ * memory when they call -- a host program whose device memory belongs to
+ * another allocator, or a latency-critical loop that cannot afford
+ * cudaMalloc/cudaFree (they can synchronise the device).
+ *
+ * Arguments, outputs and results are those of ep_dispatch.  The scratch lives
+ * in a 2 MiB static device array inside the library, held on every GPU that
+ * loads the library until the process exits; this call allocates nothing.
+ * Calls needing more than that (ep_dispatch_workspace_bytes(R, T, E) >
+ * 2 MiB, with E = 0 when topk_idx is NULL) return EP_ERR_UNSUPPORTED.
+ * The first call on a device, with that device current, looks up the array's
+ * device address (cudaGetSymbolAddress); make that first call before any
+ * stream capture.  Every call on a device shares the array and it keeps the
+ * last call's contents (the call clears what it uses on `stream` first): calls
+ * that overlap on the GPU, e.g. on two streams at once, race on it.
+ */
+EP_API int ep_dispatch_noalloc(const void *x, const int64_t *topk_idx,
+                               const float *topk_weights,
+                               const uint8_t *is_token_in_rank, int num_ranks,
+                               int num_tokens, int hidden, int num_topk,
+                               int num_experts, int expert_alignment,
+                               int capacity, void *recv_x,
+                               int64_t *recv_topk_idx,
+                               float *recv_topk_weights,
+                               int32_t *recv_src_idx,
+                               int32_t *rank_prefix_matrix,
+                               int32_t *recv_count,
+                               int32_t *num_recv_tokens_per_expert,
+                               int32_t *send_pos, int32_t *status,
+                               cudaStream_t stream);
+
+/*
  * A4: combine (gather-reduce).
  * Passage: Buffer.combine (DeepEP legacy-test analysis page, combine_args and
  * the check that (combined_x - bias) / is_token_in_rank.sum(1) equals x).
