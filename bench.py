@@ -270,28 +270,37 @@ def extra_configs(device, ep) -> dict:
     stream = torch.cuda.current_stream(device)
 
     def timeit(fn, iters=20, warm=3):
+        """Mean device time of fn(): `iters` calls captured in one CUDA graph
+        and replayed, so host launch overhead does not enter the number."""
         for _ in range(warm):
             fn()
+        torch.cuda.synchronize(device)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(iters):
+                fn()
+        g.replay()
         torch.cuda.synchronize(device)
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(iters):
-            fn()
+        g.replay()
         b.record(stream)
         b.synchronize()
+        del g
         return a.elapsed_time(b) / iters
 
     # layout only: [4096, 8] of 256 experts, 8 ranks
     w = CONFIGS["layout"]
     inp = make(w, with_x=False)
     idx = torch.from_numpy(inp["topk_idx"][0]).to(device)
-    o = {}
+    o = {"a": torch.empty((w.R,), dtype=torch.int32, device=device),
+         "b": torch.empty((w.E,), dtype=torch.int32, device=device),
+         "c": torch.empty((w.T, w.R), dtype=torch.bool, device=device)}
 
     def lay():
-        r = ep.ep_get_dispatch_layout(idx, w.E, w.R, num_tokens_per_rank=o.get("a"),
-                                      num_tokens_per_expert=o.get("b"), is_token_in_rank=o.get("c"))
-        o["a"], o["b"], o["c"] = r
+        ep.ep_get_dispatch_layout(idx, w.E, w.R, num_tokens_per_rank=o["a"],
+                                  num_tokens_per_expert=o["b"], is_token_in_rank=o["c"])
     ms = timeit(lay, iters=200, warm=10)
     out["layout_4096x8"] = {"us": ms * 1e3,
                             "gbs": layout_bytes(1, w.T, w.K, w.E, w.R) / (ms * 1e-3) / 1e9}
@@ -302,25 +311,25 @@ def extra_configs(device, ep) -> dict:
     x = to_dev_bf16(inp["x"], device)
     idx = torch.from_numpy(inp["topk_idx"]).to(device)
     wt = torch.from_numpy(inp["topk_weights"]).to(device)
-    buf = {}
-    lay_o = {}
+    a, b, c = ep.ep_get_dispatch_layout(idx, w.E, w.R)
+    d = ep.ep_dispatch(x, idx, wt, w.E, is_token_in_rank=c)
+    cx, cw = ep.ep_combine(d["recv_x"], d["send_pos"], d["recv_topk_weights"])
+    wsp = torch.empty(ep.ep_dispatch_workspace_bytes(w.R, w.T, w.E), dtype=torch.uint8,
+                      device=device)
+    buf = {"d": d}
 
     def sk():
-        a, b, c = ep.ep_get_dispatch_layout(idx, w.E, w.R, num_tokens_per_rank=lay_o.get("a"),
-                                            num_tokens_per_expert=lay_o.get("b"),
-                                            is_token_in_rank=lay_o.get("c"))
-        lay_o.update(a=a, b=b, c=c)
-        d = ep.ep_dispatch(x, idx, wt, w.E, is_token_in_rank=c, out=buf.get("d"))
-        buf["d"] = d
-        cx, cw = ep.ep_combine(d["recv_x"], d["send_pos"], d["recv_topk_weights"],
-                               combined_x=buf.get("cx"), combined_topk_weights=buf.get("cw"))
-        buf["cx"], buf["cw"] = cx, cw
+        ep.ep_get_dispatch_layout(idx, w.E, w.R, num_tokens_per_rank=a, num_tokens_per_expert=b,
+                                  is_token_in_rank=c)
+        ep.ep_dispatch(x, idx, wt, w.E, is_token_in_rank=c, out=d, workspace=wsp)
+        ep.ep_combine(d["recv_x"], d["send_pos"], d["recv_topk_weights"], combined_x=cx,
+                      combined_topk_weights=cw)
     ms = timeit(sk, iters=20)
     N = int(buf["d"]["recv_count"].sum().item())
     nb = dispatch_bytes(w.R, w.T, w.H, w.K, N) + combine_bytes(w.R, w.T, w.H, w.K, N)
     out["skewed"] = {"ms": ms, "gbs": nb / (ms * 1e-3) / 1e9, "copies": N,
                      "tokens_per_s": w.R * w.T / (ms * 1e-3)}
-    del x, idx, wt, buf, lay_o
+    del x, idx, wt, buf, d, cx, cw, a, b, c, wsp
     torch.cuda.empty_cache()
 
     # low latency: FP8 dispatch + weighted combine
@@ -376,7 +385,7 @@ def run_ours(args) -> None:
     import combine_get_dispatch_06_b200 as ep  # fails loudly without libep.so
 
     w = CONFIGS["normal"]
-    R, T, H, E, K = w.R, w.T, w.H, w.E, w.K
+    R, T, H, E, K = w.R, (args.tokens or w.T), w.H, w.E, w.K
     inp = make(Workload(w.name, R=R, T=T, H=H, E=E, K=K, seed=w.seed + rank))
     stream = torch.cuda.current_stream(device)
 
@@ -496,7 +505,7 @@ def run_ours(args) -> None:
         "metric": METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": agg["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "normal: R=8 simulated ranks x T=4096 tokens x H=7168 bf16, "
+        "config": {"workload": f"normal: R=8 simulated ranks x T={T} tokens x H=7168 bf16, "
                                "E=256 experts, top-8 distinct uniform, fp32 softmax weights, "
                                "identity experts",
                    "global_batch": R * T * ws, "seq_len": None,
@@ -515,9 +524,9 @@ def run_ours(args) -> None:
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
-    if ws == 1 and rank == 0 and not args.no_extra:
+    if ws == 1 and rank == 0 and not args.no_extra and T == CONFIGS["normal"].T:
         line["extra"] = extra_configs(device, ep)
-    if ws == 1 and rank == 0 and not args.no_cpu_baseline:
+    if ws == 1 and rank == 0 and not args.no_cpu_baseline and T == CONFIGS["normal"].T:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -533,6 +542,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="tokens per source rank (default 4096; smaller only for profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

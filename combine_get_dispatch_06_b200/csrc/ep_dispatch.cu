@@ -49,12 +49,59 @@ struct DispatchScanParams {
   unsigned flags;
 };
 
+// Received top-k metadata of one copy held by a rank whose experts are
+// [lo, hi): local id for local slots, -1 / 0.0 otherwise.  16-byte stores
+// when K allows them (rows of K int64 / K fp32 are then 16-byte aligned).
+__device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, size_t row, int K,
+                                           int64_t lo, int64_t hi, const int64_t (&ek)[kMaxTopk],
+                                           const float (&wk)[kMaxTopk]) {
+  if (recv_idx != nullptr) {
+    int64_t *dst = recv_idx + row * K;
+    if ((K & 1) == 0) {
+#pragma unroll
+      for (int k = 0; k < kMaxTopk; k += 2) {
+        if (k < K) {
+          longlong2 v;
+          v.x = (ek[k] >= lo && ek[k] < hi) ? ek[k] - lo : -1;
+          v.y = (ek[k + 1] >= lo && ek[k + 1] < hi) ? ek[k + 1] - lo : -1;
+          *reinterpret_cast<longlong2 *>(dst + k) = v;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < kMaxTopk; ++k)
+        if (k < K) dst[k] = (ek[k] >= lo && ek[k] < hi) ? ek[k] - lo : -1;
+    }
+  }
+  if (recv_w != nullptr) {
+    float *dst = recv_w + row * K;
+    if ((K & 3) == 0) {
+#pragma unroll
+      for (int k = 0; k < kMaxTopk; k += 4) {
+        if (k < K) {
+          float4 v;
+          v.x = (ek[k] >= lo && ek[k] < hi) ? wk[k] : 0.f;
+          v.y = (ek[k + 1] >= lo && ek[k + 1] < hi) ? wk[k + 1] : 0.f;
+          v.z = (ek[k + 2] >= lo && ek[k + 2] < hi) ? wk[k + 2] : 0.f;
+          v.w = (ek[k + 3] >= lo && ek[k + 3] < hi) ? wk[k + 3] : 0.f;
+          *reinterpret_cast<float4 *>(dst + k) = v;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < kMaxTopk; ++k)
+        if (k < K) dst[k] = (ek[k] >= lo && ek[k] < hi) ? wk[k] : 0.f;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanParams p) {
   __shared__ int s_tile;
   __shared__ int s_last;
   __shared__ uint32_t s_mask[kScanTile * kMaskWords];
   __shared__ int s_woff[kScanWarps][kMaxRanks];
   __shared__ int s_excl[kMaxRanks];
+  __shared__ int s_agg[kMaxRanks];
   __shared__ int s_ehist[kMaxExperts];
 
   const int tid = threadIdx.x;
@@ -114,9 +161,7 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   }
   __syncthreads();
 
-  // ---- tile totals, look-back, rank prefix matrix -----------------------
-  const bool publish = (p.flags & EP_DEBUG_SUPPRESS_PUBLISH) == 0;
-  const bool last_of_src = (tile % p.tiles_per_src) == p.tiles_per_src - 1;
+  // ---- tile totals -------------------------------------------------------
   for (int d = tid; d < p.R; d += kScanTile) {
     int run = 0;
 #pragma unroll
@@ -125,18 +170,45 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
       s_woff[w][d] = run;
       run += c;
     }
-    const uint32_t excl =
-        lookback_column(p.desc, tile, p.R, d, static_cast<uint32_t>(run), publish, p.timeout_ns,
-                        p.status);
-    s_excl[d] = static_cast<int>(excl);
-    if (last_of_src) {
-      p.P[static_cast<size_t>(s) * p.R + d] = static_cast<int>(excl) + run;
-      if (tile == p.num_tiles - 1) p.recv_count[d] = static_cast<int>(excl) + run;
+    s_agg[d] = run;
+  }
+  __syncthreads();
+
+  // ---- look-back (a group of 16 lanes per rank column), prefix matrix ----
+  const bool publish = (p.flags & EP_DEBUG_SUPPRESS_PUBLISH) == 0;
+  const bool last_of_src = (tile % p.tiles_per_src) == p.tiles_per_src - 1;
+  {
+    constexpr int G = 16;
+    const int grp = tid / G;
+    for (int d = grp; d < p.R; d += kScanTile / G) {
+      const int run = s_agg[d];
+      const uint32_t excl = lookback_window<G, 4>(p.desc, tile, p.R, d, static_cast<uint32_t>(run),
+                                                  publish, p.timeout_ns, p.status);
+      if ((tid & (G - 1)) == 0) {
+        s_excl[d] = static_cast<int>(excl);
+        if (last_of_src) {
+          p.P[static_cast<size_t>(s) * p.R + d] = static_cast<int>(excl) + run;
+          if (tile == p.num_tiles - 1) p.recv_count[d] = static_cast<int>(excl) + run;
+        }
+      }
     }
   }
   __syncthreads();
 
   // ---- pass 2: positions, handle and received metadata -------------------
+  const bool meta =
+      valid && p.topk_idx != nullptr && (p.recv_idx != nullptr || p.recv_w != nullptr);
+  int64_t ek[kMaxTopk];
+  float wk[kMaxTopk];
+#pragma unroll
+  for (int k = 0; k < kMaxTopk; ++k) {
+    ek[k] = -1;
+    wk[k] = 0.f;
+    if (meta && k < p.K) {
+      ek[k] = p.topk_idx[st * p.K + k];
+      if (p.recv_w != nullptr) wk[k] = p.topk_w[st * p.K + k];
+    }
+  }
   const uint32_t lt = lanemask_lt();
   bool overflow = false;
   for (int d0 = 0; d0 < p.R; d0 += 32) {
@@ -156,16 +228,8 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
       }
       const size_t row = static_cast<size_t>(d) * p.cap + pos;
       p.recv_src_idx[row] = t;
-      if (p.topk_idx != nullptr && (p.recv_idx != nullptr || p.recv_w != nullptr)) {
-        const int64_t *irow = p.topk_idx + st * p.K;
-        for (int k = 0; k < p.K; ++k) {
-          const int64_t e = irow[k];
-          const bool local = e >= 0 && e < p.E && static_cast<int>(e) / p.El == d;
-          if (p.recv_idx != nullptr)
-            p.recv_idx[row * p.K + k] = local ? e - static_cast<int64_t>(d) * p.El : -1;
-          if (p.recv_w != nullptr) p.recv_w[row * p.K + k] = local ? p.topk_w[st * p.K + k] : 0.0f;
-        }
-      }
+      if (meta) write_meta(p.recv_idx, p.recv_w, row, p.K, static_cast<int64_t>(d) * p.El,
+                           static_cast<int64_t>(d + 1) * p.El, ek, wk);
     }
   }
   if (overflow) report(p.status, EP_STATUS_CAPACITY);
@@ -194,8 +258,12 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
 // own bulk stores from that stage have finished reading shared memory.
 // ---------------------------------------------------------------------------
 
+// Launch shape, chosen by a sweep on B200 at R=8, H=7168 (stages x chunk x
+// CTAs per SM): the row scatter is fastest with ~28 KB in flight per SM;
+// deeper pipelines oversubscribe HBM with this write-heavy mix and lose 5-7%.
 constexpr int kCopyStages = 4;
-constexpr int kCopyChunkMax = 16384;
+constexpr int kCopyChunkMax = 4096;
+constexpr int kCopyMaxCtasPerSm = 2;
 
 template <int S>
 __global__ void __launch_bounds__(kMaxRanks)
@@ -228,8 +296,8 @@ __global__ void __launch_bounds__(kMaxRanks)
     const int off = static_cast<int>(i % nchunks) * chunk_bytes;
     const int nb = min(chunk_bytes, row_bytes - off);
     mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(nb));
-    bulk_g2s(buf + stg * stage_stride, x + u * row_bytes + off, static_cast<uint32_t>(nb),
-             &bars[stg]);
+    bulk_g2s_hint(buf + stg * stage_stride, x + u * row_bytes + off, static_cast<uint32_t>(nb),
+                  &bars[stg], l2_evict_first_policy());
   };
   auto load_pos = [&](long i) -> int {
     return d < R ? __ldg(send_pos + token_of(i) * R + d) : -1;
@@ -401,8 +469,9 @@ extern "C" EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
   const void *fn = reinterpret_cast<const void *>(dispatch_copy_kernel<kCopyStages>);
   if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
   const long num_tok = static_cast<long>(R) * T;
-  const long grid = std::min<long>(num_tok, static_cast<long>(ctas_per_sm(fn, threads, smem)) *
-                                                num_sms());
+  const long grid = std::min<long>(
+      num_tok,
+      static_cast<long>(std::min(kCopyMaxCtasPerSm, ctas_per_sm(fn, threads, smem))) * num_sms());
   dispatch_copy_kernel<kCopyStages><<<static_cast<unsigned>(grid), threads, smem, stream>>>(
       static_cast<const uint8_t *>(x), send_pos, static_cast<uint8_t *>(recv_x), R, num_tok,
       row_bytes, chunk_bytes, nchunks, stage_stride, cap, status, wc.timeout_ns);

@@ -45,7 +45,7 @@ struct LLScanParams {
 
 __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   __shared__ int s_tile;
-  __shared__ int s_last;
+  __shared__ uint32_t s_lanes[kScanWarps][kMaxExperts];  // lanes of the warp holding expert c
   __shared__ int s_whist[kScanWarps][kMaxExperts];
   __shared__ int s_excl[kMaxExperts];
 
@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   const int lane = tid & 31;
   const int warp = tid >> 5;
   if (tid == 0) s_tile = static_cast<int>(atomicAdd(&p.head->ticket, 1u));
-  for (int i = tid; i < kScanWarps * kMaxExperts; i += kScanTile) (&s_whist[0][0])[i] = 0;
+  for (int i = tid; i < kScanWarps * kMaxExperts; i += kScanTile) (&s_lanes[0][0])[i] = 0u;
   __syncthreads();
 
   const int tile = s_tile;
@@ -65,7 +65,6 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   // Distinct valid experts of this token (a repeated expert keeps only its
   // first slot in `col`; `ev` keeps every valid id).
   int ev[kMaxTopk], col[kMaxTopk], rnk[kMaxTopk];
-  uint32_t pending = 0;
   bool bad = false;
 #pragma unroll
   for (int k = 0; k < kMaxTopk; ++k) {
@@ -79,10 +78,7 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
         bool dup = false;
 #pragma unroll
         for (int k2 = 0; k2 < k; ++k2) dup |= (col[k2] == ev[k]);
-        if (!dup) {
-          col[k] = ev[k];
-          pending |= 1u << k;
-        }
+        if (!dup) col[k] = ev[k];
       } else if (e != -1) {
         bad = true;
       }
@@ -90,35 +86,26 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   }
   if (bad) report(p.status, EP_STATUS_BAD_EXPERT);
 
-  // Rank of each (token, expert) among the warp's tokens that hold that
-  // expert: one ballot per distinct expert present in the warp.
-  const uint32_t lt = lanemask_lt();
-  while (true) {
-    const uint32_t any = __ballot_sync(0xffffffffu, pending != 0u);
-    if (any == 0u) break;
-    const int leader = __ffs(any) - 1;
-    int mine = -1;
-    if (pending != 0u) {
-      const int kf = __ffs(pending) - 1;
+  // For every expert, the set of the warp's lanes (tokens) that hold it:
+  // slot by slot, lanes with the same expert find each other with match.any
+  // and their lowest lane ORs the group into the expert's word.  A token's
+  // rank among the warp's tokens with that expert is then the number of
+  // lower lanes in the word -- token order, whatever slot the expert is in.
 #pragma unroll
-      for (int k = 0; k < kMaxTopk; ++k)
-        if (k == kf) mine = col[k];
+  for (int k = 0; k < kMaxTopk; ++k) {
+    if (k < p.K) {
+      const uint32_t peers = __match_any_sync(0xffffffffu, col[k]);
+      if (col[k] >= 0 && lane == __ffs(peers) - 1) s_lanes[warp][col[k]] |= peers;
+      __syncwarp();
     }
-    const int c = __shfl_sync(0xffffffffu, mine, leader);
-    int kk = -1;
-#pragma unroll
-    for (int k = 0; k < kMaxTopk; ++k)
-      if (col[k] == c && ((pending >> k) & 1u)) kk = k;
-    const uint32_t bal = __ballot_sync(0xffffffffu, kk >= 0);
-    if (kk >= 0) {
-      const int r = __popc(bal & lt);
-#pragma unroll
-      for (int k = 0; k < kMaxTopk; ++k)
-        if (k == kk) rnk[k] = r;
-      pending &= ~(1u << kk);
-    }
-    if (lane == 0) s_whist[warp][c] = __popc(bal);
   }
+  const uint32_t lt = lanemask_lt();
+#pragma unroll
+  for (int k = 0; k < kMaxTopk; ++k)
+    if (col[k] >= 0) rnk[k] = __popc(s_lanes[warp][col[k]] & lt);
+  for (int c = tid; c < p.E; c += kScanTile)
+#pragma unroll
+    for (int w = 0; w < kScanWarps; ++w) s_whist[w][c] = __popc(s_lanes[w][c]);
   __syncthreads();
 
   const bool publish = (p.flags & EP_DEBUG_SUPPRESS_PUBLISH) == 0;
@@ -131,10 +118,13 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
       s_whist[w][c] = run;
       run += n;
     }
-    const uint32_t excl = lookback_column(p.desc, tile, p.E, c, static_cast<uint32_t>(run),
-                                          publish, p.timeout_ns, p.status);
+    const uint32_t excl = lookback_window<1, 16>(p.desc, tile, p.E, c, static_cast<uint32_t>(run),
+                                                 publish, p.timeout_ns, p.status);
     s_excl[c] = static_cast<int>(excl);
-    if (first_of_src) p.layout_range[(static_cast<size_t>(c) * p.R + s) * 2] = static_cast<int>(excl);
+    const size_t o = (static_cast<size_t>(c) * p.R + s) * 2;
+    if (first_of_src) p.layout_range[o] = static_cast<int>(excl);
+    // rows source s owns: the tiles of s add their counts (zeroed on the host)
+    if (run != 0) atomicAdd(&p.layout_range[o + 1], run);
     if (tile == p.num_tiles - 1) p.recv_count[c] = static_cast<int>(excl) + run;
   }
   __syncthreads();
@@ -170,23 +160,13 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
     if (oob) report(p.status, EP_STATUS_BAD_POSITION);
   }
 
-  if (elect_last_cta(&p.head->done, static_cast<uint32_t>(p.num_tiles), &s_last)) {
-    // rows per (expert, source rank) = next source's first row - this one's
-    const int n = p.E * p.R;
-    for (int i = tid; i < n; i += kScanTile) {
-      const int c = i / p.R;
-      const int s2 = i % p.R;
-      const size_t o = (static_cast<size_t>(c) * p.R + s2) * 2;
-      const int begin = __ldcg(&p.layout_range[o]);
-      const int end = (s2 + 1 < p.R) ? __ldcg(&p.layout_range[o + 2]) : __ldcg(&p.recv_count[c]);
-      p.layout_range[o + 1] = end - begin;
-    }
-  }
 }
 
 // ---------------------------------------------------------------------------
 
-constexpr int kLLWarps = 4;
+constexpr int kLLThreads = 256;  // 8 warps quantise one token row together
+constexpr int kLLInStages = 3;
+constexpr int kLLMaxCtasPerSm = 3;
 
 __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float d) {
   // element order in memory: a, b, c, d (a in the lowest byte)
@@ -196,31 +176,79 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float 
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
+// Shared-memory plan of one CTA: 128 bytes of mbarriers, kLLInStages input
+// rows (bf16, filled by bulk copies), then (FP8 only) two e4m3 output rows
+// with their scales, used alternately by consecutive tokens.
+struct LLSmem {
+  int in_stride;   // bytes per input stage (multiple of 128)
+  int out_stride;  // bytes per output buffer (e4m3 row + scales, multiple of 128)
+  int sc_off;      // offset of the scales inside an output buffer
+  int bytes;       // total
+};
+
+__host__ __device__ inline LLSmem ll_smem_plan(int H, bool fp8) {
+  LLSmem m;
+  m.in_stride = (2 * H + 127) & ~127;
+  m.sc_off = (H + 127) & ~127;
+  m.out_stride = fp8 ? m.sc_off + (((H / 128) * 4 + 127) & ~127) : 0;
+  m.bytes = 128 + kLLInStages * m.in_stride + 2 * m.out_stride;
+  return m;
+}
+
+// One CTA per token at a time, tokens strided over the grid.  Thread 0 keeps
+// kLLInStages bulk loads of upcoming rows in flight; all 256 threads quantise
+// the current row (16 consecutive threads per 128-channel block, amax by
+// xor-shuffles); then warp 0's lanes, one per distinct expert of the token,
+// send the e4m3 row and its scales with bulk shared->global stores.
 template <bool kFP8>
-__global__ void __launch_bounds__(kLLWarps * 32)
+__global__ void __launch_bounds__(kLLThreads)
     ll_dispatch_kernel(const uint8_t *__restrict__ x, const int64_t *__restrict__ topk_idx,
                        const int32_t *__restrict__ ll_pos, long num_tok, int H, int K, int E,
-                       int cap, int buf_stride, int pay_bytes, int sc_bytes, int sc_off,
-                       uint8_t *__restrict__ recv, float *__restrict__ scales,
-                       int32_t *status) {
+                       int cap, LLSmem plan, uint8_t *__restrict__ recv,
+                       float *__restrict__ scales, int32_t *status,
+                       unsigned long long timeout_ns) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  uint8_t *wbuf = smem + static_cast<size_t>(warp) * 2 * buf_stride;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+  uint8_t *inb = smem + 128;
+  uint8_t *outb = inb + kLLInStages * plan.in_stride;
   const int nvec = H >> 3;
   const int nblk = H >> 7;
+  const int row_in = 2 * H;
+  const int pay = kFP8 ? H : 2 * H;
+  const int sc_bytes = nblk * 4;
   const bool bulk_scales = (sc_bytes & 15) == 0;
-  int it = 0;
-  for (long u = static_cast<long>(blockIdx.x) * kLLWarps + warp; u < num_tok;
-       u += static_cast<long>(gridDim.x) * kLLWarps, ++it) {
-    uint8_t *b = wbuf + (it & 1) * buf_stride;
-    // the buffer was last used two tokens ago: its stores must have read it
-    bulk_wait_read<1>();
-    __syncwarp();
+  const long n = static_cast<long>(blockIdx.x) < num_tok
+                     ? (num_tok - 1 - blockIdx.x) / gridDim.x + 1
+                     : 0;
 
-    // destination of slot `lane`: one row per distinct expert
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < kLLInStages; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](long i) {  // thread 0
+    const int stg = static_cast<int>(i % kLLInStages);
+    const long u = static_cast<long>(blockIdx.x) + i * gridDim.x;
+    mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(row_in));
+    bulk_g2s_hint(inb + stg * plan.in_stride, x + u * row_in, static_cast<uint32_t>(row_in),
+                  &bars[stg], l2_evict_first_policy());
+  };
+  if (tid == 0)
+    for (long i = 0; i < kLLInStages && i < n; ++i) issue(i);
+
+  bool all_ok = true;
+  long stop = n;
+  for (long i = 0; i < n; ++i) {
+    const int stg = static_cast<int>(i % kLLInStages);
+    const long u = static_cast<long>(blockIdx.x) + i * gridDim.x;
+    uint8_t *in = inb + stg * plan.in_stride;
+
+    // destination of slot `lane` (warp 0): one row per distinct expert
     long dst = -1;
-    {
+    if (tid < 32) {
       int e = -1, pos = -1;
       if (lane < K) {
         const int64_t ee = topk_idx[u * K + lane];
@@ -240,75 +268,110 @@ __global__ void __launch_bounds__(kLLWarps * 32)
         else
           report(status, EP_STATUS_BAD_POSITION);
       }
+      // FP8: the output buffer of token i - 2 must have been read by its stores
+      if (kFP8) bulk_wait_read<1>();
+    }
+    const bool ok =
+        mbar_wait_bounded(&bars[stg], static_cast<uint32_t>((i / kLLInStages) & 1), timeout_ns);
+    if (__syncthreads_and(ok) == 0) {
+      all_ok = false;
+      stop = i;
+      break;
     }
 
-    const uint8_t *xr = x + u * static_cast<long>(H) * 2;
-    for (int c0 = 0; c0 < nvec; c0 += 32) {
-      const int c = c0 + lane;
-      const bool act = c < nvec;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (act) v = __ldg(reinterpret_cast<const uint4 *>(xr) + c);
-      if constexpr (kFP8) {
+    const uint8_t *src = in;
+    float *sc = nullptr;
+    if constexpr (kFP8) {
+      uint8_t *q = outb + static_cast<int>(i & 1) * plan.out_stride;
+      sc = reinterpret_cast<float *>(q + plan.sc_off);
+#pragma unroll 2
+      for (int c0 = 0; c0 < nvec; c0 += kLLThreads) {
+        const int c = c0 + tid;
+        const bool act = c < nvec;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (act) v = reinterpret_cast<const uint4 *>(in)[c];
         float f[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
                       bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
         float amax = 0.f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
-        // 16 lanes hold one 128-channel block (nvec is a multiple of 16)
+        // 16 consecutive threads hold one 128-channel block (nvec % 16 == 0)
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         amax = fmaxf(amax, 1e-4f);
         const float inv = __fdiv_rn(448.0f, amax);
         if (act) {
-          uint2 q;
-          q.x = cvt_e4m3x4(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv), __fmul_rn(f[2], inv),
-                           __fmul_rn(f[3], inv));
-          q.y = cvt_e4m3x4(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv), __fmul_rn(f[6], inv),
-                           __fmul_rn(f[7], inv));
-          *reinterpret_cast<uint2 *>(b + static_cast<size_t>(c) * 8) = q;
-          if ((lane & 15) == 0)
-            reinterpret_cast<float *>(b + sc_off)[c >> 4] = __fdiv_rn(amax, 448.0f);
-        }
-      } else {
-        if (act) *reinterpret_cast<uint4 *>(b + static_cast<size_t>(c) * 16) = v;
-      }
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (dst >= 0) {
-      bulk_s2g(recv + dst * pay_bytes, b, static_cast<uint32_t>(pay_bytes));
-      if constexpr (kFP8) {
-        if (bulk_scales) {
-          bulk_s2g(scales + dst * nblk, b + sc_off, static_cast<uint32_t>(sc_bytes));
-        } else {
-          const float *sb = reinterpret_cast<const float *>(b + sc_off);
-          for (int j = 0; j < nblk; ++j) scales[dst * nblk + j] = sb[j];
+          uint2 qq;
+          qq.x = cvt_e4m3x4(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv), __fmul_rn(f[2], inv),
+                            __fmul_rn(f[3], inv));
+          qq.y = cvt_e4m3x4(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv), __fmul_rn(f[6], inv),
+                            __fmul_rn(f[7], inv));
+          reinterpret_cast<uint2 *>(q)[c] = qq;
+          if ((c & 15) == 0) sc[c >> 4] = __fdiv_rn(amax, 448.0f);
         }
       }
+      fence_proxy_async_smem();
+      __syncthreads();
+      src = q;
     }
-    bulk_commit();
+    if (tid < 32) {
+      if (dst >= 0) {
+        bulk_s2g(recv + dst * pay, src, static_cast<uint32_t>(pay));
+        if constexpr (kFP8) {
+          if (bulk_scales)
+            bulk_s2g(scales + dst * nblk, sc, static_cast<uint32_t>(sc_bytes));
+          else
+            for (int j = 0; j < nblk; ++j) scales[dst * nblk + j] = sc[j];
+        }
+      }
+      bulk_commit();
+      if (!kFP8) bulk_wait_read<0>();  // bf16 forwards straight from `in`
+    }
+    if (!kFP8) __syncthreads();
+    // `in` is free: quantised (FP8) or read by the stores (bf16)
+    if (tid == 0 && i + kLLInStages < n) {
+      fence_proxy_async_smem();
+      issue(i + kLLInStages);
+    }
   }
-  bulk_wait_all<0>();
+  if (tid < 32) bulk_wait_all<0>();
+  if (!all_ok) {
+    report(status, EP_STATUS_WAIT_TIMEOUT);
+    if (tid == 0) {
+      const long end = min(n, stop + kLLInStages);
+      for (long k = stop; k < end; ++k)
+        (void)mbar_wait_bounded(&bars[k % kLLInStages],
+                                static_cast<uint32_t>((k / kLLInStages) & 1), timeout_ns);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
 
 constexpr int kLLCombineWarps = 8;
 
+// One warp per (token, channel segment): the token's up-to-K slab rows are
+// listed in slot order, then each lane accumulates 16-byte chunks of the
+// segment with fmaf in that order.  Splitting rows into `nseg` segments gives
+// enough work items to keep every warp busy to the end.
 __global__ void __launch_bounds__(kLLCombineWarps * 32)
     ll_combine_kernel(const uint8_t *__restrict__ y, const int64_t *__restrict__ topk_idx,
                       const float *__restrict__ topk_w, const int32_t *__restrict__ ll_pos,
-                      long num_tok, int H, int K, int E, int cap, uint8_t *__restrict__ out,
-                      int32_t *status) {
+                      long num_tok, int H, int K, int E, int cap, int nseg,
+                      uint8_t *__restrict__ out, int32_t *status) {
   __shared__ int64_t s_row[kLLCombineWarps][kMaxTopk];
   __shared__ float s_w[kLLCombineWarps][kMaxTopk];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const uint32_t lt = lanemask_lt();
   const int nvec = H >> 3;
+  const int seg_vec = (nvec + nseg - 1) / nseg;
   const long row_bytes = static_cast<long>(H) * 2;
-  for (long u = static_cast<long>(blockIdx.x) * kLLCombineWarps + warp; u < num_tok;
-       u += static_cast<long>(gridDim.x) * kLLCombineWarps) {
+  const long items = num_tok * nseg;
+  for (long it = static_cast<long>(blockIdx.x) * kLLCombineWarps + warp; it < items;
+       it += static_cast<long>(gridDim.x) * kLLCombineWarps) {
+    const long u = it / nseg;
+    const int sg = static_cast<int>(it % nseg);
     bool take = false;
     long row = 0;
     float w = 0.f;
@@ -320,7 +383,7 @@ __global__ void __launch_bounds__(kLLCombineWarps * 32)
           take = true;
           row = e * cap + pos;
           w = topk_w[u * K + lane];
-        } else {
+        } else if (sg == 0) {
           report(status, EP_STATUS_BAD_POSITION);
         }
       }
@@ -335,7 +398,8 @@ __global__ void __launch_bounds__(kLLCombineWarps * 32)
     __syncwarp();
 
     uint8_t *orow = out + u * row_bytes;
-    for (int c = lane; c < nvec; c += 32) {
+    const int c_end = min(nvec, (sg + 1) * seg_vec);
+    for (int c = sg * seg_vec + lane; c < c_end; c += 32) {
       float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       for (int i = 0; i < n; i += 8) {
         uint4 v[8];
@@ -390,7 +454,6 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx, int
   if (R < 1 || R > kMaxRanks || T < 0 || K < 1 || K > kMaxTopk || E < 1 || E > kMaxExperts ||
       E % R != 0 || H < 8 || (use_fp8 ? (H % 128 != 0) : (H % 8 != 0)))
     return EP_ERR_INVALID_ARG;
-  if (H > 65536) return EP_ERR_UNSUPPORTED;
   if (recv_count == nullptr || layout_range == nullptr) return EP_ERR_INVALID_ARG;
   if (T == 0) {
     if (cudaMemsetAsync(recv_count, 0, sizeof(int32_t) * E, stream) != cudaSuccess ||
@@ -413,7 +476,10 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx, int
   const int tiles_per_src = (T + kScanTile - 1) / kScanTile;
   const long num_tiles = static_cast<long>(R) * tiles_per_src;
   if (cap > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
-  if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return EP_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess ||
+      cudaMemsetAsync(layout_range, 0, sizeof(int32_t) * 2 * static_cast<size_t>(E) * R,
+                      stream) != cudaSuccess)
+    return EP_ERR_CUDA;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   LLScanParams p;
@@ -438,29 +504,27 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx, int
   ll_scan_kernel<<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
   if (launch_status() != EP_OK) return EP_ERR_CUDA;
 
-  const int pay = use_fp8 ? H : 2 * H;
-  const int sc_bytes = use_fp8 ? (H / 128) * 4 : 0;
-  const int sc_off = (pay + 127) & ~127;
-  const int buf_stride = sc_off + ((sc_bytes + 127) & ~127);
-  const size_t smem = static_cast<size_t>(kLLWarps) * 2 * buf_stride;
-  const int threads = kLLWarps * 32;
+  const LLSmem plan = ll_smem_plan(H, use_fp8 != 0);
+  const size_t smem = static_cast<size_t>(plan.bytes);
+  if (smem > 227 * 1024) return EP_ERR_UNSUPPORTED;
   const long num_tok = static_cast<long>(R) * T;
   const void *fn = use_fp8 ? reinterpret_cast<const void *>(ll_dispatch_kernel<true>)
                            : reinterpret_cast<const void *>(ll_dispatch_kernel<false>);
   if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
-  const long want = (num_tok + kLLWarps - 1) / kLLWarps;
-  const long grid =
-      std::min<long>(want, static_cast<long>(ctas_per_sm(fn, threads, smem)) * num_sms());
+  const long grid = std::min<long>(
+      num_tok,
+      static_cast<long>(std::min(kLLMaxCtasPerSm, ctas_per_sm(fn, kLLThreads, smem))) *
+          num_sms());
   if (use_fp8)
-    ll_dispatch_kernel<true><<<static_cast<unsigned>(grid), threads, smem, stream>>>(
+    ll_dispatch_kernel<true><<<static_cast<unsigned>(grid), kLLThreads, smem, stream>>>(
         static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, H, K, E,
-        static_cast<int>(cap), buf_stride, pay, sc_bytes, sc_off,
-        static_cast<uint8_t *>(recv_x), recv_scales, status);
+        static_cast<int>(cap), plan, static_cast<uint8_t *>(recv_x), recv_scales, status,
+        wc.timeout_ns);
   else
-    ll_dispatch_kernel<false><<<static_cast<unsigned>(grid), threads, smem, stream>>>(
+    ll_dispatch_kernel<false><<<static_cast<unsigned>(grid), kLLThreads, smem, stream>>>(
         static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, H, K, E,
-        static_cast<int>(cap), buf_stride, pay, sc_bytes, sc_off,
-        static_cast<uint8_t *>(recv_x), nullptr, status);
+        static_cast<int>(cap), plan, static_cast<uint8_t *>(recv_x), nullptr, status,
+        wc.timeout_ns);
   return launch_status();
 }
 
@@ -485,10 +549,15 @@ extern "C" EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
   const long num_tok = static_cast<long>(R) * T;
   const int threads = kLLCombineWarps * 32;
   const void *fn = reinterpret_cast<const void *>(ll_combine_kernel);
-  const long want = (num_tok + kLLCombineWarps - 1) / kLLCombineWarps;
-  const long grid = std::min<long>(want, static_cast<long>(ctas_per_sm(fn, threads, 0)) * num_sms());
+  const long resident = static_cast<long>(ctas_per_sm(fn, threads, 0)) * num_sms();
+  // split rows into segments until there are >= 4 work items per resident warp
+  const int nvec = H / 8;
+  int nseg = static_cast<int>((4 * resident * kLLCombineWarps + num_tok - 1) / num_tok);
+  nseg = std::max(1, std::min(nseg, std::max(1, nvec / 32)));
+  const long items = num_tok * nseg;
+  const long grid = std::min<long>((items + kLLCombineWarps - 1) / kLLCombineWarps, resident);
   ll_combine_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(
       static_cast<const uint8_t *>(y), topk_idx, topk_weights, ll_pos, num_tok, H, K, E,
-      static_cast<int>(cap), static_cast<uint8_t *>(out), status);
+      static_cast<int>(cap), nseg, static_cast<uint8_t *>(out), status);
   return launch_status();
 }

@@ -34,43 +34,86 @@ __host__ __device__ inline size_t scan_workspace_bytes(long num_tiles, int colum
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
-// Returns the exclusive prefix of column `c` before tile `tile`, and publishes
-// the tile's inclusive prefix (unless `publish` is false, a debug mode).
-__device__ __forceinline__ uint32_t lookback_column(uint64_t *desc, int tile, int columns, int c,
+// Windowed look-back for column `c` of tile `tile`, run by an aligned group of
+// G lanes (G a power of two <= 32; all G lanes call it with the same
+// arguments).  Each round the group reads a window of G*U predecessor
+// descriptors at once (lane l, slot u -> tile - 1 - (l + G*u)), finds the
+// nearest inclusive prefix in it, and adds every value up to that one; if
+// the window holds none, it adds all of them and moves on.  A descriptor that
+// is not yet published makes the group re-read the window, at most
+// `timeout_ns` in total.  Returns the exclusive prefix to every lane of the
+// group and publishes the tile's inclusive prefix (lane 0 of the group).
+template <int G, int U>
+__device__ __forceinline__ uint32_t lookback_window(uint64_t *desc, int tile, int columns, int c,
                                                     uint32_t agg, bool publish,
                                                     unsigned long long timeout_ns,
                                                     int32_t *status) {
+  static_assert(G >= 1 && G <= 32 && (G & (G - 1)) == 0, "G must be a power of two");
+  constexpr int W = G * U;
+  const int lane = threadIdx.x & 31;
+  const int gl = lane & (G - 1);
+  const int gbase = lane & ~(G - 1);
+  const uint32_t gmask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << gbase);
   uint64_t *mine = desc + static_cast<size_t>(tile) * columns + c;
   if (tile == 0) {
-    if (publish) st_relaxed_gpu(mine, (2ull << 32) | agg);
+    if (publish && gl == 0) st_relaxed_gpu(mine, (2ull << 32) | agg);
     return 0u;
   }
-  if (publish) st_relaxed_gpu(mine, (1ull << 32) | agg);
+  if (publish && gl == 0) st_relaxed_gpu(mine, (1ull << 32) | agg);
+
   uint32_t excl = 0;
-  for (int j = tile - 1; j >= 0; --j) {
-    const uint64_t *p = desc + static_cast<size_t>(j) * columns + c;
-    uint64_t w = ld_relaxed_gpu(p);
-    if ((w >> 32) == 0) {
-      const uint64_t t0 = globaltimer();
-      bool ok = false;
-      while (true) {
-        __nanosleep(100);
-        w = ld_relaxed_gpu(p);
-        if ((w >> 32) != 0) {
-          ok = true;
-          break;
-        }
-        if (globaltimer() - t0 > timeout_ns) break;
-      }
-      if (!ok) {
-        report(status, EP_STATUS_WAIT_TIMEOUT);
-        break;
+  int base = tile - 1;
+  uint64_t t0 = 0;
+  bool timed_out = false;
+  while (true) {
+    uint32_t flag[U], val[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = base - (gl + G * u);
+      if (j >= 0) {
+        const uint64_t w = ld_relaxed_gpu(desc + static_cast<size_t>(j) * columns + c);
+        flag[u] = static_cast<uint32_t>(w >> 32);
+        val[u] = static_cast<uint32_t>(w);
+      } else {  // before tile 0: an inclusive prefix of 0
+        flag[u] = 2u;
+        val[u] = 0u;
       }
     }
-    excl += static_cast<uint32_t>(w);
-    if ((w >> 32) == 2) break;
+    // nearest inclusive prefix in the window (position gl + G*u)
+    int pstar = W;
+#pragma unroll
+    for (int u = U - 1; u >= 0; --u)
+      if (flag[u] == 2u) pstar = gl + G * u;
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) pstar = min(pstar, __shfl_xor_sync(gmask, pstar, o));
+    bool missing = false;
+    uint32_t sum = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int pos = gl + G * u;
+      if (pos <= pstar) {
+        missing |= (flag[u] == 0u);
+        sum += val[u];
+      }
+    }
+    if (__ballot_sync(gmask, missing) & gmask) {
+      const uint64_t now = __shfl_sync(gmask, globaltimer(), gbase);
+      if (t0 == 0) t0 = now;
+      if (now - t0 > timeout_ns) {
+        timed_out = true;
+        break;
+      }
+      __nanosleep(64);
+      continue;
+    }
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) sum += __shfl_xor_sync(gmask, sum, o);
+    excl += sum;
+    if (pstar < W) break;
+    base -= W;
   }
-  if (publish) st_relaxed_gpu(mine, (2ull << 32) | (excl + agg));
+  if (timed_out && gl == 0) report(status, EP_STATUS_WAIT_TIMEOUT);
+  if (publish && gl == 0) st_relaxed_gpu(mine, (2ull << 32) | (excl + agg));
   return excl;
 }
 
