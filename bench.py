@@ -256,6 +256,38 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def kernel_source_hash() -> str:
+    """sha1 of the CUDA sources, to tell whether recorded counters still apply."""
+    import glob
+    import hashlib
+
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "combine_get_dispatch_06_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, T: int):
+    """DRAM bytes (read + write) per launch of `kernel` on the normal workload,
+    from the ncu capture summarised in profiles/dram_traffic_normal.md -- or
+    None if that capture is of another build of the kernels."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic_normal.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    import re
+
+    m = re.search(r"source_sha1:\s*([0-9a-f]{40})", text)
+    if not m or m.group(1) != kernel_source_hash() or T != CONFIGS["normal"].T:
+        return None
+    m = re.search(rf"{kernel}\s*\|\s*traffic_bytes_per_launch\s*\|\s*(\d+)", text)
+    return int(m.group(1)) if m else None
+
+
 def to_dev_bf16(a: np.ndarray, device):
     import torch
 
@@ -417,20 +449,25 @@ def run_ours(args) -> None:
     status = ep.new_status(device)
 
     def step(ev=None):
+        # ep_dispatch == ep_notify_dispatch + ep_dispatch_cached; the two halves
+        # are called separately so that the row-copy kernel gets its own events
         if ev is not None:
             ev[0].record(stream)
         ep.ep_get_dispatch_layout(idx, E, R, num_tokens_per_rank=ntpr, num_tokens_per_expert=ntpe,
                                   is_token_in_rank=inr, status=status)
         if ev is not None:
             ev[1].record(stream)
-        ep.ep_dispatch(x, idx, wt, E, is_token_in_rank=inr, out=out, workspace=wsp,
-                       status=status)
+        ep.ep_notify_dispatch(idx, wt, T, R, E, is_token_in_rank=inr, out=out, workspace=wsp,
+                              status=status)
         if ev is not None:
             ev[2].record(stream)
+        ep.ep_dispatch_cached(x, out["send_pos"], recv_x=out["recv_x"], status=status)
+        if ev is not None:
+            ev[3].record(stream)
         ep.ep_combine(out["recv_x"], out["send_pos"], out["recv_topk_weights"], combined_x=cx,
                       combined_topk_weights=cw, status=status)
         if ev is not None:
-            ev[3].record(stream)
+            ev[4].record(stream)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -443,7 +480,7 @@ def run_ours(args) -> None:
     bytes_step = bytes_d + bytes_c
 
     # ---- timed region: exactly K steps, device-resident inputs ------------
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
@@ -460,8 +497,10 @@ def run_ours(args) -> None:
     clocks = sampler.stop()
     ms_local = t_start.elapsed_time(t_end) / args.steps
     lay_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    disp_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    comb_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    notify_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    copy_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    comb_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
+    disp_ms = notify_ms + copy_ms
     agg = aggregate(bytes_step, R * T, ms_local, device)
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the timed region")
@@ -496,10 +535,13 @@ def run_ours(args) -> None:
     d2h = cx_h.numel() * 2 + cw_h.numel() * 4
 
     peak, peak_kind = load_peak()
-    dominant = "combine_kernel" if comb_ms >= disp_ms else "ep_dispatch (scan + copy kernels)"
-    dom_bytes = bytes_c if comb_ms >= disp_ms else bytes_d
-    dom_ms = comb_ms if comb_ms >= disp_ms else disp_ms
+    bytes_copy = R * T * H * 2 + N * H * 2       # rows: read once, written per copy
+    if copy_ms >= comb_ms:
+        dominant, dom_bytes, dom_ms = "dispatch_copy_kernel", bytes_copy, copy_ms
+    else:
+        dominant, dom_bytes, dom_ms = "combine_kernel", bytes_c, comb_ms
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    traffic = recorded_traffic(dominant, T)
 
     line = {
         "metric": METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
@@ -513,15 +555,17 @@ def run_ours(args) -> None:
                    "l2": "inputs larger than L2 (x 470 MB, recv_x 2.5 GB written); no flush"},
         "tokens_per_s": agg["tokens_per_s"],
         "pct_of_8TBps": 100.0 * agg["gbs"] / (SPEC_HBM_GBS * ws),
-        "phases_ms": {"layout": lay_ms, "dispatch": disp_ms, "combine": comb_ms},
+        "phases_ms": {"layout": lay_ms, "dispatch": disp_ms, "dispatch_notify": notify_ms,
+                      "dispatch_copy": copy_ms, "combine": comb_ms},
         "bytes_per_step": {"dispatch": bytes_d, "combine": bytes_c, "copies": N},
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                     "algorithmic_bytes": dom_bytes,
                      "peak_source": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_kind == "measured" else "fallback 6.65 TB/s"},
         "e2e": {"value": e2e["gbs"], "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e["ms_per_step"]},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 4 * args.steps,   # layout, scan, copy, combine per step
         "clocks": clocks,
     }
     if ws == 1 and rank == 0 and not args.no_extra and T == CONFIGS["normal"].T:

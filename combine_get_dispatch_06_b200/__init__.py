@@ -41,9 +41,13 @@ _SIGS = {
     "ep_dispatch_workspace_bytes": (_Z, [_I, _I, _I]),
     "ep_dispatch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                          _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P]),
+    "ep_notify_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P]),
+    "ep_dispatch_cached": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "ep_dispatch_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                  _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
-    "ep_combine": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "ep_dispatch_cached_fp8": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "ep_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "ep_ll_workspace_bytes": (_Z, [_I, _I, _I]),
     "ep_ll_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                             _P, _Z, _P, _P]),
@@ -219,6 +223,102 @@ def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor],
     return o
 
 
+def ep_notify_dispatch(topk_idx: Optional[torch.Tensor], topk_weights: Optional[torch.Tensor],
+                       num_tokens: int, num_ranks: int, num_experts: int, *,
+                       is_token_in_rank: Optional[torch.Tensor] = None,
+                       expert_alignment: int = 1, capacity: Optional[int] = None,
+                       out: Optional[dict] = None, with_metadata: bool = True,
+                       workspace: Optional[torch.Tensor] = None, status=None,
+                       stream=None) -> dict:
+    """The first half of ep_dispatch: handle + received metadata (no rows)."""
+    R, T = num_ranks, num_tokens
+    src = topk_idx if topk_idx is not None else is_token_in_rank
+    dev = src.device
+    K = topk_idx.shape[2] if topk_idx is not None else 0
+    E = num_experts
+    cap = R * T if capacity is None else int(capacity)
+    o = dict(out or {})
+
+    def get(name, shape, dtype):
+        if o.get(name) is None:
+            o[name] = torch.empty(shape, dtype=dtype, device=dev)
+        _need(o[name], dtype, shape, name)
+        return o[name]
+
+    get("recv_src_idx", (R, cap), torch.int32)
+    get("rank_prefix_matrix", (R, R), torch.int32)
+    get("recv_count", (R,), torch.int32)
+    get("send_pos", (R, T, R), torch.int32)
+    meta = with_metadata and topk_idx is not None
+    if meta:
+        get("recv_topk_idx", (R, cap, K), torch.int64)
+        get("num_recv_tokens_per_expert", (R, E // R), torch.int32)
+        if topk_weights is not None:
+            get("recv_topk_weights", (R, cap, K), torch.float32)
+    if topk_idx is not None:
+        _need(topk_idx, torch.int64, (R, T, K), "topk_idx")
+    if topk_weights is not None:
+        _need(topk_weights, torch.float32, (R, T, K), "topk_weights")
+    if is_token_in_rank is not None:
+        _need(is_token_in_rank, torch.bool, (R, T, R), "is_token_in_rank")
+    need = ep_dispatch_workspace_bytes(R, T, E if topk_idx is not None else 0)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    rc = _lib.ep_notify_dispatch(
+        _ptr(topk_idx), _ptr(topk_weights), _ptr(is_token_in_rank), R, T, K, E,
+        int(expert_alignment), cap, _ptr(o.get("recv_topk_idx") if meta else None),
+        _ptr(o.get("recv_topk_weights") if meta else None), _ptr(o["recv_src_idx"]),
+        _ptr(o["rank_prefix_matrix"]), _ptr(o["recv_count"]),
+        _ptr(o.get("num_recv_tokens_per_expert") if meta else None), _ptr(o["send_pos"]),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
+    _check(rc, "ep_notify_dispatch")
+    return o
+
+
+def ep_dispatch_cached(x: torch.Tensor, send_pos: torch.Tensor, *, capacity: Optional[int] = None,
+                       recv_x: Optional[torch.Tensor] = None, status=None,
+                       stream=None) -> torch.Tensor:
+    """Cached-mode dispatch: rows of x to the rows send_pos names."""
+    R, T, H = x.shape
+    _need(x, torch.bfloat16, (R, T, H), "x")
+    _need(send_pos, torch.int32, (R, T, R), "send_pos")
+    cap = R * T if capacity is None else int(capacity)
+    if recv_x is None:
+        recv_x = torch.empty((R, cap, H), dtype=torch.bfloat16, device=x.device)
+    _need(recv_x, torch.bfloat16, (R, cap, H), "recv_x")
+    rc = _lib.ep_dispatch_cached(_ptr(x), _ptr(send_pos), R, T, H, cap, _ptr(recv_x),
+                                 _ptr(status), _stream(stream))
+    _check(rc, "ep_dispatch_cached")
+    return recv_x
+
+
+def ep_dispatch_cached_fp8(x_e4m3: torch.Tensor, x_scales: torch.Tensor, send_pos: torch.Tensor,
+                           *, scales_col_major: bool = False, capacity: Optional[int] = None,
+                           recv_x: Optional[torch.Tensor] = None,
+                           recv_scales: Optional[torch.Tensor] = None, status=None,
+                           stream=None):
+    """FP8 rows (uint8 e4m3 [R, T, H]) and their scales ([R, T, H/128], or
+    [R, H/128, T] when scales_col_major) to the rows send_pos names.  Returns
+    (recv_x uint8 [R, cap, H], recv_scales fp32 [R, cap, H/128])."""
+    R, T, H = x_e4m3.shape
+    nb = H // 128
+    _need(x_e4m3, torch.uint8, (R, T, H), "x_e4m3")
+    _need(x_scales, torch.float32, (R, nb, T) if scales_col_major else (R, T, nb), "x_scales")
+    _need(send_pos, torch.int32, (R, T, R), "send_pos")
+    cap = R * T if capacity is None else int(capacity)
+    if recv_x is None:
+        recv_x = torch.empty((R, cap, H), dtype=torch.uint8, device=x_e4m3.device)
+    if recv_scales is None:
+        recv_scales = torch.empty((R, cap, nb), dtype=torch.float32, device=x_e4m3.device)
+    _need(recv_x, torch.uint8, (R, cap, H), "recv_x")
+    _need(recv_scales, torch.float32, (R, cap, nb), "recv_scales")
+    rc = _lib.ep_dispatch_cached_fp8(_ptr(x_e4m3), _ptr(x_scales), 1 if scales_col_major else 0,
+                                     _ptr(send_pos), R, T, H, cap, _ptr(recv_x),
+                                     _ptr(recv_scales), _ptr(status), _stream(stream))
+    _check(rc, "ep_dispatch_cached_fp8")
+    return recv_x, recv_scales
+
+
 def ep_dispatch_noalloc(x: torch.Tensor, topk_idx: Optional[torch.Tensor],
                         topk_weights: Optional[torch.Tensor], num_experts: int, *,
                         is_token_in_rank: Optional[torch.Tensor] = None,
@@ -264,6 +364,7 @@ def ep_dispatch_noalloc(x: torch.Tensor, topk_idx: Optional[torch.Tensor],
 
 def ep_combine(y: torch.Tensor, send_pos: torch.Tensor,
                recv_topk_weights: Optional[torch.Tensor] = None, *,
+               bias: Optional[tuple] = None,
                combined_x: Optional[torch.Tensor] = None,
                combined_topk_weights: Optional[torch.Tensor] = None,
                status=None, stream=None):
@@ -283,8 +384,13 @@ def ep_combine(y: torch.Tensor, send_pos: torch.Tensor,
     if combined_x is None:
         combined_x = torch.empty((R, T, H), dtype=torch.bfloat16, device=dev)
     _need(combined_x, torch.bfloat16, (R, T, H), "combined_x")
+    b0, b1 = (bias if bias is not None else (None, None))
+    for b, nm in ((b0, "bias_0"), (b1, "bias_1")):
+        if b is not None:
+            _need(b, torch.bfloat16, (R, T, H), nm)
     rc = _lib.ep_combine(
-        _ptr(y), _ptr(recv_topk_weights), _ptr(send_pos), R, T, H, K, cap, _ptr(combined_x),
+        _ptr(y), _ptr(recv_topk_weights), _ptr(send_pos), _ptr(b0), _ptr(b1), R, T, H, K, cap,
+        _ptr(combined_x),
         _ptr(combined_topk_weights if recv_topk_weights is not None else None), _ptr(status),
         _stream(stream))
     _check(rc, "ep_combine")

@@ -1,9 +1,10 @@
 // ep_combine.cu -- A4: combine (gather-reduce of the dispatched copies).
 //
 // Semantics (DeepEP legacy-test analysis page, combine call and its check
-// (combined_x - bias) / is_token_in_rank.sum(1) == x): every source token
-// gets back the sum of the rows its destinations return, summed in fp32 in
-// ascending destination rank, then rounded once to bf16 (nearest even).
+// (combined_x - bias_0 - bias_1) / is_token_in_rank.sum(1) == x): every
+// source token gets back the sum of the rows its destinations return, summed
+// in fp32 in ascending destination rank, plus bias_0 then bias_1 if given,
+// then rounded once to bf16 (nearest even).
 //
 // One warp per source token.  The warp reads send_pos[s][t][0..R), compacts
 // the valid (d, row) pairs in ascending d into shared memory with a ballot,
@@ -43,7 +44,8 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float (&a)[8]) {
 
 __global__ void __launch_bounds__(kCombineWarps * 32)
     combine_kernel(const uint8_t *__restrict__ y, const float *__restrict__ recv_w,
-                   const int32_t *__restrict__ send_pos, int R, long num_tok, int H, int K,
+                   const int32_t *__restrict__ send_pos, const uint8_t *__restrict__ bias0,
+                   const uint8_t *__restrict__ bias1, int R, long num_tok, int H, int K,
                    int cap, uint8_t *__restrict__ out, float *__restrict__ out_w,
                    int32_t *status) {
   extern __shared__ __align__(16) int64_t s_rows[];  // [warps][R] row indices d*cap + pos
@@ -94,6 +96,15 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
           }
         }
       }
+      // bias terms come after the sum of the copies: first bias_0, then bias_1
+      if (bias0 != nullptr) {
+        add_bf16x8(a0, ld_stream_v4(bias0 + u * row_bytes + static_cast<long>(c) * 16));
+        if (two) add_bf16x8(a1, ld_stream_v4(bias0 + u * row_bytes + static_cast<long>(c + 32) * 16));
+      }
+      if (bias1 != nullptr) {
+        add_bf16x8(a0, ld_stream_v4(bias1 + u * row_bytes + static_cast<long>(c) * 16));
+        if (two) add_bf16x8(a1, ld_stream_v4(bias1 + u * row_bytes + static_cast<long>(c + 32) * 16));
+      }
       st_stream_v4(orow + static_cast<long>(c) * 16, pack_bf16x8(a0));
       if (two) st_stream_v4(orow + static_cast<long>(c + 32) * 16, pack_bf16x8(a1));
     }
@@ -110,10 +121,10 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 }  // namespace ep
 
 extern "C" EP_API int ep_combine(const void *y, const float *recv_topk_weights,
-                                 const int32_t *send_pos, int num_ranks, int num_tokens,
-                                 int hidden, int num_topk, int capacity, void *combined_x,
-                                 float *combined_topk_weights, int32_t *status,
-                                 cudaStream_t stream) {
+                                 const int32_t *send_pos, const void *bias_0, const void *bias_1,
+                                 int num_ranks, int num_tokens, int hidden, int num_topk,
+                                 int capacity, void *combined_x, float *combined_topk_weights,
+                                 int32_t *status, cudaStream_t stream) {
   using namespace ep;
   const int R = num_ranks, T = num_tokens, H = hidden, K = num_topk, cap = capacity;
   if (R < 1 || R > kMaxRanks || T < 0 || H < 8 || H % 8 != 0 || cap < 0) return EP_ERR_INVALID_ARG;
@@ -122,7 +133,8 @@ extern "C" EP_API int ep_combine(const void *y, const float *recv_topk_weights,
     return EP_ERR_INVALID_ARG;
   if (T == 0) return EP_OK;
   if (y == nullptr || send_pos == nullptr || combined_x == nullptr) return EP_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(y) & 15u) || (reinterpret_cast<uintptr_t>(combined_x) & 15u))
+  if ((reinterpret_cast<uintptr_t>(y) & 15u) || (reinterpret_cast<uintptr_t>(combined_x) & 15u) ||
+      (reinterpret_cast<uintptr_t>(bias_0) & 15u) || (reinterpret_cast<uintptr_t>(bias_1) & 15u))
     return EP_ERR_INVALID_ARG;
   const long num_tok = static_cast<long>(R) * T;
   const int threads = kCombineWarps * 32;
@@ -134,7 +146,7 @@ extern "C" EP_API int ep_combine(const void *y, const float *recv_topk_weights,
       std::min<long>(want, static_cast<long>(ctas_per_sm(fn, threads, smem)) * num_sms());
   combine_kernel<<<static_cast<unsigned>(grid), threads, smem, stream>>>(
       static_cast<const uint8_t *>(y), combined_topk_weights ? recv_topk_weights : nullptr,
-      send_pos, R, num_tok, H, K, cap, static_cast<uint8_t *>(combined_x), combined_topk_weights,
-      status);
+      send_pos, static_cast<const uint8_t *>(bias_0), static_cast<const uint8_t *>(bias_1), R,
+      num_tok, H, K, cap, static_cast<uint8_t *>(combined_x), combined_topk_weights, status);
   return launch_status();
 }

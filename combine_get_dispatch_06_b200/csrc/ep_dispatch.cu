@@ -252,10 +252,11 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
 
 // ---------------------------------------------------------------------------
 // Row scatter.  One thread per destination rank (blockDim = 32 * ceil(R/32)),
-// thread 0 also drives the loads.  Items are (token, chunk) pairs; CTA b owns
-// tokens b, b + grid, b + 2*grid, ...  Stage i % S holds item i.  Loads run
-// S - 1 items ahead; before a stage is reloaded every thread waits until its
-// own bulk stores from that stage have finished reading shared memory.
+// thread 0 also drives the loads.  Each token is cut into items: `nchunks`
+// chunks of its data row and, for FP8 input, one item for its scales row.
+// CTA b owns tokens b, b + grid, b + 2*grid, ...; stage i % S holds item i.
+// Loads run S - 1 items ahead; before a stage is reloaded every thread waits
+// until its own bulk stores from that stage have finished reading it.
 // ---------------------------------------------------------------------------
 
 // Launch shape, chosen by a sweep on B200 at R=8, H=7168 (stages x chunk x
@@ -265,21 +266,42 @@ constexpr int kCopyStages = 4;
 constexpr int kCopyChunkMax = 4096;
 constexpr int kCopyMaxCtasPerSm = 2;
 
+// How the scales row of a token reaches shared memory.
+enum ScaleMode : int {
+  kScalesNone = 0,      // bf16 input: no scales
+  kScalesBulk = 1,      // row-major, rows a multiple of 16 bytes: bulk copy
+  kScalesGatherRow = 2, // row-major, other sizes: threads load
+  kScalesGatherCol = 3  // column-major [R][H/128][T]: threads gather
+};
+
+struct CopyArgs {
+  const uint8_t *x;       // data rows [R*T][row_bytes]
+  const float *xs;        // scales (FP8 input) or nullptr
+  const int32_t *send_pos;
+  uint8_t *recv_x;        // [R][cap][row_bytes]
+  float *recv_s;          // [R][cap][nblk] or nullptr
+  int R, T, cap;
+  long num_tok;
+  int row_bytes, chunk_bytes, nchunks, stage_stride;
+  int nblk, sc_mode, sc_store_bulk;
+  int32_t *status;
+  unsigned long long timeout_ns;
+};
+
 template <int S>
-__global__ void __launch_bounds__(kMaxRanks)
-    dispatch_copy_kernel(const uint8_t *__restrict__ x, const int32_t *__restrict__ send_pos,
-                         uint8_t *__restrict__ recv_x, int R, long num_tok, int row_bytes,
-                         int chunk_bytes, int nchunks, int stage_stride, int cap,
-                         int32_t *status, unsigned long long timeout_ns) {
+__global__ void __launch_bounds__(kMaxRanks) dispatch_copy_kernel(CopyArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
   uint8_t *buf = smem + 128;
   const int tid = threadIdx.x;
   const int d = tid;
+  const int ipt = a.nchunks + (a.sc_mode != kScalesNone ? 1 : 0);  // items per token
+  const int sc_bytes = a.nblk * 4;
 
-  const long ntok_cta =
-      static_cast<long>(blockIdx.x) < num_tok ? (num_tok - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  const long nitems = ntok_cta * nchunks;
+  const long ntok_cta = static_cast<long>(blockIdx.x) < a.num_tok
+                            ? (a.num_tok - 1 - blockIdx.x) / gridDim.x + 1
+                            : 0;
+  const long nitems = ntok_cta * ipt;
 
   if (tid == 0) {
 #pragma unroll
@@ -289,18 +311,27 @@ __global__ void __launch_bounds__(kMaxRanks)
   __syncthreads();
 
   auto token_of = [&](long i) -> long {
-    return static_cast<long>(blockIdx.x) + (i / nchunks) * static_cast<long>(gridDim.x);
+    return static_cast<long>(blockIdx.x) + (i / ipt) * static_cast<long>(gridDim.x);
   };
-  auto issue_load = [&](long i, int stg) {
+  auto issue_load = [&](long i, int stg) {  // thread 0
     const long u = token_of(i);
-    const int off = static_cast<int>(i % nchunks) * chunk_bytes;
-    const int nb = min(chunk_bytes, row_bytes - off);
-    mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(nb));
-    bulk_g2s_hint(buf + stg * stage_stride, x + u * row_bytes + off, static_cast<uint32_t>(nb),
-                  &bars[stg], l2_evict_first_policy());
+    const int sub = static_cast<int>(i % ipt);
+    if (sub < a.nchunks) {
+      const int off = sub * a.chunk_bytes;
+      const int nb = min(a.chunk_bytes, a.row_bytes - off);
+      mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(nb));
+      bulk_g2s_hint(buf + stg * a.stage_stride, a.x + u * a.row_bytes + off,
+                    static_cast<uint32_t>(nb), &bars[stg], l2_evict_first_policy());
+    } else if (a.sc_mode == kScalesBulk) {
+      mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(sc_bytes));
+      bulk_g2s(buf + stg * a.stage_stride, a.xs + u * a.nblk, static_cast<uint32_t>(sc_bytes),
+               &bars[stg]);
+    } else {
+      mbar_arrive(&bars[stg]);  // gathered by the threads when the item is used
+    }
   };
   auto load_pos = [&](long i) -> int {
-    return d < R ? __ldg(send_pos + token_of(i) * R + d) : -1;
+    return d < a.R ? __ldg(a.send_pos + token_of(i) * a.R + d) : -1;
   };
 
   int sp[S];
@@ -322,16 +353,36 @@ __global__ void __launch_bounds__(kMaxRanks)
     for (int st = 0; st < S; ++st) {
       const long i = base + st;
       if (i >= nitems) break;
-      const bool ok = mbar_wait_bounded(&bars[st], parity, timeout_ns);
-      const int chunk = static_cast<int>(i % nchunks);
+      const bool ok = mbar_wait_bounded(&bars[st], parity, a.timeout_ns);
+      const int sub = static_cast<int>(i % ipt);
+      uint8_t *stage = buf + st * a.stage_stride;
+      if (sub == a.nchunks && a.sc_mode >= kScalesGatherRow) {  // uniform in the CTA
+        const long u = token_of(i);
+        float *f = reinterpret_cast<float *>(stage);
+        for (int j = tid; j < a.nblk; j += blockDim.x) {
+          if (a.sc_mode == kScalesGatherRow) {
+            f[j] = __ldg(a.xs + u * a.nblk + j);
+          } else {
+            const long s = u / a.T, t = u % a.T;
+            f[j] = __ldg(a.xs + (s * a.nblk + j) * a.T + t);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+      }
       if (ok && sp[st] >= 0) {  // sp < 0: no copy to this rank
-        if (sp[st] < cap) {
-          const int off = chunk * chunk_bytes;
-          const int nb = min(chunk_bytes, row_bytes - off);
-          bulk_s2g(recv_x + (static_cast<long>(d) * cap + sp[st]) * row_bytes + off,
-                   buf + st * stage_stride, static_cast<uint32_t>(nb));
-        } else if (chunk == 0) {
-          report(status, EP_STATUS_CAPACITY);
+        const long row = static_cast<long>(d) * a.cap + sp[st];
+        if (sp[st] >= a.cap) {
+          if (sub == 0) report(a.status, EP_STATUS_CAPACITY);
+        } else if (sub < a.nchunks) {
+          const int off = sub * a.chunk_bytes;
+          const int nb = min(a.chunk_bytes, a.row_bytes - off);
+          bulk_s2g(a.recv_x + row * a.row_bytes + off, stage, static_cast<uint32_t>(nb));
+        } else if (a.sc_store_bulk) {
+          bulk_s2g(a.recv_s + row * a.nblk, stage, static_cast<uint32_t>(sc_bytes));
+        } else {
+          const float *f = reinterpret_cast<const float *>(stage);
+          for (int j = 0; j < a.nblk; ++j) a.recv_s[row * a.nblk + j] = f[j];
         }
       }
       bulk_commit();
@@ -351,12 +402,13 @@ __global__ void __launch_bounds__(kMaxRanks)
   }
   bulk_wait_all<0>();
   if (!all_ok) {
-    report(status, EP_STATUS_WAIT_TIMEOUT);
+    report(a.status, EP_STATUS_WAIT_TIMEOUT);
     if (tid == 0) {
       // drain loads still in flight before the CTA's shared memory goes away
       const long end = min(nitems, stop + S - 1);
       for (long k = stop; k < end; ++k)
-        (void)mbar_wait_bounded(&bars[k % S], static_cast<uint32_t>((k / S) & 1), timeout_ns);
+        (void)mbar_wait_bounded(&bars[k % S], static_cast<uint32_t>((k / S) & 1),
+                                a.timeout_ns);
     }
   }
 }
@@ -372,25 +424,17 @@ extern "C" EP_API size_t ep_dispatch_workspace_bytes(int num_ranks, int num_toke
   return scan_workspace_bytes(tiles, num_ranks, num_experts);
 }
 
-extern "C" EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
-                                  const float *topk_weights, const uint8_t *is_token_in_rank,
-                                  int num_ranks, int num_tokens, int hidden, int num_topk,
-                                  int num_experts, int expert_alignment, int capacity,
-                                  void *recv_x, int64_t *recv_topk_idx, float *recv_topk_weights,
-                                  int32_t *recv_src_idx, int32_t *rank_prefix_matrix,
-                                  int32_t *recv_count, int32_t *num_recv_tokens_per_expert,
-                                  int32_t *send_pos, void *workspace, size_t workspace_bytes,
-                                  int32_t *status, cudaStream_t stream) {
-  using namespace ep;
-  const int R = num_ranks, T = num_tokens, H = hidden, K = num_topk, E = num_experts;
-  const int cap = capacity;
-  if (R < 1 || R > kMaxRanks || T < 0 || H < 8 || H % 8 != 0 || cap < 0 || expert_alignment < 1)
-    return EP_ERR_INVALID_ARG;
-  if (rank_prefix_matrix == nullptr || recv_count == nullptr) return EP_ERR_INVALID_ARG;
-  if (T == 0) {  // nothing to route; an empty tensor's pointers may be NULL
-    if (num_recv_tokens_per_expert != nullptr &&
-        (E < 1 || E > kMaxExperts || E % R != 0))
-      return EP_ERR_INVALID_ARG;
+namespace ep {
+namespace {
+
+// A2 (+ received metadata): the scan kernel.  Arguments already checked.
+int notify_impl(const int64_t *topk_idx, const float *topk_weights,
+                const uint8_t *is_token_in_rank, int R, int T, int K, int E, int align, int cap,
+                int64_t *recv_topk_idx, float *recv_topk_weights, int32_t *recv_src_idx,
+                int32_t *rank_prefix_matrix, int32_t *recv_count,
+                int32_t *num_recv_tokens_per_expert, int32_t *send_pos, void *workspace,
+                int32_t *status, cudaStream_t stream) {
+  if (T == 0) {  // nothing to route
     if (cudaMemsetAsync(rank_prefix_matrix, 0, sizeof(int32_t) * R * R, stream) != cudaSuccess ||
         cudaMemsetAsync(recv_count, 0, sizeof(int32_t) * R, stream) != cudaSuccess)
       return EP_ERR_CUDA;
@@ -398,34 +442,24 @@ extern "C" EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
         cudaMemsetAsync(num_recv_tokens_per_expert, 0, sizeof(int32_t) * E, stream) !=
             cudaSuccess)
       return EP_ERR_CUDA;
+    if (recv_topk_idx != nullptr && cap > 0 &&
+        cudaMemsetAsync(recv_topk_idx, 0xFF, sizeof(int64_t) * R * static_cast<size_t>(cap) * K,
+                        stream) != cudaSuccess)
+      return EP_ERR_CUDA;
     return EP_OK;
   }
-  if (topk_idx == nullptr && is_token_in_rank == nullptr) return EP_ERR_INVALID_ARG;
-  if (topk_idx != nullptr &&
-      (K < 1 || K > kMaxTopk || E < 1 || E > kMaxExperts || E % R != 0))
-    return EP_ERR_INVALID_ARG;
-  if ((recv_topk_idx != nullptr || num_recv_tokens_per_expert != nullptr) && topk_idx == nullptr)
-    return EP_ERR_INVALID_ARG;
-  if (recv_topk_weights != nullptr && (topk_idx == nullptr || topk_weights == nullptr))
-    return EP_ERR_INVALID_ARG;
-  const int El = topk_idx != nullptr ? E / R : 1;
-  if (send_pos == nullptr || recv_src_idx == nullptr || x == nullptr ||
-      (cap > 0 && recv_x == nullptr))
-    return EP_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(recv_x) & 15u))
-    return EP_ERR_INVALID_ARG;
   const int Ectr = topk_idx != nullptr ? E : 0;
   const size_t need = ep_dispatch_workspace_bytes(R, T, Ectr);
-  if (workspace == nullptr || workspace_bytes < need ||
-      (reinterpret_cast<uintptr_t>(workspace) & 15u))
-    return EP_ERR_INVALID_ARG;
   if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return EP_ERR_CUDA;
+  // rows past the receive count read -1 (fixed worst-case capacity): every
+  // int64 of all-ones bytes is -1, and the scan overwrites the real rows
+  if (recv_topk_idx != nullptr && cap > 0 &&
+      cudaMemsetAsync(recv_topk_idx, 0xFF, sizeof(int64_t) * R * static_cast<size_t>(cap) * K,
+                      stream) != cudaSuccess)
+    return EP_ERR_CUDA;
 
   const int tiles_per_src = (T + kScanTile - 1) / kScanTile;
   const long num_tiles = static_cast<long>(R) * tiles_per_src;
-  if (num_tiles > 0x7fffffffL || static_cast<long>(R) * T > 0x7fffffffL)
-    return EP_ERR_UNSUPPORTED;
-
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   DispatchScanParams p;
   p.topk_idx = topk_idx;
@@ -435,9 +469,9 @@ extern "C" EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
   p.T = T;
   p.K = K;
   p.E = E;
-  p.El = El;
+  p.El = topk_idx != nullptr ? E / R : 1;
   p.cap = cap;
-  p.align = expert_alignment;
+  p.align = align;
   p.tiles_per_src = tiles_per_src;
   p.num_tiles = static_cast<int>(num_tiles);
   p.W = (R + 31) / 32;
@@ -457,25 +491,177 @@ extern "C" EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
   p.timeout_ns = wc.timeout_ns;
   p.flags = wc.flags;
   dispatch_scan_kernel<<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
-  if (launch_status() != EP_OK) return EP_ERR_CUDA;
+  return launch_status();
+}
 
-  if (cap == 0) return EP_OK;
-  const int row_bytes = H * 2;
-  const int nchunks = (row_bytes + kCopyChunkMax - 1) / kCopyChunkMax;
-  const int chunk_bytes = ((row_bytes + nchunks - 1) / nchunks + 15) & ~15;
-  const int stage_stride = (chunk_bytes + 127) & ~127;
-  const size_t smem = 128 + static_cast<size_t>(kCopyStages) * stage_stride;
+// A3 rows: the bulk-copy kernel.  Arguments already checked.  `xs` (FP8
+// scales, [R][T][nblk] or, col_major, [R][nblk][T]) may be nullptr.
+int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int32_t *send_pos,
+              int R, int T, int row_bytes, int cap, void *recv_x, float *recv_s,
+              int32_t *status, cudaStream_t stream) {
+  if (T == 0 || cap == 0) return EP_OK;
+  CopyArgs a;
+  a.x = static_cast<const uint8_t *>(x);
+  a.xs = xs;
+  a.send_pos = send_pos;
+  a.recv_x = static_cast<uint8_t *>(recv_x);
+  a.recv_s = recv_s;
+  a.R = R;
+  a.T = T;
+  a.cap = cap;
+  a.num_tok = static_cast<long>(R) * T;
+  a.row_bytes = row_bytes;
+  a.nchunks = (row_bytes + kCopyChunkMax - 1) / kCopyChunkMax;
+  a.chunk_bytes = ((row_bytes + a.nchunks - 1) / a.nchunks + 15) & ~15;
+  a.nblk = xs != nullptr ? nblk : 0;
+  const int sc_bytes = a.nblk * 4;
+  const bool rows16 = (sc_bytes % 16) == 0;
+  if (xs == nullptr)
+    a.sc_mode = kScalesNone;
+  else if (col_major)
+    a.sc_mode = kScalesGatherCol;
+  else if (rows16 && (reinterpret_cast<uintptr_t>(xs) & 15u) == 0)
+    a.sc_mode = kScalesBulk;
+  else
+    a.sc_mode = kScalesGatherRow;
+  a.sc_store_bulk = xs != nullptr && rows16 && (reinterpret_cast<uintptr_t>(recv_s) & 15u) == 0;
+  a.stage_stride = (std::max(a.chunk_bytes, sc_bytes) + 127) & ~127;
+  a.status = status;
+  a.timeout_ns = wait_config().timeout_ns;
+  const size_t smem = 128 + static_cast<size_t>(kCopyStages) * a.stage_stride;
   const int threads = 32 * ((R + 31) / 32);
   const void *fn = reinterpret_cast<const void *>(dispatch_copy_kernel<kCopyStages>);
   if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
-  const long num_tok = static_cast<long>(R) * T;
   const long grid = std::min<long>(
-      num_tok,
+      a.num_tok,
       static_cast<long>(std::min(kCopyMaxCtasPerSm, ctas_per_sm(fn, threads, smem))) * num_sms());
-  dispatch_copy_kernel<kCopyStages><<<static_cast<unsigned>(grid), threads, smem, stream>>>(
-      static_cast<const uint8_t *>(x), send_pos, static_cast<uint8_t *>(recv_x), R, num_tok,
-      row_bytes, chunk_bytes, nchunks, stage_stride, cap, status, wc.timeout_ns);
+  dispatch_copy_kernel<kCopyStages><<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
   return launch_status();
+}
+
+// Checks shared by ep_dispatch and ep_notify_dispatch.
+int check_notify_args(const int64_t *topk_idx, const float *topk_weights,
+                      const uint8_t *is_token_in_rank, int R, int T, int K, int E, int align,
+                      int cap, const int64_t *recv_topk_idx, const float *recv_topk_weights,
+                      const int32_t *recv_src_idx, const int32_t *rank_prefix_matrix,
+                      const int32_t *recv_count, const int32_t *nrte, const int32_t *send_pos,
+                      const void *workspace, size_t workspace_bytes) {
+  if (R < 1 || R > kMaxRanks || T < 0 || cap < 0 || align < 1) return EP_ERR_INVALID_ARG;
+  if (rank_prefix_matrix == nullptr || recv_count == nullptr) return EP_ERR_INVALID_ARG;
+  const bool meta = recv_topk_idx != nullptr || recv_topk_weights != nullptr || nrte != nullptr;
+  if (meta && (K < 1 || K > kMaxTopk || E < 1 || E > kMaxExperts || E % R != 0))
+    return EP_ERR_INVALID_ARG;
+  if (T == 0) return EP_OK;  // an empty tensor's pointers may be NULL
+  if (topk_idx == nullptr && is_token_in_rank == nullptr) return EP_ERR_INVALID_ARG;
+  if (topk_idx != nullptr && (K < 1 || K > kMaxTopk || E < 1 || E > kMaxExperts || E % R != 0))
+    return EP_ERR_INVALID_ARG;
+  if (meta && topk_idx == nullptr) return EP_ERR_INVALID_ARG;
+  if (recv_topk_weights != nullptr && topk_weights == nullptr) return EP_ERR_INVALID_ARG;
+  if (send_pos == nullptr || recv_src_idx == nullptr) return EP_ERR_INVALID_ARG;
+  if (static_cast<long>(R) * ((T + kScanTile - 1) / kScanTile) > 0x7fffffffL ||
+      static_cast<long>(R) * T > 0x7fffffffL)
+    return EP_ERR_UNSUPPORTED;
+  const size_t need = ep_dispatch_workspace_bytes(R, T, topk_idx != nullptr ? E : 0);
+  if (workspace == nullptr || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 15u))
+    return EP_ERR_INVALID_ARG;
+  return EP_OK;
+}
+
+int check_copy_args(const void *x, const int32_t *send_pos, int R, int T, int H, int cap,
+                    const void *recv_x) {
+  if (R < 1 || R > kMaxRanks || T < 0 || H < 8 || H % 8 != 0 || cap < 0)
+    return EP_ERR_INVALID_ARG;
+  if (T == 0 || cap == 0) return EP_OK;
+  if (x == nullptr || send_pos == nullptr || recv_x == nullptr) return EP_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(recv_x) & 15u))
+    return EP_ERR_INVALID_ARG;
+  if (static_cast<long>(R) * T > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
+  return EP_OK;
+}
+
+}  // namespace
+}  // namespace ep
+
+extern "C" EP_API int ep_notify_dispatch(const int64_t *topk_idx, const float *topk_weights,
+                                         const uint8_t *is_token_in_rank, int num_ranks,
+                                         int num_tokens, int num_topk, int num_experts,
+                                         int expert_alignment, int capacity,
+                                         int64_t *recv_topk_idx, float *recv_topk_weights,
+                                         int32_t *recv_src_idx, int32_t *rank_prefix_matrix,
+                                         int32_t *recv_count,
+                                         int32_t *num_recv_tokens_per_expert, int32_t *send_pos,
+                                         void *workspace, size_t workspace_bytes,
+                                         int32_t *status, cudaStream_t stream) {
+  using namespace ep;
+  const int rc = check_notify_args(topk_idx, topk_weights, is_token_in_rank, num_ranks,
+                                   num_tokens, num_topk, num_experts, expert_alignment, capacity,
+                                   recv_topk_idx, recv_topk_weights, recv_src_idx,
+                                   rank_prefix_matrix, recv_count, num_recv_tokens_per_expert,
+                                   send_pos, workspace, workspace_bytes);
+  if (rc != EP_OK) return rc;
+  return notify_impl(topk_idx, topk_weights, is_token_in_rank, num_ranks, num_tokens, num_topk,
+                     num_experts, expert_alignment, capacity, recv_topk_idx, recv_topk_weights,
+                     recv_src_idx, rank_prefix_matrix, recv_count, num_recv_tokens_per_expert,
+                     send_pos, workspace, status, stream);
+}
+
+extern "C" EP_API int ep_dispatch_cached(const void *x, const int32_t *send_pos, int num_ranks,
+                                         int num_tokens, int hidden, int capacity, void *recv_x,
+                                         int32_t *status, cudaStream_t stream) {
+  using namespace ep;
+  const int rc = check_copy_args(x, send_pos, num_ranks, num_tokens, hidden, capacity, recv_x);
+  if (rc != EP_OK) return rc;
+  return copy_impl(x, nullptr, 0, 0, send_pos, num_ranks, num_tokens, hidden * 2, capacity,
+                   recv_x, nullptr, status, stream);
+}
+
+extern "C" EP_API int ep_dispatch_cached_fp8(const void *x_e4m3, const float *x_scales,
+                                             int scales_col_major, const int32_t *send_pos,
+                                             int num_ranks, int num_tokens, int hidden,
+                                             int capacity, void *recv_x, float *recv_scales,
+                                             int32_t *status, cudaStream_t stream) {
+  using namespace ep;
+  const int R = num_ranks, T = num_tokens, H = hidden, cap = capacity;
+  if (R < 1 || R > kMaxRanks || T < 0 || H < 128 || H % 128 != 0 || cap < 0)
+    return EP_ERR_INVALID_ARG;
+  if (T == 0 || cap == 0) return EP_OK;
+  if (x_e4m3 == nullptr || x_scales == nullptr || send_pos == nullptr || recv_x == nullptr ||
+      recv_scales == nullptr)
+    return EP_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x_e4m3) & 15u) || (reinterpret_cast<uintptr_t>(recv_x) & 15u) ||
+      (reinterpret_cast<uintptr_t>(x_scales) & 3u) ||
+      (reinterpret_cast<uintptr_t>(recv_scales) & 3u))
+    return EP_ERR_INVALID_ARG;
+  if (static_cast<long>(R) * T > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
+  return copy_impl(x_e4m3, x_scales, scales_col_major, H / 128, send_pos, R, T, H, cap, recv_x,
+                   recv_scales, status, stream);
+}
+
+extern "C" EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
+                                  const float *topk_weights, const uint8_t *is_token_in_rank,
+                                  int num_ranks, int num_tokens, int hidden, int num_topk,
+                                  int num_experts, int expert_alignment, int capacity,
+                                  void *recv_x, int64_t *recv_topk_idx, float *recv_topk_weights,
+                                  int32_t *recv_src_idx, int32_t *rank_prefix_matrix,
+                                  int32_t *recv_count, int32_t *num_recv_tokens_per_expert,
+                                  int32_t *send_pos, void *workspace, size_t workspace_bytes,
+                                  int32_t *status, cudaStream_t stream) {
+  using namespace ep;
+  int rc = check_notify_args(topk_idx, topk_weights, is_token_in_rank, num_ranks, num_tokens,
+                             num_topk, num_experts, expert_alignment, capacity, recv_topk_idx,
+                             recv_topk_weights, recv_src_idx, rank_prefix_matrix, recv_count,
+                             num_recv_tokens_per_expert, send_pos, workspace, workspace_bytes);
+  if (rc != EP_OK) return rc;
+  rc = check_copy_args(x, send_pos, num_ranks, num_tokens, hidden, capacity, recv_x);
+  if (rc != EP_OK) return rc;
+  rc = notify_impl(topk_idx, topk_weights, is_token_in_rank, num_ranks, num_tokens, num_topk,
+                   num_experts, expert_alignment, capacity, recv_topk_idx, recv_topk_weights,
+                   recv_src_idx, rank_prefix_matrix, recv_count, num_recv_tokens_per_expert,
+                   send_pos, workspace, status, stream);
+  if (rc != EP_OK) return rc;
+  return copy_impl(x, nullptr, 0, 0, send_pos, num_ranks, num_tokens, hidden * 2, capacity,
+                   recv_x, nullptr, status, stream);
 }
 
 // ---------------------------------------------------------------------------

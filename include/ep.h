@@ -148,7 +148,11 @@ EP_API size_t ep_dispatch_workspace_bytes(int num_ranks, int num_tokens,
  *                      send_pos and recv_count form the dispatch handle.)
  *   workspace          ep_dispatch_workspace_bytes(R, T, E) bytes, any content
  * A copy whose row is >= cap is not written and sets EP_STATUS_CAPACITY;
- * send_pos still holds its row.
+ * send_pos still holds its row.  With a fixed capacity this is the pages'
+ * num_worst_tokens mode: recv_topk_idx rows from recv_count[d] to cap - 1 read
+ * -1 (DeepEP legacy-test analysis page, the num_worst_tokens check), and no
+ * count has to travel to the host.  ep_dispatch = ep_notify_dispatch followed
+ * by ep_dispatch_cached on the handle it produced.
  */
 EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
                        const float *topk_weights,
@@ -161,6 +165,64 @@ EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
                        int32_t *num_recv_tokens_per_expert, int32_t *send_pos,
                        void *workspace, size_t workspace_bytes,
                        int32_t *status, cudaStream_t stream);
+
+/*
+ * A2 + received metadata: the first half of ep_dispatch (the notify step of
+ * the pages' dispatch, reduced to a prefix scan because all ranks share one
+ * HBM).  Arguments, outputs and rules are ep_dispatch's, without x and
+ * recv_x; it computes the handle (send_pos, rank_prefix_matrix, recv_count,
+ * recv_src_idx), recv_topk_idx / recv_topk_weights and
+ * num_recv_tokens_per_expert.
+ */
+EP_API int ep_notify_dispatch(const int64_t *topk_idx, const float *topk_weights,
+                              const uint8_t *is_token_in_rank, int num_ranks,
+                              int num_tokens, int num_topk, int num_experts,
+                              int expert_alignment, int capacity,
+                              int64_t *recv_topk_idx, float *recv_topk_weights,
+                              int32_t *recv_src_idx, int32_t *rank_prefix_matrix,
+                              int32_t *recv_count,
+                              int32_t *num_recv_tokens_per_expert,
+                              int32_t *send_pos, void *workspace,
+                              size_t workspace_bytes, int32_t *status,
+                              cudaStream_t stream);
+
+/*
+ * A3 rows: cached-mode dispatch.  Passage: Buffer.dispatch with a handle
+ * (DeepEP "Python 接口" page, Dispatch API, cached mode: the layout step is
+ * skipped and only recv_x is returned; legacy-test analysis page, the cached
+ * re-dispatch check that reproduces recv_x).
+ *
+ *   x         bf16 [R, T, H] (H % 8 == 0, 16-byte aligned)
+ *   send_pos  int32 [R, T, R] from ep_dispatch / ep_notify_dispatch
+ *   recv_x    out bf16 [R, cap, H]: row send_pos[s][t][d] of d = x[s][t]
+ * Only the rows named by send_pos are written; entries >= cap are skipped
+ * and set EP_STATUS_CAPACITY.
+ */
+EP_API int ep_dispatch_cached(const void *x, const int32_t *send_pos,
+                              int num_ranks, int num_tokens, int hidden,
+                              int capacity, void *recv_x, int32_t *status,
+                              cudaStream_t stream);
+
+/*
+ * A3 rows for FP8 input (the pages' x = (x_e4m3, x_scales) form; DeepEP
+ * "Python 接口" page, Dispatch API, FP8 tuple input; legacy-test analysis
+ * page, the column-major scale layout prepared for TMA).  Cached mode: the
+ * handle comes from ep_notify_dispatch (FP8 dispatch = ep_notify_dispatch +
+ * this call).
+ *
+ *   x_e4m3            e4m3 bytes [R, T, H], H % 128 == 0, 16-byte aligned
+ *   x_scales          fp32 per 128 channels: [R, T, H/128] (row-major) or,
+ *                     with scales_col_major = 1, [R, H/128, T]
+ *   recv_x            out e4m3 [R, cap, H]; recv_scales out fp32
+ *                     [R, cap, H/128] (row-major)
+ * Bytes are copied unchanged.
+ */
+EP_API int ep_dispatch_cached_fp8(const void *x_e4m3, const float *x_scales,
+                                  int scales_col_major, const int32_t *send_pos,
+                                  int num_ranks, int num_tokens, int hidden,
+                                  int capacity, void *recv_x,
+                                  float *recv_scales, int32_t *status,
+                                  cudaStream_t stream);
 
 /*
  * ep_dispatch without a workspace argument.  The routing method has no
@@ -205,17 +267,21 @@ EP_API int ep_dispatch_noalloc(const void *x, const int64_t *topk_idx,
  *                          y = recv_x); H % 8 == 0, 16-byte aligned
  *   recv_topk_weights      fp32 [R, cap, K] or NULL
  *   send_pos               int32 [R, T, R] from ep_dispatch
+ *   bias_0, bias_1         bf16 [R, T, H] or NULL (the pages' bias tuple),
+ *                          16-byte aligned
  *   combined_x             out bf16 [R, T, H]:
  *                          bf16_rne( sum over d ascending with send_pos >= 0
- *                          of float(y[d][send_pos]) ), fp32 accumulation from
- *                          +0.0; a token with no destination gives +0.0
+ *                          of float(y[d][send_pos]), then + bias_0, then +
+ *                          bias_1 ), fp32 accumulation from +0.0; a token with
+ *                          no destination gives +0.0 (+ its biases)
  *   combined_topk_weights  out fp32 [R, T, K] or NULL: the same ascending sum
  *                          of recv_topk_weights (needs recv_topk_weights)
  * A send_pos entry outside [-1, cap) is skipped and sets
  * EP_STATUS_BAD_POSITION.
  */
 EP_API int ep_combine(const void *y, const float *recv_topk_weights,
-                      const int32_t *send_pos, int num_ranks, int num_tokens,
+                      const int32_t *send_pos, const void *bias_0,
+                      const void *bias_1, int num_ranks, int num_tokens,
                       int hidden, int num_topk, int capacity, void *combined_x,
                       float *combined_topk_weights, int32_t *status,
                       cudaStream_t stream);

@@ -72,7 +72,9 @@ def lib() -> ctypes.CDLL:
         L.orc_dispatch_meta.restype = None
         L.orc_dispatch_meta.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P]
         L.orc_combine.restype = None
-        L.orc_combine.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _P, _L, _P, _P]
+        L.orc_combine.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _L, _P, _P]
+        L.orc_dispatch_rows_fp8.restype = None
+        L.orc_dispatch_rows_fp8.argtypes = [_P, _P, _I, _P, _I, _I, _I, _I, _P, _P]
         L.orc_ll_layout.restype = _L
         L.orc_ll_layout.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P]
         L.orc_quantize_row.restype = None
@@ -215,8 +217,9 @@ def dispatch_meta(topk_idx, topk_weights, send_pos, num_experts: int,
 
 
 def combine(y: np.ndarray, send_pos: np.ndarray, recv_topk_weights=None,
-            tokens=None) -> tuple:
-    """y [R,cap,H] bf16 bits, send_pos [R,T,R] -> (out [R,T,H], out_w [R,T,K]|None)."""
+            tokens=None, bias=None) -> tuple:
+    """y [R,cap,H] bf16 bits, send_pos [R,T,R] -> (out [R,T,H], out_w [R,T,K]|None).
+    bias: optional (bias_0, bias_1), each bf16 bits [R,T,H] or None."""
     yy = _c(y, np.uint16)
     R, cap, H = yy.shape
     sp = _c(send_pos, np.int32)
@@ -229,10 +232,28 @@ def combine(y: np.ndarray, send_pos: np.ndarray, recv_topk_weights=None,
         rw = _c(recv_topk_weights, np.float32)
         K = rw.shape[2]
         out_w = np.zeros((R, T, K), np.float32)
+    b0, b1 = bias if bias is not None else (None, None)
+    b0 = None if b0 is None else _c(b0, np.uint16)
+    b1 = None if b1 is None else _c(b1, np.uint16)
     tk, nt = _tokens(tokens)
-    lib().orc_combine(_ptr(yy), _ptr(rw), _ptr(sp), R, T, H, K, cap, _ptr(tk), nt,
-                      _ptr(out), _ptr(out_w))
+    lib().orc_combine(_ptr(yy), _ptr(rw), _ptr(sp), _ptr(b0), _ptr(b1), R, T, H, K, cap,
+                      _ptr(tk), nt, _ptr(out), _ptr(out_w))
     return out, out_w
+
+
+def dispatch_rows_fp8(x_q: np.ndarray, x_scales: np.ndarray, send_pos: np.ndarray,
+                      col_major: bool = False, cap: Optional[int] = None):
+    """FP8 input rows: x_q uint8 [R,T,H], scales [R,T,H/128] (or [R,H/128,T])."""
+    xq = _c(x_q, np.uint8)
+    R, T, H = xq.shape
+    xs = _c(x_scales, np.float32)
+    sp = _c(send_pos, np.int32)
+    cap = R * T if cap is None else cap
+    rq = np.zeros((R, cap, H), np.uint8)
+    rs = np.zeros((R, cap, H // 128), np.float32)
+    lib().orc_dispatch_rows_fp8(_ptr(xq), _ptr(xs), 1 if col_major else 0, _ptr(sp), R, T, H,
+                                cap, _ptr(rq), _ptr(rs))
+    return rq, rs
 
 
 def ll_layout(topk_idx: np.ndarray, num_experts: int) -> dict:

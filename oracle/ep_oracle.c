@@ -293,6 +293,33 @@ void orc_dispatch_rows(const uint16_t *x, const int32_t *send_pos,
 }
 
 /*
+ * FP8 input: recv_q[d][send_pos[s][t][d]] = x_q[s][t] (H bytes) and the
+ * token's H/128 scales to recv_scales[d][row].  x_scales is [R][T][H/128], or
+ * [R][H/128][T] when col_major.
+ */
+void orc_dispatch_rows_fp8(const uint8_t *x_q, const float *x_scales, int col_major,
+                           const int32_t *send_pos, int R, int T, int H, int cap,
+                           uint8_t *recv_q, float *recv_scales)
+{
+    int nb = H / 128;
+    for (int s = 0; s < R; ++s)
+        for (int t = 0; t < T; ++t) {
+            size_t st = (size_t)s * T + t;
+            for (int d = 0; d < R; ++d) {
+                int32_t row = send_pos[st * R + d];
+                if (row < 0 || row >= cap)
+                    continue;
+                size_t o = (size_t)d * cap + row;
+                memcpy(recv_q + o * H, x_q + st * H, (size_t)H);
+                for (int j = 0; j < nb; ++j)
+                    recv_scales[o * nb + j] =
+                        col_major ? x_scales[((size_t)s * nb + j) * T + t]
+                                  : x_scales[st * nb + j];
+            }
+        }
+}
+
+/*
  * Received metadata.  For the copy of (s,t) held by destination d at row p:
  *   recv_topk_idx[d][p][k]     = idx - d*El if idx / El == d, else -1
  *   recv_topk_weights[d][p][k] = w          if idx / El == d, else 0.0
@@ -330,14 +357,15 @@ void orc_dispatch_meta(const int64_t *topk_idx, const float *topk_weights,
 
 /*
  * out[s][t][h] = bf16( sum over d ascending with send_pos[s][t][d] in [0,cap)
- *                      of float(y[d][send_pos][h]) ), accumulated in fp32
- *                      from +0.0.
+ *                      of float(y[d][send_pos][h]), then + bias0, then +
+ *                      bias1 (each optional) ), accumulated in fp32 from +0.0.
  * out_w[s][t][k] = sum over the same d of recv_w[d][send_pos][k] (fp32), when
  * both recv_w and out_w are given.
  * tokens: optional list of flat token ids (NULL = all); out/out_w are indexed
  * by the flat token id in both cases.
  */
 void orc_combine(const uint16_t *y, const float *recv_w, const int32_t *send_pos,
+                 const uint16_t *bias0, const uint16_t *bias1,
                  int R, int T, int H, int K, int cap,
                  const int64_t *tokens, long ntokens,
                  uint16_t *out, float *out_w)
@@ -353,6 +381,10 @@ void orc_combine(const uint16_t *y, const float *recv_w, const int32_t *send_pos
                     continue;
                 acc = acc + orc_bf16_to_f32(y[((size_t)d * cap + row) * H + h]);
             }
+            if (bias0)
+                acc = acc + orc_bf16_to_f32(bias0[(size_t)st * H + h]);
+            if (bias1)
+                acc = acc + orc_bf16_to_f32(bias1[(size_t)st * H + h]);
             out[(size_t)st * H + h] = orc_f32_to_bf16(acc);
         }
         if (recv_w && out_w) {

@@ -268,6 +268,46 @@ def test_combine_signed_zero():
     assert (res["combined_x"][1, 0] == 0x0000).all()
 
 
+def test_combine_bias_matches_the_pages_check():
+    # (combined - bias_0 - bias_1) / n_dest == x, to within two fp32 roundings of
+    # the bias adds and one bf16 rounding of the result (fp64 reference)
+    w = Workload("cb", R=4, T=60, H=64, E=16, K=3)
+    inp = make(w)
+    b0 = make(Workload("cb0", R=4, T=60, H=64, E=16, K=3, seed=1))["x"]
+    b1 = make(Workload("cb1", R=4, T=60, H=64, E=16, K=3, seed=2))["x"]
+    res = oracle.normal_path(inp["x"], inp["topk_idx"], inp["topk_weights"], w.E)
+    out, _ = oracle.combine(res["recv_x"], res["send_pos"], bias=(b0, b1))
+    n = res["is_token_in_rank"].sum(axis=2).astype(np.float64)[..., None]
+    xf, f0, f1 = (b2f(a).astype(np.float64) for a in (inp["x"], b0, b1))
+    exact = n * xf + f0 + f1
+    mag = np.abs(n * xf) + np.abs(f0) + np.abs(f1)
+    got = b2f(out).astype(np.float64)
+    assert (np.abs(got - exact) <= 2.0 ** -8 * np.abs(exact) + 3 * 2.0 ** -24 * mag + 1e-30).all()
+    # and without the second bias it differs by exactly that bias, up to rounding
+    out0, _ = oracle.combine(res["recv_x"], res["send_pos"], bias=(b0, None))
+    got0 = b2f(out0).astype(np.float64)
+    assert (np.abs(got0 - (n * xf + f0)) <= 2.0 ** -8 * np.abs(n * xf + f0) + 2 * 2.0 ** -24 * mag + 1e-30).all()
+
+
+def test_fp8_input_rows_are_copied_by_send_pos():
+    rng = np.random.default_rng(9)
+    R, T, H = 3, 7, 256
+    q = rng.integers(0, 256, size=(R, T, H), dtype=np.uint8)
+    sc = rng.random((R, T, H // 128)).astype(np.float32)
+    in_rank = (rng.random((R, T, R)) < 0.5).astype(np.uint8)
+    pre = oracle.prefix(in_rank)
+    rq, rs = oracle.dispatch_rows_fp8(q, sc, pre["send_pos"])
+    rq2, rs2 = oracle.dispatch_rows_fp8(q, np.ascontiguousarray(sc.transpose(0, 2, 1)),
+                                        pre["send_pos"], col_major=True)
+    for d in range(R):
+        triples = sorted((s, t) for s in range(R) for t in range(T) if in_rank[s, t, d])
+        for row, (s, t) in enumerate(triples):
+            np.testing.assert_array_equal(rq[d, row], q[s, t])
+            np.testing.assert_array_equal(rs[d, row], sc[s, t])
+            np.testing.assert_array_equal(rs2[d, row], sc[s, t])
+    np.testing.assert_array_equal(rq, rq2)
+
+
 def test_combine_random_y_error_bound():
     rng = np.random.default_rng(3)
     R, T, H, E, K = 5, 40, 64, 20, 4

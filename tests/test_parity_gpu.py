@@ -451,3 +451,130 @@ def test_ll_full_size_sampled():
         pos = np.zeros((1, 1, K), np.int32)
         ro = oracle.ll_combine(ysmall, idx[s:s + 1, t:t + 1], wts[s:s + 1, t:t + 1], pos)
         np.testing.assert_array_equal(got[u], ro[0, 0])
+
+
+# ---------------------------------------------------------------------------
+# cached mode and the fixed worst-case receive capacity
+# ---------------------------------------------------------------------------
+
+def test_cached_dispatch_replays_the_handle():
+    """Re-dispatching with the handle reproduces recv_x; a new payload goes to
+    the same rows (legacy-test analysis page, cached dispatch check)."""
+    w = Workload("cache", R=6, T=300, H=136, E=24, K=4, masked_frac=0.1, seed=41)
+    inp = make(w)
+    xd, idd, wd = to_dev(inp["x"]), to_dev(inp["topk_idx"]), to_dev(inp["topk_weights"])
+    st = ep.new_status()
+    out = ep.ep_dispatch(xd, idd, wd, w.E, status=st)
+    first = out["recv_x"].clone()
+    again = ep.ep_dispatch_cached(xd, out["send_pos"], status=st)
+    x2 = make(Workload("cache2", R=6, T=300, H=136, E=24, K=4, seed=42))["x"]
+    other = ep.ep_dispatch_cached(to_dev(x2), out["send_pos"], status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rc = to_host(out["recv_count"])
+    for d in range(w.R):
+        assert torch.equal(again[d, :rc[d]].view(torch.int16), first[d, :rc[d]].view(torch.int16))
+    ref2 = oracle.dispatch_rows(x2, to_host(out["send_pos"]))
+    got2 = to_host(other)
+    for d in range(w.R):
+        np.testing.assert_array_equal(got2[d, :rc[d]], ref2[d, :rc[d]])
+
+
+def test_notify_then_cached_equals_dispatch():
+    w = Workload("split", R=8, T=260, H=256, E=64, K=8, seed=43)
+    inp = make(w)
+    xd, idd, wd = to_dev(inp["x"]), to_dev(inp["topk_idx"]), to_dev(inp["topk_weights"])
+    ref = ep.ep_dispatch(xd, idd, wd, w.E, expert_alignment=2)
+    h = ep.ep_notify_dispatch(idd, wd, w.T, w.R, w.E, expert_alignment=2)
+    rx = ep.ep_dispatch_cached(xd, h["send_pos"])
+    torch.cuda.synchronize()
+    for name in ("send_pos", "rank_prefix_matrix", "recv_count", "num_recv_tokens_per_expert"):
+        assert torch.equal(h[name], ref[name]), name
+    rc = to_host(ref["recv_count"])
+    for d in range(w.R):
+        n = rc[d]
+        assert torch.equal(rx[d, :n].view(torch.int16), ref["recv_x"][d, :n].view(torch.int16))
+        for name in ("recv_src_idx", "recv_topk_idx", "recv_topk_weights"):
+            assert torch.equal(h[name][d, :n], ref[name][d, :n]), name
+
+
+def test_worst_case_capacity_pads_recv_topk_idx():
+    """Fixed capacity = the pages' num_worst_tokens mode: rows past the receive
+    count hold recv_topk_idx == -1, and the real rows are the same as with an
+    exactly sized buffer."""
+    w = Workload("worst", R=4, T=200, H=64, E=16, K=3, seed=44)
+    inp = make(w)
+    xd, idd, wd = to_dev(inp["x"]), to_dev(inp["topk_idx"]), to_dev(inp["topk_weights"])
+    ref = oracle.normal_path(inp["x"], inp["topk_idx"], inp["topk_weights"], w.E)
+    exact = int(ref["recv_count"].max())
+    small = ep.ep_dispatch(xd, idd, wd, w.E, capacity=exact)
+    out = {"recv_topk_idx": torch.full((w.R, w.R * w.T, w.K), 7, dtype=torch.int64,
+                                       device="cuda")}
+    worst = ep.ep_dispatch(xd, idd, wd, w.E, out=out)
+    torch.cuda.synchronize()
+    rc = ref["recv_count"]
+    ri = to_host(worst["recv_topk_idx"])
+    for d in range(w.R):
+        assert (ri[d, rc[d]:] == -1).all()
+        np.testing.assert_array_equal(ri[d, :rc[d]], ref["recv_topk_idx"][d, :rc[d]])
+        assert torch.equal(worst["recv_x"][d, :rc[d]].view(torch.int16),
+                           small["recv_x"][d, :rc[d]].view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# FP8 input to normal dispatch; combine with bias
+# ---------------------------------------------------------------------------
+
+FP8_CASES = [
+    ("rowmajor_bulk", Workload("f1", R=4, T=300, H=512, E=16, K=3, seed=51), False),
+    ("rowmajor_unaligned", Workload("f2", R=5, T=140, H=384, E=20, K=2, seed=52), False),
+    ("colmajor", Workload("f3", R=4, T=257, H=512, E=8, K=2, seed=53), True),
+    ("colmajor_7168", Workload("f4", R=3, T=130, H=7168, E=12, K=4, seed=54), True),
+]
+
+
+@pytest.mark.parametrize("name,w,colmaj", FP8_CASES, ids=[c[0] for c in FP8_CASES])
+def test_fp8_input_dispatch(name, w, colmaj):
+    inp = make(w)
+    R, T, H = w.R, w.T, w.H
+    nb = H // 128
+    # realistic FP8 input: the oracle's per-token cast of the bf16 rows
+    q = np.zeros((R, T, H), np.uint8)
+    sc = np.zeros((R, T, nb), np.float32)
+    for s in range(R):
+        for t in range(T):
+            q[s, t], sc[s, t] = oracle.quantize_row(inp["x"][s, t])
+    sc_in = np.ascontiguousarray(sc.transpose(0, 2, 1)) if colmaj else sc
+    idd = to_dev(inp["topk_idx"])
+    h = ep.ep_notify_dispatch(idd, None, T, R, w.E)
+    st = ep.new_status()
+    rq, rs = ep.ep_dispatch_cached_fp8(to_dev(q), to_dev(sc_in), h["send_pos"],
+                                       scales_col_major=colmaj, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    sp = to_host(h["send_pos"])
+    eq, es = oracle.dispatch_rows_fp8(q, sc_in, sp, col_major=colmaj)
+    rc = to_host(h["recv_count"])
+    gq, gs = to_host(rq), to_host(rs)
+    for d in range(R):
+        np.testing.assert_array_equal(gq[d, :rc[d]], eq[d, :rc[d]])
+        np.testing.assert_array_equal(gs[d, :rc[d]], es[d, :rc[d]])
+
+
+def test_combine_with_bias():
+    w = Workload("bias", R=6, T=210, H=264, E=24, K=4, masked_frac=0.05, seed=55)
+    inp = make(w)
+    ref = oracle.normal_path(inp["x"], inp["topk_idx"], inp["topk_weights"], w.E)
+    b = make(Workload("b", R=6, T=210, H=264, E=24, K=4, seed=56))["x"]
+    b1 = make(Workload("b1", R=6, T=210, H=264, E=24, K=4, seed=57))["x"]
+    out = ep.ep_dispatch(to_dev(inp["x"]), to_dev(inp["topk_idx"]), to_dev(inp["topk_weights"]),
+                         w.E)
+    st = ep.new_status()
+    cx, _ = ep.ep_combine(out["recv_x"], out["send_pos"], bias=(to_dev(b), to_dev(b1)), status=st)
+    c0, _ = ep.ep_combine(out["recv_x"], out["send_pos"], bias=(to_dev(b), None), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    e2, _ = oracle.combine(ref["recv_x"], ref["send_pos"], bias=(b, b1))
+    e1, _ = oracle.combine(ref["recv_x"], ref["send_pos"], bias=(b, None))
+    np.testing.assert_array_equal(to_host(cx), e2)
+    np.testing.assert_array_equal(to_host(c0), e1)
