@@ -49,9 +49,9 @@ _SIGS = {
     "ep_dispatch_cached_fp8": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _P, _P, _P, _P]),
     "ep_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "ep_ll_workspace_bytes": (_Z, [_I, _I, _I]),
-    "ep_ll_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
-                            _P, _Z, _P, _P]),
-    "ep_ll_combine": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "ep_ll_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
+                            _P, _P, _Z, _P, _P]),
+    "ep_ll_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -64,6 +64,7 @@ EP_STATUS_CAPACITY = 2
 EP_STATUS_WAIT_TIMEOUT = 4
 EP_STATUS_BAD_POSITION = 8
 EP_DEBUG_SUPPRESS_PUBLISH = 1
+EP_LL_FP8, EP_LL_ROUND_SCALE, EP_LL_UE8M0 = 1, 2, 4
 
 
 class EPError(RuntimeError):
@@ -406,11 +407,14 @@ def ep_ll_workspace_bytes(num_ranks: int, num_tokens: int, num_experts: int) -> 
 
 
 def ep_ll_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int, *,
-                   use_fp8: bool = True, out: Optional[dict] = None,
-                   workspace: Optional[torch.Tensor] = None, status=None, stream=None) -> dict:
+                   use_fp8: bool = True, round_scale: bool = False, use_ue8m0: bool = False,
+                   rank_mask: Optional[torch.Tensor] = None,
+                   cumulative_local_expert_recv_stats: Optional[torch.Tensor] = None,
+                   out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None,
+                   status=None, stream=None) -> dict:
     """x bf16 [R, T, H] -> dict of recv_x (uint8 e4m3 or bf16 [R, E_l, R*T, H]),
-    recv_scales (fp32 [R, E_l, R*T, H/128] or None), recv_count, recv_src_info,
-    layout_range, ll_pos."""
+    recv_scales (fp32, or uint8 UE8M0, [R, E_l, R*T, H/128]; None for bf16),
+    recv_count, recv_src_info, layout_range, ll_pos."""
     R, T, H = x.shape
     K = topk_idx.shape[2]
     E = num_experts
@@ -418,6 +422,13 @@ def ep_ll_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int, *,
     dev = x.device
     _need(x, torch.bfloat16, (R, T, H), "x")
     _need(topk_idx, torch.int64, (R, T, K), "topk_idx")
+    if rank_mask is not None:
+        _need(rank_mask, torch.int32, (R,), "rank_mask")
+    if cumulative_local_expert_recv_stats is not None:
+        _need(cumulative_local_expert_recv_stats, torch.int32, (R, El),
+              "cumulative_local_expert_recv_stats")
+    flags = (EP_LL_FP8 if use_fp8 else 0) | (EP_LL_ROUND_SCALE if round_scale else 0) | \
+        (EP_LL_UE8M0 if use_ue8m0 else 0)
     o = dict(out or {})
 
     def get(name, shape, dtype):
@@ -428,7 +439,7 @@ def ep_ll_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int, *,
 
     get("recv_x", (R, El, R * T, H), torch.uint8 if use_fp8 else torch.bfloat16)
     if use_fp8:
-        get("recv_scales", (R, El, R * T, H // 128), torch.float32)
+        get("recv_scales", (R, El, R * T, H // 128), torch.uint8 if use_ue8m0 else torch.float32)
     else:
         o["recv_scales"] = None
     get("recv_count", (R, El), torch.int32)
@@ -439,16 +450,17 @@ def ep_ll_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int, *,
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     rc = _lib.ep_ll_dispatch(
-        _ptr(x), _ptr(topk_idx), R, T, H, K, E, 1 if use_fp8 else 0, _ptr(o["recv_x"]),
+        _ptr(x), _ptr(topk_idx), _ptr(rank_mask), R, T, H, K, E, flags, _ptr(o["recv_x"]),
         _ptr(o["recv_scales"]), _ptr(o["recv_count"]), _ptr(o["recv_src_info"]),
-        _ptr(o["layout_range"]), _ptr(o["ll_pos"]), _ptr(workspace), workspace.numel(),
-        _ptr(status), _stream(stream))
+        _ptr(o["layout_range"]), _ptr(o["ll_pos"]), _ptr(cumulative_local_expert_recv_stats),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
     _check(rc, "ep_ll_dispatch")
     return o
 
 
 def ep_ll_combine(y: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
-                  ll_pos: torch.Tensor, *, out: Optional[torch.Tensor] = None, status=None,
+                  ll_pos: torch.Tensor, *, rank_mask: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None, status=None,
                   stream=None) -> torch.Tensor:
     """y bf16 [R, E_l, R*T, H] -> out bf16 [R, T, H]."""
     R, El, cap, H = y.shape
@@ -462,7 +474,10 @@ def ep_ll_combine(y: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.T
     if out is None:
         out = torch.empty((R, T, H), dtype=torch.bfloat16, device=y.device)
     _need(out, torch.bfloat16, (R, T, H), "out")
-    rc = _lib.ep_ll_combine(_ptr(y), _ptr(topk_idx), _ptr(topk_weights), _ptr(ll_pos), R, T, H,
-                            K, E, _ptr(out), _ptr(status), _stream(stream))
+    if rank_mask is not None:
+        _need(rank_mask, torch.int32, (R,), "rank_mask")
+    rc = _lib.ep_ll_combine(_ptr(y), _ptr(topk_idx), _ptr(topk_weights), _ptr(ll_pos),
+                            _ptr(rank_mask), R, T, H, K, E, _ptr(out), _ptr(status),
+                            _stream(stream))
     _check(rc, "ep_ll_combine")
     return out

@@ -31,7 +31,9 @@ namespace {
 
 struct LLScanParams {
   const int64_t *topk_idx;
-  int R, T, K, E, cap, tiles_per_src, num_tiles;
+  const int32_t *mask;   // [R], non-zero = failed rank; nullptr = none
+  int32_t *stats;        // [E] cumulative received rows, or nullptr
+  int R, T, K, E, El, cap, tiles_per_src, num_tiles;
   int32_t *ll_pos;
   int32_t *recv_src_info;
   int32_t *layout_range;
@@ -61,9 +63,12 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   const int t = (tile % p.tiles_per_src) * kScanTile + tid;
   const bool valid = t < p.T;
   const size_t st = static_cast<size_t>(s) * p.T + t;
+  // a failed (masked) source rank sends nothing
+  const bool src_ok = p.mask == nullptr || p.mask[s] == 0;
 
   // Distinct valid experts of this token (a repeated expert keeps only its
-  // first slot in `col`; `ev` keeps every valid id).
+  // first slot in `col`; `ev` keeps every valid id).  Experts on a failed
+  // rank are dropped.
   int ev[kMaxTopk], col[kMaxTopk], rnk[kMaxTopk];
   bool bad = false;
 #pragma unroll
@@ -74,6 +79,7 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
     if (valid && k < p.K) {
       const int64_t e = p.topk_idx[st * p.K + k];
       if (e >= 0 && e < p.E) {
+        if (!src_ok || (p.mask != nullptr && p.mask[static_cast<int>(e) / p.El] != 0)) continue;
         ev[k] = static_cast<int>(e);
         bool dup = false;
 #pragma unroll
@@ -124,7 +130,10 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
     const size_t o = (static_cast<size_t>(c) * p.R + s) * 2;
     if (first_of_src) p.layout_range[o] = static_cast<int>(excl);
     // rows source s owns: the tiles of s add their counts (zeroed on the host)
-    if (run != 0) atomicAdd(&p.layout_range[o + 1], run);
+    if (run != 0) {
+      atomicAdd(&p.layout_range[o + 1], run);
+      if (p.stats != nullptr) atomicAdd(&p.stats[c], run);
+    }
     if (tile == p.num_tiles - 1) p.recv_count[c] = static_cast<int>(excl) + run;
   }
   __syncthreads();
@@ -204,9 +213,9 @@ template <bool kFP8>
 __global__ void __launch_bounds__(kLLThreads)
     ll_dispatch_kernel(const uint8_t *__restrict__ x, const int64_t *__restrict__ topk_idx,
                        const int32_t *__restrict__ ll_pos, long num_tok, int H, int K, int E,
-                       int cap, LLSmem plan, uint8_t *__restrict__ recv,
-                       float *__restrict__ scales, int32_t *status,
-                       unsigned long long timeout_ns) {
+                       int cap, int round_scale, int ue8m0, LLSmem plan,
+                       uint8_t *__restrict__ recv, void *__restrict__ scales_out,
+                       int32_t *status, unsigned long long timeout_ns) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -217,8 +226,10 @@ __global__ void __launch_bounds__(kLLThreads)
   const int nblk = H >> 7;
   const int row_in = 2 * H;
   const int pay = kFP8 ? H : 2 * H;
-  const int sc_bytes = nblk * 4;
+  const int sc_bytes = ue8m0 ? nblk : nblk * 4;  // fp32 scales or UE8M0 exponent bytes
   const bool bulk_scales = (sc_bytes & 15) == 0;
+  float *scales = static_cast<float *>(scales_out);
+  uint8_t *scales8 = static_cast<uint8_t *>(scales_out);
   const long n = static_cast<long>(blockIdx.x) < num_tok
                      ? (num_tok - 1 - blockIdx.x) / gridDim.x + 1
                      : 0;
@@ -262,10 +273,10 @@ __global__ void __launch_bounds__(kLLThreads)
         const int e2 = __shfl_sync(0xffffffffu, e, k2);
         dup |= (k2 < lane && e2 == e);
       }
-      if (e >= 0 && !dup) {
+      if (e >= 0 && !dup) {  // pos -1: the slot was dropped (failed rank)
         if (pos >= 0 && pos < cap)
           dst = static_cast<long>(e) * cap + pos;
-        else
+        else if (pos != -1)
           report(status, EP_STATUS_BAD_POSITION);
       }
       // FP8: the output buffer of token i - 2 must have been read by its stores
@@ -299,7 +310,18 @@ __global__ void __launch_bounds__(kLLThreads)
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
         amax = fmaxf(amax, 1e-4f);
-        const float inv = __fdiv_rn(448.0f, amax);
+        float inv, scale;
+        uint32_t ebits = 0;
+        if (round_scale) {
+          // smallest power of two >= amax / 448, and its exact reciprocal
+          const uint32_t u = __float_as_uint(__fdiv_rn(amax, 448.0f));
+          ebits = (u >> 23) + ((u & 0x7FFFFFu) != 0u ? 1u : 0u);
+          scale = __uint_as_float(ebits << 23);
+          inv = __uint_as_float((254u - ebits) << 23);
+        } else {
+          inv = __fdiv_rn(448.0f, amax);
+          scale = __fdiv_rn(amax, 448.0f);
+        }
         if (act) {
           uint2 qq;
           qq.x = cvt_e4m3x4(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv), __fmul_rn(f[2], inv),
@@ -307,7 +329,12 @@ __global__ void __launch_bounds__(kLLThreads)
           qq.y = cvt_e4m3x4(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv), __fmul_rn(f[6], inv),
                             __fmul_rn(f[7], inv));
           reinterpret_cast<uint2 *>(q)[c] = qq;
-          if ((c & 15) == 0) sc[c >> 4] = __fdiv_rn(amax, 448.0f);
+          if ((c & 15) == 0) {
+            if (ue8m0)
+              reinterpret_cast<uint8_t *>(sc)[c >> 4] = static_cast<uint8_t>(ebits);
+            else
+              sc[c >> 4] = scale;
+          }
         }
       }
       fence_proxy_async_smem();
@@ -319,7 +346,10 @@ __global__ void __launch_bounds__(kLLThreads)
         bulk_s2g(recv + dst * pay, src, static_cast<uint32_t>(pay));
         if constexpr (kFP8) {
           if (bulk_scales)
-            bulk_s2g(scales + dst * nblk, sc, static_cast<uint32_t>(sc_bytes));
+            bulk_s2g(scales8 + dst * sc_bytes, sc, static_cast<uint32_t>(sc_bytes));
+          else if (ue8m0)
+            for (int j = 0; j < nblk; ++j)
+              scales8[dst * nblk + j] = reinterpret_cast<const uint8_t *>(sc)[j];
           else
             for (int j = 0; j < nblk; ++j) scales[dst * nblk + j] = sc[j];
         }
@@ -357,8 +387,8 @@ constexpr int kLLCombineWarps = 8;
 __global__ void __launch_bounds__(kLLCombineWarps * 32)
     ll_combine_kernel(const uint8_t *__restrict__ y, const int64_t *__restrict__ topk_idx,
                       const float *__restrict__ topk_w, const int32_t *__restrict__ ll_pos,
-                      long num_tok, int H, int K, int E, int cap, int nseg,
-                      uint8_t *__restrict__ out, int32_t *status) {
+                      const int32_t *__restrict__ mask, long num_tok, int T, int H, int K, int E,
+                      int cap, int nseg, uint8_t *__restrict__ out, int32_t *status) {
   __shared__ int64_t s_row[kLLCombineWarps][kMaxTopk];
   __shared__ float s_w[kLLCombineWarps][kMaxTopk];
   const int lane = threadIdx.x & 31;
@@ -366,6 +396,7 @@ __global__ void __launch_bounds__(kLLCombineWarps * 32)
   const uint32_t lt = lanemask_lt();
   const int nvec = H >> 3;
   const int seg_vec = (nvec + nseg - 1) / nseg;
+  const int El = E / (cap / T);  // cap = R * T
   const long row_bytes = static_cast<long>(H) * 2;
   const long items = num_tok * nseg;
   for (long it = static_cast<long>(blockIdx.x) * kLLCombineWarps + warp; it < items;
@@ -375,15 +406,16 @@ __global__ void __launch_bounds__(kLLCombineWarps * 32)
     bool take = false;
     long row = 0;
     float w = 0.f;
-    if (lane < K) {
+    const bool src_ok = mask == nullptr || mask[u / T] == 0;
+    if (lane < K && src_ok) {
       const int64_t e = topk_idx[u * K + lane];
-      if (e >= 0 && e < E) {
+      if (e >= 0 && e < E && (mask == nullptr || mask[e / El] == 0)) {
         const int pos = ll_pos[u * K + lane];
         if (pos >= 0 && pos < cap) {
           take = true;
           row = e * cap + pos;
           w = topk_w[u * K + lane];
-        } else if (sg == 0) {
+        } else if (sg == 0 && pos != -1) {  // -1: dropped at dispatch
           report(status, EP_STATUS_BAD_POSITION);
         }
       }
@@ -442,15 +474,22 @@ extern "C" EP_API size_t ep_ll_workspace_bytes(int num_ranks, int num_tokens, in
   return scan_workspace_bytes(tiles, num_experts, 0);
 }
 
-extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx, int num_ranks,
-                                     int num_tokens, int hidden, int num_topk, int num_experts,
-                                     int use_fp8, void *recv_x, float *recv_scales,
-                                     int32_t *recv_count, int32_t *recv_src_info,
-                                     int32_t *layout_range, int32_t *ll_pos, void *workspace,
-                                     size_t workspace_bytes, int32_t *status,
+extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
+                                     const int32_t *rank_mask, int num_ranks, int num_tokens,
+                                     int hidden, int num_topk, int num_experts, int fp8_flags,
+                                     void *recv_x, void *recv_scales, int32_t *recv_count,
+                                     int32_t *recv_src_info, int32_t *layout_range,
+                                     int32_t *ll_pos, int32_t *cumulative_local_expert_recv_stats,
+                                     void *workspace, size_t workspace_bytes, int32_t *status,
                                      cudaStream_t stream) {
   using namespace ep;
   const int R = num_ranks, T = num_tokens, H = hidden, K = num_topk, E = num_experts;
+  const int use_fp8 = (fp8_flags & EP_LL_FP8) != 0;
+  const int round_scale = (fp8_flags & EP_LL_ROUND_SCALE) != 0;
+  const int ue8m0 = (fp8_flags & EP_LL_UE8M0) != 0;
+  if ((fp8_flags & ~(EP_LL_FP8 | EP_LL_ROUND_SCALE | EP_LL_UE8M0)) != 0 ||
+      (round_scale && !use_fp8) || (ue8m0 && !round_scale))
+    return EP_ERR_INVALID_ARG;
   if (R < 1 || R > kMaxRanks || T < 0 || K < 1 || K > kMaxTopk || E < 1 || E > kMaxExperts ||
       E % R != 0 || H < 8 || (use_fp8 ? (H % 128 != 0) : (H % 8 != 0)))
     return EP_ERR_INVALID_ARG;
@@ -468,6 +507,9 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx, int
   if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(recv_x) & 15u) ||
       (use_fp8 && (reinterpret_cast<uintptr_t>(recv_scales) & 15u)))
     return EP_ERR_INVALID_ARG;
+  if (cumulative_local_expert_recv_stats != nullptr &&
+      (reinterpret_cast<uintptr_t>(cumulative_local_expert_recv_stats) & 3u))
+    return EP_ERR_INVALID_ARG;
   const size_t need = ep_ll_workspace_bytes(R, T, E);
   if (workspace == nullptr || workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(workspace) & 15u))
@@ -484,6 +526,9 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx, int
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   LLScanParams p;
   p.topk_idx = topk_idx;
+  p.mask = rank_mask;
+  p.stats = cumulative_local_expert_recv_stats;
+  p.El = E / R;
   p.R = R;
   p.T = T;
   p.K = K;
@@ -518,21 +563,21 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx, int
   if (use_fp8)
     ll_dispatch_kernel<true><<<static_cast<unsigned>(grid), kLLThreads, smem, stream>>>(
         static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, H, K, E,
-        static_cast<int>(cap), plan, static_cast<uint8_t *>(recv_x), recv_scales, status,
-        wc.timeout_ns);
+        static_cast<int>(cap), round_scale, ue8m0, plan, static_cast<uint8_t *>(recv_x),
+        recv_scales, status, wc.timeout_ns);
   else
     ll_dispatch_kernel<false><<<static_cast<unsigned>(grid), kLLThreads, smem, stream>>>(
         static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, H, K, E,
-        static_cast<int>(cap), plan, static_cast<uint8_t *>(recv_x), nullptr, status,
+        static_cast<int>(cap), 0, 0, plan, static_cast<uint8_t *>(recv_x), nullptr, status,
         wc.timeout_ns);
   return launch_status();
 }
 
 extern "C" EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
                                     const float *topk_weights, const int32_t *ll_pos,
-                                    int num_ranks, int num_tokens, int hidden, int num_topk,
-                                    int num_experts, void *out, int32_t *status,
-                                    cudaStream_t stream) {
+                                    const int32_t *rank_mask, int num_ranks, int num_tokens,
+                                    int hidden, int num_topk, int num_experts, void *out,
+                                    int32_t *status, cudaStream_t stream) {
   using namespace ep;
   const int R = num_ranks, T = num_tokens, H = hidden, K = num_topk, E = num_experts;
   if (R < 1 || R > kMaxRanks || T < 0 || K < 1 || K > kMaxTopk || E < 1 || E > kMaxExperts ||
@@ -557,7 +602,7 @@ extern "C" EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
   const long items = num_tok * nseg;
   const long grid = std::min<long>((items + kLLCombineWarps - 1) / kLLCombineWarps, resident);
   ll_combine_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(
-      static_cast<const uint8_t *>(y), topk_idx, topk_weights, ll_pos, num_tok, H, K, E,
-      static_cast<int>(cap), nseg, static_cast<uint8_t *>(out), status);
+      static_cast<const uint8_t *>(y), topk_idx, topk_weights, ll_pos, rank_mask, num_tok, T, H,
+      K, E, static_cast<int>(cap), nseg, static_cast<uint8_t *>(out), status);
   return launch_status();
 }

@@ -65,6 +65,12 @@ extern "C" {
 #define EP_STATUS_WAIT_TIMEOUT     4  /* a bounded wait ran out; results are invalid   */
 #define EP_STATUS_BAD_POSITION     8  /* a send_pos / ll_pos entry outside its buffer  */
 
+/* Flags of ep_ll_dispatch (fp8_flags). */
+#define EP_LL_FP8          1  /* e4m3 payload with one scale per 128 channels      */
+#define EP_LL_ROUND_SCALE  2  /* scales rounded up to powers of two (needs FP8)    */
+#define EP_LL_UE8M0        4  /* scales stored as UE8M0 exponent bytes (needs
+                                 ROUND_SCALE): value 2^(byte - 127)              */
+
 /* Debug flags for ep_set_debug_flags(). */
 #define EP_DEBUG_SUPPRESS_PUBLISH  1u /* scan tiles publish nothing, so every tile but
                                          the first waits until its limit runs out:
@@ -302,25 +308,39 @@ EP_API size_t ep_ll_workspace_bytes(int num_ranks, int num_tokens,
  * overflow.
  *   x              bf16 [R, T, H]; H % 128 == 0 for FP8, H % 8 == 0 for bf16
  *   topk_idx       int64 [R, T, K]
- *   use_fp8        1: recv_x is e4m3 [R, E_l, R*T, H] and recv_scales fp32
- *                  [R, E_l, R*T, H/128] with, per 128-channel block,
+ *   rank_mask      int32 [R] or NULL: non-zero marks a failed rank (the pages'
+ *                  shrink mode, low_latency_query_mask_buffer): a failed source
+ *                  rank sends nothing, and slots whose expert lives on a
+ *                  failed rank are dropped (ll_pos -1, not counted)
+ *   fp8_flags      0: recv_x is bf16 [R, E_l, R*T, H], recv_scales unused;
+ *                  EP_LL_FP8: recv_x is e4m3 [R, E_l, R*T, H] and recv_scales
+ *                  fp32 [R, E_l, R*T, H/128] with, per 128-channel block,
  *                  amax' = max(max|x|, 1e-4), q = e4m3_rne_satfinite(x *
  *                  (448 / amax')), scale = amax' / 448;
- *                  0: recv_x is bf16 [R, E_l, R*T, H], recv_scales unused
+ *                  | EP_LL_ROUND_SCALE: scale = the smallest power of two
+ *                  >= amax' / 448 and q = e4m3(x * (1 / scale)) (exact
+ *                  reciprocal); | EP_LL_UE8M0: recv_scales is uint8
+ *                  [R, E_l, R*T, H/128] holding each scale's biased exponent
  *   recv_count     out int32 [R, E_l]: rows of each local expert
  *   recv_src_info  out int32 [R, E_l, R*T]: source token index of each row
  *   layout_range   out int32 [R, E_l, R, 2]: (first row, rows) per source rank
  *   ll_pos         out int32 [R, T, K]: slab row of each slot, -1 if the slot
- *                  is unselected or invalid (a repeated expert in a token
- *                  shares its first slot's row)
+ *                  is unselected, invalid or dropped (a repeated expert in a
+ *                  token shares its first slot's row)
+ *   cumulative_local_expert_recv_stats  int32 [R, E_l] or NULL: each call adds
+ *                  its recv_count (the pages' cumulative per-expert counter)
  *   workspace      ep_ll_workspace_bytes(R, T, E) bytes, any content
+ * H is limited by shared memory (three staged input rows per CTA): FP8 needs
+ * H <= 28672 and bf16 H <= 38720; larger returns EP_ERR_UNSUPPORTED.
  */
 EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
-                          int num_ranks, int num_tokens, int hidden,
-                          int num_topk, int num_experts, int use_fp8,
-                          void *recv_x, float *recv_scales,
-                          int32_t *recv_count, int32_t *recv_src_info,
-                          int32_t *layout_range, int32_t *ll_pos,
+                          const int32_t *rank_mask, int num_ranks,
+                          int num_tokens, int hidden, int num_topk,
+                          int num_experts, int fp8_flags, void *recv_x,
+                          void *recv_scales, int32_t *recv_count,
+                          int32_t *recv_src_info, int32_t *layout_range,
+                          int32_t *ll_pos,
+                          int32_t *cumulative_local_expert_recv_stats,
                           void *workspace, size_t workspace_bytes,
                           int32_t *status, cudaStream_t stream);
 
@@ -334,17 +354,21 @@ EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
  *                  ep_ll_dispatch laid out its slabs; H % 8 == 0
  *   topk_idx, topk_weights  int64 / fp32 [R, T, K]
  *   ll_pos         int32 [R, T, K] from ep_ll_dispatch
+ *   rank_mask      int32 [R] or NULL: slots of failed source ranks and slots
+ *                  whose expert lives on a failed rank contribute nothing
  *   out            bf16 [R, T, H]: bf16_rne(acc), acc = +0.0 then, for k
  *                  ascending over valid slots, acc = fmaf(float(y[e][ll_pos]),
  *                  w[k], acc)
- * A slot with a valid expert but ll_pos outside [0, R*T) is skipped and sets
+ * A slot with ll_pos -1 (dropped at dispatch) contributes nothing; a valid
+ * expert with ll_pos outside [-1, R*T) is skipped and sets
  * EP_STATUS_BAD_POSITION.
  */
 EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
                          const float *topk_weights, const int32_t *ll_pos,
-                         int num_ranks, int num_tokens, int hidden,
-                         int num_topk, int num_experts, void *out,
-                         int32_t *status, cudaStream_t stream);
+                         const int32_t *rank_mask, int num_ranks,
+                         int num_tokens, int hidden, int num_topk,
+                         int num_experts, void *out, int32_t *status,
+                         cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -77,6 +77,12 @@ def lib() -> ctypes.CDLL:
         L.orc_dispatch_rows_fp8.argtypes = [_P, _P, _I, _P, _I, _I, _I, _I, _P, _P]
         L.orc_ll_layout.restype = _L
         L.orc_ll_layout.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P]
+        L.orc_quantize_row_ex.restype = None
+        L.orc_quantize_row_ex.argtypes = [_P, _I, _I, _P, _P, _P]
+        L.orc_ll_layout_masked.restype = _L
+        L.orc_ll_layout_masked.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P]
+        L.orc_ll_combine_masked.restype = None
+        L.orc_ll_combine_masked.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _L, _P]
         L.orc_quantize_row.restype = None
         L.orc_quantize_row.argtypes = [_P, _I, _P, _P]
         L.orc_ll_dispatch_rows.restype = None
@@ -256,7 +262,7 @@ def dispatch_rows_fp8(x_q: np.ndarray, x_scales: np.ndarray, send_pos: np.ndarra
     return rq, rs
 
 
-def ll_layout(topk_idx: np.ndarray, num_experts: int) -> dict:
+def ll_layout(topk_idx: np.ndarray, num_experts: int, mask=None) -> dict:
     idx = _c(topk_idx, np.int64)
     R, T, K = idx.shape
     E = num_experts
@@ -265,7 +271,9 @@ def ll_layout(topk_idx: np.ndarray, num_experts: int) -> dict:
     lr = np.zeros((E, R, 2), np.int32)
     pos = np.zeros((R, T, K), np.int32)
     rsi = np.full((E, R * T), -1, np.int32)
-    bad = lib().orc_ll_layout(_ptr(idx), R, T, K, E, _ptr(count), _ptr(lr), _ptr(pos), _ptr(rsi))
+    m = None if mask is None else _c(mask, np.int32)
+    bad = lib().orc_ll_layout_masked(_ptr(idx), _ptr(m), R, T, K, E, _ptr(count), _ptr(lr),
+                                     _ptr(pos), _ptr(rsi))
     return {"recv_count": count.reshape(R, El), "layout_range": lr.reshape(R, El, R, 2),
             "ll_pos": pos, "recv_src_info": rsi.reshape(R, El, R * T), "bad_slots": int(bad)}
 
@@ -277,6 +285,17 @@ def quantize_row(x_row: np.ndarray):
     s = np.zeros((H // 128,), np.float32)
     lib().orc_quantize_row(_ptr(xr), H, _ptr(q), _ptr(s))
     return q, s
+
+
+def quantize_row_ex(x_row: np.ndarray, round_scale: bool = False):
+    """-> (q uint8 [H], scales fp32 [H/128], ue8m0 uint8 [H/128] or None)."""
+    xr = _c(x_row, np.uint16)
+    H = xr.shape[-1]
+    q = np.zeros((H,), np.uint8)
+    s = np.zeros((H // 128,), np.float32)
+    u = np.zeros((H // 128,), np.uint8) if round_scale else None
+    lib().orc_quantize_row_ex(_ptr(xr), H, 1 if round_scale else 0, _ptr(q), _ptr(s), _ptr(u))
+    return q, s, u
 
 
 def ll_dispatch_rows(x, topk_idx, ll_pos, num_experts: int, use_fp8: bool = True,
@@ -311,7 +330,7 @@ def dequant_rows(q: np.ndarray, scales: np.ndarray) -> np.ndarray:
     return y
 
 
-def ll_combine(y, topk_idx, topk_weights, ll_pos, tokens=None) -> np.ndarray:
+def ll_combine(y, topk_idx, topk_weights, ll_pos, tokens=None, mask=None) -> np.ndarray:
     """y [R,El,R*T,H] bf16 bits -> out [R,T,H] bf16 bits."""
     yy = _c(y, np.uint16)
     idx = _c(topk_idx, np.int64)
@@ -323,8 +342,9 @@ def ll_combine(y, topk_idx, topk_weights, ll_pos, tokens=None) -> np.ndarray:
     assert idx.shape[0] == R and cap == R * T, "y must be [R, E_l, R*T, H] for topk_idx [R, T, K]"
     out = np.zeros((R, T, H), np.uint16)
     tk, nt = _tokens(tokens)
-    lib().orc_ll_combine(_ptr(yy), _ptr(idx), _ptr(w), _ptr(pos), R, T, H, K, R * El,
-                         _ptr(tk), nt, _ptr(out))
+    m = None if mask is None else _c(mask, np.int32)
+    lib().orc_ll_combine_masked(_ptr(yy), _ptr(idx), _ptr(w), _ptr(pos), _ptr(m), R, T, H, K,
+                                R * El, _ptr(tk), nt, _ptr(out))
     return out
 
 

@@ -418,12 +418,30 @@ void orc_combine(const uint16_t *y, const float *recv_w, const int32_t *send_pos
  *   recv_src_info[E][R*T]     token index t of each row
  * Returns the number of invalid slots (outside [-1, E)).
  */
+long orc_ll_layout_masked(const int64_t *topk_idx, const int32_t *mask, int R, int T,
+                          int K, int E, int32_t *count, int32_t *layout_range,
+                          int32_t *ll_pos, int32_t *recv_src_info);
+
 long orc_ll_layout(const int64_t *topk_idx, int R, int T, int K, int E,
                    int32_t *count, int32_t *layout_range, int32_t *ll_pos,
                    int32_t *recv_src_info)
 {
+    return orc_ll_layout_masked(topk_idx, NULL, R, T, K, E, count, layout_range, ll_pos,
+                                recv_src_info);
+}
+
+/*
+ * As orc_ll_layout, with an optional rank mask [R] (non-zero = the rank has
+ * failed, the pages' shrink mode): a masked source rank sends nothing and a
+ * slot whose expert lives on a masked rank is dropped; both read ll_pos -1.
+ */
+long orc_ll_layout_masked(const int64_t *topk_idx, const int32_t *mask, int R, int T,
+                          int K, int E, int32_t *count, int32_t *layout_range,
+                          int32_t *ll_pos, int32_t *recv_src_info)
+{
     long bad = 0;
     int cap = R * T;
+    int El = E / R;
     for (int e = 0; e < E; ++e)
         count[e] = 0;
     for (int s = 0; s < R; ++s) {
@@ -439,6 +457,10 @@ long orc_ll_layout(const int64_t *topk_idx, int R, int T, int K, int E,
                 }
                 if (e < -1 || e >= E) {
                     bad++;
+                    ll_pos[st * K + k] = -1;
+                    continue;
+                }
+                if (mask && (mask[s] || mask[e / El])) {
                     ll_pos[st * K + k] = -1;
                     continue;
                 }
@@ -472,6 +494,49 @@ long orc_ll_layout(const int64_t *topk_idx, int R, int T, int K, int E,
  *   q[i]  = e4m3(x[i] * inv)    (fp32 multiply, then nearest-even, saturate)
  *   scale = amax / 448          (fp32 division)
  */
+/*
+ * Variants of the per-128-channel cast:
+ *   round_scale = 0: as orc_quantize_row;
+ *   round_scale = 1: the scale amax' / 448 is rounded UP to a power of two
+ *                    2^e (so |x| / scale <= 448), and x is multiplied by the
+ *                    exact reciprocal 2^-e;
+ * scales_f32 (fp32 scale per block) and/or scales_ue8m0 (the scale's biased
+ * exponent byte, value 2^(byte - 127); only with round_scale) may be NULL.
+ */
+void orc_quantize_row_ex(const uint16_t *x, int H, int round_scale, uint8_t *q,
+                         float *scales_f32, uint8_t *scales_ue8m0)
+{
+    for (int b = 0; b < H / 128; ++b) {
+        float amax = 0.0f;
+        for (int i = 0; i < 128; ++i) {
+            float a = fabsf(orc_bf16_to_f32(x[b * 128 + i]));
+            if (a > amax)
+                amax = a;
+        }
+        if (amax < 1e-4f)
+            amax = 1e-4f;
+        float scale, inv;
+        if (round_scale) {
+            /* smallest power of two >= amax / 448 (a normal float here) */
+            double sf = (double)(amax / 448.0f);
+            int ex;
+            double fr = frexp(sf, &ex);            /* sf = fr * 2^ex, fr in [0.5,1) */
+            int e = (fr == 0.5) ? ex - 1 : ex;     /* 2^e >= sf, 2^(e-1) < sf */
+            scale = (float)ldexp(1.0, e);
+            inv = (float)ldexp(1.0, -e);
+            if (scales_ue8m0)
+                scales_ue8m0[b] = (uint8_t)(e + 127);
+        } else {
+            inv = 448.0f / amax;
+            scale = amax / 448.0f;
+        }
+        for (int i = 0; i < 128; ++i)
+            q[b * 128 + i] = orc_f32_to_e4m3(orc_bf16_to_f32(x[b * 128 + i]) * inv);
+        if (scales_f32)
+            scales_f32[b] = scale;
+    }
+}
+
 void orc_quantize_row(const uint16_t *x, int H, uint8_t *q, float *scales)
 {
     for (int b = 0; b < H / 128; ++b) {
@@ -553,12 +618,29 @@ void orc_dequant_rows(const uint8_t *q, const float *scales, long rows, int H,
  *     acc = fmaf(float(y[idx][ll_pos][h]), w[s][t][k], acc)
  * y is [E][R*T][H] bf16 bits.  tokens: optional flat token list.
  */
+void orc_ll_combine_masked(const uint16_t *y, const int64_t *topk_idx,
+                           const float *topk_weights, const int32_t *ll_pos,
+                           const int32_t *mask, int R, int T, int H, int K, int E,
+                           const int64_t *tokens, long ntokens, uint16_t *out);
+
 void orc_ll_combine(const uint16_t *y, const int64_t *topk_idx,
                     const float *topk_weights, const int32_t *ll_pos,
                     int R, int T, int H, int K, int E,
                     const int64_t *tokens, long ntokens, uint16_t *out)
 {
+    orc_ll_combine_masked(y, topk_idx, topk_weights, ll_pos, NULL, R, T, H, K, E, tokens,
+                          ntokens, out);
+}
+
+/* As orc_ll_combine; with a rank mask, slots of masked source ranks and slots
+ * whose expert lives on a masked rank contribute nothing. */
+void orc_ll_combine_masked(const uint16_t *y, const int64_t *topk_idx,
+                           const float *topk_weights, const int32_t *ll_pos,
+                           const int32_t *mask, int R, int T, int H, int K, int E,
+                           const int64_t *tokens, long ntokens, uint16_t *out)
+{
     int cap = R * T;
+    int El = E / R;
     long n = tokens ? ntokens : (long)R * T;
     for (long i = 0; i < n; ++i) {
         long st = tokens ? tokens[i] : i;
@@ -568,6 +650,8 @@ void orc_ll_combine(const uint16_t *y, const int64_t *topk_idx,
                 int64_t e = topk_idx[(size_t)st * K + k];
                 int32_t row = ll_pos[(size_t)st * K + k];
                 if (e < 0 || e >= E || row < 0 || row >= cap)
+                    continue;
+                if (mask && (mask[st / T] || mask[e / El]))
                     continue;
                 float v = orc_bf16_to_f32(y[((size_t)e * cap + row) * H + h]);
                 acc = fmaf(v, topk_weights[(size_t)st * K + k], acc);

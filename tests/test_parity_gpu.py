@@ -578,3 +578,69 @@ def test_combine_with_bias():
     e1, _ = oracle.combine(ref["recv_x"], ref["send_pos"], bias=(b, None))
     np.testing.assert_array_equal(to_host(cx), e2)
     np.testing.assert_array_equal(to_host(c0), e1)
+
+
+# ---------------------------------------------------------------------------
+# low-latency variants: power-of-two / UE8M0 scales, failed ranks, statistics
+# ---------------------------------------------------------------------------
+
+RS_CASES = [
+    ("h384_plain_scales", Workload("r1", R=4, T=70, H=384, E=16, K=4, seed=61)),
+    ("h2048_bulk_ue8m0", Workload("r2", R=3, T=130, H=2048, E=12, K=3, seed=62)),
+    ("h7168", Workload("r3", R=4, T=40, H=7168, E=16, K=4, seed=63)),
+]
+
+
+@pytest.mark.parametrize("ue8m0", [False, True])
+@pytest.mark.parametrize("name,w", RS_CASES, ids=[c[0] for c in RS_CASES])
+def test_ll_round_scale(name, w, ue8m0):
+    inp = make(w)
+    x, idx = inp["x"], inp["topk_idx"]
+    R, T, H, E = w.R, w.T, w.H, w.E
+    El = E // R
+    ref = oracle.ll_layout(idx, E)
+    st = ep.new_status()
+    out = ep.ep_ll_dispatch(to_dev(x), to_dev(idx), E, use_fp8=True, round_scale=True,
+                            use_ue8m0=ue8m0, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(to_host(out["ll_pos"]), ref["ll_pos"])
+    q = to_host(out["recv_x"])
+    sc = to_host(out["recv_scales"])
+    for s in range(R):
+        for t in range(T):
+            qr, sr, ur = oracle.quantize_row_ex(x[s, t], round_scale=True)
+            for k in range(w.K):
+                e = int(idx[s, t, k])
+                p = int(ref["ll_pos"][s, t, k])
+                d, j = divmod(e, El)
+                np.testing.assert_array_equal(q[d, j, p], qr)
+                np.testing.assert_array_equal(sc[d, j, p], ur if ue8m0 else sr)
+
+
+def test_ll_failed_ranks_and_cumulative_stats():
+    w = Workload("mk", R=8, T=150, H=256, E=32, K=4, masked_frac=0.05, seed=64)
+    inp = make(w)
+    x, idx, wts = inp["x"], inp["topk_idx"], inp["topk_weights"]
+    R, E = w.R, w.E
+    mask = np.array([0, 1, 0, 0, 0, 1, 0, 0], np.int32)   # ranks 1 and 5 failed
+    ref = oracle.ll_layout(idx, E, mask=mask)
+    md = to_dev(mask)
+    stats = torch.zeros((R, E // R), dtype=torch.int32, device="cuda")
+    st = ep.new_status()
+    xd, idd, wd = to_dev(x), to_dev(idx), to_dev(wts)
+    for _ in range(2):
+        out = ep.ep_ll_dispatch(xd, idd, E, use_fp8=False, rank_mask=md,
+                                cumulative_local_expert_recv_stats=stats, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(to_host(out["recv_count"]), ref["recv_count"])
+    np.testing.assert_array_equal(to_host(out["layout_range"]), ref["layout_range"])
+    np.testing.assert_array_equal(to_host(out["ll_pos"]), ref["ll_pos"])
+    np.testing.assert_array_equal(to_host(stats), 2 * ref["recv_count"])
+    slab, _ = oracle.ll_dispatch_rows(x, idx, ref["ll_pos"], E, use_fp8=False)
+    ro = oracle.ll_combine(slab, idx, wts, ref["ll_pos"], mask=mask)
+    co = ep.ep_ll_combine(to_dev(slab), idd, wd, out["ll_pos"], rank_mask=md, status=st)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_host(co), ro)
+    assert (to_host(co)[1] == 0).all() and (to_host(co)[5] == 0).all()
