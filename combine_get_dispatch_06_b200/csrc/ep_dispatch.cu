@@ -266,6 +266,104 @@ constexpr int kCopyStages = 4;
 constexpr int kCopyChunkMax = 4096;
 constexpr int kCopyMaxCtasPerSm = 2;
 
+// bf16 rows only (the headline path): the row scatter described above.
+template <int S>
+__global__ void __launch_bounds__(kMaxRanks)
+    dispatch_copy_rows_kernel(const uint8_t *__restrict__ x, const int32_t *__restrict__ send_pos,
+                         uint8_t *__restrict__ recv_x, int R, long num_tok, int row_bytes,
+                         int chunk_bytes, int nchunks, int stage_stride, int cap,
+                         int32_t *status, unsigned long long timeout_ns) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
+  uint8_t *buf = smem + 128;
+  const int tid = threadIdx.x;
+  const int d = tid;
+
+  const long ntok_cta =
+      static_cast<long>(blockIdx.x) < num_tok ? (num_tok - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const long nitems = ntok_cta * nchunks;
+
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  auto token_of = [&](long i) -> long {
+    return static_cast<long>(blockIdx.x) + (i / nchunks) * static_cast<long>(gridDim.x);
+  };
+  auto issue_load = [&](long i, int stg) {
+    const long u = token_of(i);
+    const int off = static_cast<int>(i % nchunks) * chunk_bytes;
+    const int nb = min(chunk_bytes, row_bytes - off);
+    mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(nb));
+    bulk_g2s_hint(buf + stg * stage_stride, x + u * row_bytes + off, static_cast<uint32_t>(nb),
+                  &bars[stg], l2_evict_first_policy());
+  };
+  auto load_pos = [&](long i) -> int {
+    return d < R ? __ldg(send_pos + token_of(i) * R + d) : -1;
+  };
+
+  int sp[S];
+#pragma unroll
+  for (int k = 0; k < S; ++k) sp[k] = -1;
+#pragma unroll
+  for (int k = 0; k < S - 1; ++k) {
+    if (k < nitems) {
+      if (tid == 0) issue_load(k, k);
+      sp[k] = load_pos(k);
+    }
+  }
+
+  bool all_ok = true;
+  long stop = nitems;  // first item whose load may still be in flight on failure
+  for (long base = 0; base < nitems && all_ok; base += S) {
+    const uint32_t parity = static_cast<uint32_t>((base / S) & 1);
+#pragma unroll
+    for (int st = 0; st < S; ++st) {
+      const long i = base + st;
+      if (i >= nitems) break;
+      const bool ok = mbar_wait_bounded(&bars[st], parity, timeout_ns);
+      const int chunk = static_cast<int>(i % nchunks);
+      if (ok && sp[st] >= 0) {  // sp < 0: no copy to this rank
+        if (sp[st] < cap) {
+          const int off = chunk * chunk_bytes;
+          const int nb = min(chunk_bytes, row_bytes - off);
+          bulk_s2g(recv_x + (static_cast<long>(d) * cap + sp[st]) * row_bytes + off,
+                   buf + st * stage_stride, static_cast<uint32_t>(nb));
+        } else if (chunk == 0) {
+          report(status, EP_STATUS_CAPACITY);
+        }
+      }
+      bulk_commit();
+      bulk_wait_read<1>();
+      all_ok = __syncthreads_and(ok) != 0;
+      if (!all_ok) {
+        stop = i;
+        break;
+      }
+      const long j = i + S - 1;
+      const int ps = (st + S - 1) % S;
+      if (j < nitems) {
+        if (tid == 0) issue_load(j, ps);
+        sp[ps] = load_pos(j);
+      }
+    }
+  }
+  bulk_wait_all<0>();
+  if (!all_ok) {
+    report(status, EP_STATUS_WAIT_TIMEOUT);
+    if (tid == 0) {
+      // drain loads still in flight before the CTA's shared memory goes away
+      const long end = min(nitems, stop + S - 1);
+      for (long k = stop; k < end; ++k)
+        (void)mbar_wait_bounded(&bars[k % S], static_cast<uint32_t>((k / S) & 1), timeout_ns);
+    }
+  }
+}
+
+
 // How the scales row of a token reaches shared memory.
 enum ScaleMode : int {
   kScalesNone = 0,      // bf16 input: no scales
@@ -288,14 +386,14 @@ struct CopyArgs {
   unsigned long long timeout_ns;
 };
 
-template <int S>
-__global__ void __launch_bounds__(kMaxRanks) dispatch_copy_kernel(CopyArgs a) {
+template <int S, bool kScales>
+__global__ void __launch_bounds__(kMaxRanks) dispatch_copy_planes_kernel(CopyArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
   uint8_t *buf = smem + 128;
   const int tid = threadIdx.x;
   const int d = tid;
-  const int ipt = a.nchunks + (a.sc_mode != kScalesNone ? 1 : 0);  // items per token
+  const int ipt = a.nchunks + (kScales ? 1 : 0);  // items per token
   const int sc_bytes = a.nblk * 4;
 
   const long ntok_cta = static_cast<long>(blockIdx.x) < a.num_tok
@@ -310,40 +408,48 @@ __global__ void __launch_bounds__(kMaxRanks) dispatch_copy_kernel(CopyArgs a) {
   }
   __syncthreads();
 
-  auto token_of = [&](long i) -> long {
-    return static_cast<long>(blockIdx.x) + (i / ipt) * static_cast<long>(gridDim.x);
-  };
-  auto issue_load = [&](long i, int stg) {  // thread 0
-    const long u = token_of(i);
-    const int sub = static_cast<int>(i % ipt);
-    if (sub < a.nchunks) {
-      const int off = sub * a.chunk_bytes;
-      const int nb = min(a.chunk_bytes, a.row_bytes - off);
-      mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(nb));
-      bulk_g2s_hint(buf + stg * a.stage_stride, a.x + u * a.row_bytes + off,
-                    static_cast<uint32_t>(nb), &bars[stg], l2_evict_first_policy());
-    } else if (a.sc_mode == kScalesBulk) {
-      mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(sc_bytes));
-      bulk_g2s(buf + stg * a.stage_stride, a.xs + u * a.nblk, static_cast<uint32_t>(sc_bytes),
-               &bars[stg]);
-    } else {
-      mbar_arrive(&bars[stg]);  // gathered by the threads when the item is used
+  // Item cursors, advanced one item at a time (no divisions on the path):
+  // `is_*` for the next item to load, `cs_*` for the next item to use.
+  long is_tok = blockIdx.x;  // global token index of the item to load
+  int is_sub = 0;
+  long cs_tok = blockIdx.x;
+  int cs_sub = 0;
+  int sp[S];                 // send_pos of the item held by each stage
+  // Threads past R read rank R-1's entry and ignore it: the load then needs
+  // no select, so its result lands in sp[] untouched until S-1 items later
+  // (a select or a register copy would stall the warp on the load).
+  const bool mine = d < a.R;
+  const int dd = mine ? d : a.R - 1;
+
+  auto issue_next = [&](int stg) -> int {  // all threads; returns this thread's pos
+    if (tid == 0) {
+      if (!kScales || is_sub < a.nchunks) {
+        const int off = is_sub * a.chunk_bytes;
+        const int nb = min(a.chunk_bytes, a.row_bytes - off);
+        mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(nb));
+        bulk_g2s_hint(buf + stg * a.stage_stride, a.x + is_tok * a.row_bytes + off,
+                      static_cast<uint32_t>(nb), &bars[stg], l2_evict_first_policy());
+      } else if (a.sc_mode == kScalesBulk) {
+        mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(sc_bytes));
+        bulk_g2s(buf + stg * a.stage_stride, a.xs + is_tok * a.nblk,
+                 static_cast<uint32_t>(sc_bytes), &bars[stg]);
+      } else {
+        mbar_arrive(&bars[stg]);  // gathered by the threads when the item is used
+      }
     }
-  };
-  auto load_pos = [&](long i) -> int {
-    return d < a.R ? __ldg(a.send_pos + token_of(i) * a.R + d) : -1;
+    const int pos = __ldg(a.send_pos + is_tok * a.R + dd);
+    if (++is_sub == ipt) {
+      is_sub = 0;
+      is_tok += gridDim.x;
+    }
+    return pos;
   };
 
-  int sp[S];
 #pragma unroll
   for (int k = 0; k < S; ++k) sp[k] = -1;
 #pragma unroll
-  for (int k = 0; k < S - 1; ++k) {
-    if (k < nitems) {
-      if (tid == 0) issue_load(k, k);
-      sp[k] = load_pos(k);
-    }
-  }
+  for (int k = 0; k < S - 1; ++k)
+    if (k < nitems) sp[k] = issue_next(k);
 
   bool all_ok = true;
   long stop = nitems;  // first item whose load may still be in flight on failure
@@ -354,27 +460,27 @@ __global__ void __launch_bounds__(kMaxRanks) dispatch_copy_kernel(CopyArgs a) {
       const long i = base + st;
       if (i >= nitems) break;
       const bool ok = mbar_wait_bounded(&bars[st], parity, a.timeout_ns);
-      const int sub = static_cast<int>(i % ipt);
+      const int sub = cs_sub;
       uint8_t *stage = buf + st * a.stage_stride;
-      if (sub == a.nchunks && a.sc_mode >= kScalesGatherRow) {  // uniform in the CTA
-        const long u = token_of(i);
+      if (kScales && sub == a.nchunks && a.sc_mode >= kScalesGatherRow) {  // uniform in CTA
         float *f = reinterpret_cast<float *>(stage);
         for (int j = tid; j < a.nblk; j += blockDim.x) {
           if (a.sc_mode == kScalesGatherRow) {
-            f[j] = __ldg(a.xs + u * a.nblk + j);
+            f[j] = __ldg(a.xs + cs_tok * a.nblk + j);
           } else {
-            const long s = u / a.T, t = u % a.T;
+            const long s = cs_tok / a.T, t = cs_tok % a.T;
             f[j] = __ldg(a.xs + (s * a.nblk + j) * a.T + t);
           }
         }
         fence_proxy_async_smem();
         __syncthreads();
       }
-      if (ok && sp[st] >= 0) {  // sp < 0: no copy to this rank
-        const long row = static_cast<long>(d) * a.cap + sp[st];
-        if (sp[st] >= a.cap) {
+      const int pos = sp[st];
+      if (ok && mine && pos >= 0) {  // pos < 0: no copy to this rank
+        const long row = static_cast<long>(d) * a.cap + pos;
+        if (pos >= a.cap) {
           if (sub == 0) report(a.status, EP_STATUS_CAPACITY);
-        } else if (sub < a.nchunks) {
+        } else if (!kScales || sub < a.nchunks) {
           const int off = sub * a.chunk_bytes;
           const int nb = min(a.chunk_bytes, a.row_bytes - off);
           bulk_s2g(a.recv_x + row * a.row_bytes + off, stage, static_cast<uint32_t>(nb));
@@ -386,18 +492,18 @@ __global__ void __launch_bounds__(kMaxRanks) dispatch_copy_kernel(CopyArgs a) {
         }
       }
       bulk_commit();
+      if (++cs_sub == ipt) {
+        cs_sub = 0;
+        cs_tok += gridDim.x;
+      }
       bulk_wait_read<1>();
       all_ok = __syncthreads_and(ok) != 0;
       if (!all_ok) {
         stop = i;
         break;
       }
-      const long j = i + S - 1;
       const int ps = (st + S - 1) % S;
-      if (j < nitems) {
-        if (tid == 0) issue_load(j, ps);
-        sp[ps] = load_pos(j);
-      }
+      if (i + S - 1 < nitems) sp[ps] = issue_next(ps);
     }
   }
   bulk_wait_all<0>();
@@ -407,8 +513,7 @@ __global__ void __launch_bounds__(kMaxRanks) dispatch_copy_kernel(CopyArgs a) {
       // drain loads still in flight before the CTA's shared memory goes away
       const long end = min(nitems, stop + S - 1);
       for (long k = stop; k < end; ++k)
-        (void)mbar_wait_bounded(&bars[k % S], static_cast<uint32_t>((k / S) & 1),
-                                a.timeout_ns);
+        (void)mbar_wait_bounded(&bars[k % S], static_cast<uint32_t>((k / S) & 1), a.timeout_ns);
     }
   }
 }
@@ -530,12 +635,20 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
   a.timeout_ns = wait_config().timeout_ns;
   const size_t smem = 128 + static_cast<size_t>(kCopyStages) * a.stage_stride;
   const int threads = 32 * ((R + 31) / 32);
-  const void *fn = reinterpret_cast<const void *>(dispatch_copy_kernel<kCopyStages>);
+  const void *fn = xs != nullptr
+                       ? reinterpret_cast<const void *>(dispatch_copy_planes_kernel<kCopyStages, true>)
+                       : reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStages>);
   if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
   const long grid = std::min<long>(
       a.num_tok,
       static_cast<long>(std::min(kCopyMaxCtasPerSm, ctas_per_sm(fn, threads, smem))) * num_sms());
-  dispatch_copy_kernel<kCopyStages><<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
+  if (xs != nullptr)
+    dispatch_copy_planes_kernel<kCopyStages, true>
+        <<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
+  else
+    dispatch_copy_rows_kernel<kCopyStages><<<static_cast<unsigned>(grid), threads, smem, stream>>>(
+        a.x, a.send_pos, a.recv_x, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
+        a.stage_stride, a.cap, a.status, a.timeout_ns);
   return launch_status();
 }
 
