@@ -120,6 +120,22 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   const bool valid = t < p.T;
   const size_t st = static_cast<size_t>(s) * p.T + t;
 
+  // ---- the token's top-k ids and weights, loaded once, all at once --------
+  const bool meta =
+      valid && p.topk_idx != nullptr && (p.recv_idx != nullptr || p.recv_w != nullptr);
+  const bool need_idx = valid && p.topk_idx != nullptr;
+  int64_t ek[kMaxTopk];
+  float wk[kMaxTopk];
+#pragma unroll
+  for (int k = 0; k < kMaxTopk; ++k) {
+    ek[k] = -1;
+    wk[k] = 0.f;
+    if (need_idx && k < p.K) {
+      ek[k] = p.topk_idx[st * p.K + k];
+      if (meta && p.recv_w != nullptr) wk[k] = p.topk_w[st * p.K + k];
+    }
+  }
+
   // ---- routing bits of this token --------------------------------------
   uint32_t *my_mask = s_mask + tid * p.W;
   for (int w = 0; w < p.W; ++w) my_mask[w] = 0u;
@@ -130,10 +146,11 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
         if (ir[d]) my_mask[d >> 5] |= 1u << (d & 31);
     }
     if (p.topk_idx != nullptr && (p.in_rank == nullptr || count_experts)) {
-      const int64_t *row = p.topk_idx + st * p.K;
       bool bad = false;
-      for (int k = 0; k < p.K; ++k) {
-        const int64_t e = row[k];
+#pragma unroll
+      for (int k = 0; k < kMaxTopk; ++k) {
+        if (k >= p.K) break;
+        const int64_t e = ek[k];
         if (e == -1) continue;
         if (e < -1 || e >= p.E) {
           bad = true;
@@ -196,19 +213,6 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   __syncthreads();
 
   // ---- pass 2: positions, handle and received metadata -------------------
-  const bool meta =
-      valid && p.topk_idx != nullptr && (p.recv_idx != nullptr || p.recv_w != nullptr);
-  int64_t ek[kMaxTopk];
-  float wk[kMaxTopk];
-#pragma unroll
-  for (int k = 0; k < kMaxTopk; ++k) {
-    ek[k] = -1;
-    wk[k] = 0.f;
-    if (meta && k < p.K) {
-      ek[k] = p.topk_idx[st * p.K + k];
-      if (p.recv_w != nullptr) wk[k] = p.topk_w[st * p.K + k];
-    }
-  }
   const uint32_t lt = lanemask_lt();
   bool overflow = false;
   for (int d0 = 0; d0 < p.R; d0 += 32) {
@@ -532,6 +536,28 @@ extern "C" EP_API size_t ep_dispatch_workspace_bytes(int num_ranks, int num_toke
 namespace ep {
 namespace {
 
+// recv_topk_idx rows from recv_count[d] to cap - 1 := -1 (grid: x over the
+// rows, y over the destination ranks).  16-byte stores when a row of K int64
+// is a multiple of 16 bytes.
+__global__ void __launch_bounds__(256)
+    pad_recv_idx_kernel(const int32_t *__restrict__ recv_count, int cap, int K,
+                        int64_t *__restrict__ recv_idx) {
+  const int d = blockIdx.y;
+  const long first = min(max(recv_count[d], 0), cap);
+  int64_t *base = recv_idx + static_cast<long>(d) * cap * K;
+  const long lo = first * K, hi = static_cast<long>(cap) * K;  // in int64 elements
+  const long step = static_cast<long>(gridDim.x) * blockDim.x;
+  if ((K & 1) == 0) {
+    const longlong2 v = make_longlong2(-1, -1);
+    for (long i = lo / 2 + static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; i < hi / 2;
+         i += step)
+      reinterpret_cast<longlong2 *>(base)[i] = v;
+  } else {
+    for (long i = lo + static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; i < hi; i += step)
+      base[i] = -1;
+  }
+}
+
 // A2 (+ received metadata): the scan kernel.  Arguments already checked.
 int notify_impl(const int64_t *topk_idx, const float *topk_weights,
                 const uint8_t *is_token_in_rank, int R, int T, int K, int E, int align, int cap,
@@ -556,12 +582,6 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   const int Ectr = topk_idx != nullptr ? E : 0;
   const size_t need = ep_dispatch_workspace_bytes(R, T, Ectr);
   if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return EP_ERR_CUDA;
-  // rows past the receive count read -1 (fixed worst-case capacity): every
-  // int64 of all-ones bytes is -1, and the scan overwrites the real rows
-  if (recv_topk_idx != nullptr && cap > 0 &&
-      cudaMemsetAsync(recv_topk_idx, 0xFF, sizeof(int64_t) * R * static_cast<size_t>(cap) * K,
-                      stream) != cudaSuccess)
-    return EP_ERR_CUDA;
 
   const int tiles_per_src = (T + kScanTile - 1) / kScanTile;
   const long num_tiles = static_cast<long>(R) * tiles_per_src;
@@ -596,7 +616,15 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   p.timeout_ns = wc.timeout_ns;
   p.flags = wc.flags;
   dispatch_scan_kernel<<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
-  return launch_status();
+  if (launch_status() != EP_OK) return EP_ERR_CUDA;
+  // rows past the receive count read -1 (fixed worst-case capacity)
+  if (recv_topk_idx != nullptr && cap > 0) {
+    const long words = static_cast<long>(cap) * K / ((K & 1) == 0 ? 2 : 1);
+    const int bx = static_cast<int>(std::min<long>((words + 255) / 256, 64));
+    pad_recv_idx_kernel<<<dim3(bx, R), 256, 0, stream>>>(recv_count, cap, K, recv_topk_idx);
+    return launch_status();
+  }
+  return EP_OK;
 }
 
 // A3 rows: the bulk-copy kernel.  Arguments already checked.  `xs` (FP8
