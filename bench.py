@@ -256,16 +256,23 @@ def load_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
-    """sha1 of the CUDA sources, to tell whether recorded counters still apply."""
-    import glob
+# the source files each timed kernel is built from (for staleness checks)
+KERNEL_SOURCES = {
+    "dispatch_copy_kernel": ["ep_dispatch.cu", "ep_scan.cuh", "ep_common.cuh"],
+    "combine_kernel": ["ep_combine.cu", "ep_common.cuh"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """sha1 of the CUDA sources of `kernel`, to tell whether recorded counters
+    still describe the kernel that runs."""
     import hashlib
 
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "combine_get_dispatch_06_b200", "csrc")
-    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
-        h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(f.encode())
+        with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()
 
@@ -273,19 +280,20 @@ def kernel_source_hash() -> str:
 def recorded_traffic(kernel: str, T: int):
     """DRAM bytes (read + write) per launch of `kernel` on the normal workload,
     from the ncu capture summarised in profiles/dram_traffic_normal.md -- or
-    None if that capture is of another build of the kernels."""
+    None if that capture is of another build of the kernel."""
+    import re
+
     path = os.path.join(ROOT, "profiles", "dram_traffic_normal.md")
     try:
         text = open(path).read()
     except OSError:
         return None
-    import re
-
-    m = re.search(r"source_sha1:\s*([0-9a-f]{40})", text)
-    if not m or m.group(1) != kernel_source_hash() or T != CONFIGS["normal"].T:
+    if T != CONFIGS["normal"].T:
         return None
-    m = re.search(rf"{kernel}\s*\|\s*traffic_bytes_per_launch\s*\|\s*(\d+)", text)
-    return int(m.group(1)) if m else None
+    m = re.search(rf"\|\s*{kernel}\s*\|\s*(\d+)\s*\|\s*([0-9a-f]{{40}})\s*\|", text)
+    if not m or m.group(2) != kernel_source_hash(kernel):
+        return None
+    return int(m.group(1))
 
 
 def to_dev_bf16(a: np.ndarray, device):
