@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
 #pragma unroll
   for (int k = 0; k < kMaxTopk; ++k)
     if (col[k] >= 0) rnk[k] = __popc(s_lanes[warp][col[k]] & lt);
+  __syncthreads();  // every warp's lane masks are complete before they are counted
   for (int c = tid; c < p.E; c += kScanTile)
 #pragma unroll
     for (int w = 0; w < kScanWarps; ++w) s_whist[w][c] = __popc(s_lanes[w][c]);

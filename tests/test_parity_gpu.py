@@ -644,3 +644,88 @@ def test_ll_failed_ranks_and_cumulative_stats():
     torch.cuda.synchronize()
     np.testing.assert_array_equal(to_host(co), ro)
     assert (to_host(co)[1] == 0).all() and (to_host(co)[5] == 0).all()
+
+
+# ---------------------------------------------------------------------------
+# limits of the ABI: K = 16, E = 512, R > 32 on every path, empty inputs
+# ---------------------------------------------------------------------------
+
+def test_dispatch_combine_k16_e512():
+    w = Workload("lim", R=16, T=150, H=136, E=512, K=16, masked_frac=0.05, seed=71)
+    inp = make(w)
+    x, idx, wts = inp["x"], inp["topk_idx"], inp["topk_weights"]
+    ref = oracle.normal_path(x, idx, wts, w.E, alignment=4)
+    st = ep.new_status()
+    out = ep.ep_dispatch(to_dev(x), to_dev(idx), to_dev(wts), w.E, expert_alignment=4, status=st)
+    cx, cw = ep.ep_combine(out["recv_x"], out["send_pos"], out["recv_topk_weights"], status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    check_dispatch(out, ref, w.R, w.K)
+    np.testing.assert_array_equal(to_host(cx), ref["combined_x"])
+    np.testing.assert_array_equal(to_host(cw), ref["combined_topk_weights"])
+
+
+def test_ll_k16_e512():
+    w = Workload("llim", R=8, T=70, H=256, E=512, K=16, masked_frac=0.05, seed=72)
+    inp = make(w)
+    x, idx, wts = inp["x"], _dup_slots(inp["topk_idx"], 0.2, 72), inp["topk_weights"]
+    ref = oracle.ll_layout(idx, w.E)
+    rq, rs = oracle.ll_dispatch_rows(x, idx, ref["ll_pos"], w.E, use_fp8=True)
+    st = ep.new_status()
+    idd = to_dev(idx)
+    out = ep.ep_ll_dispatch(to_dev(x), idd, w.E, use_fp8=True, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(to_host(out["ll_pos"]), ref["ll_pos"])
+    np.testing.assert_array_equal(to_host(out["recv_count"]), ref["recv_count"])
+    np.testing.assert_array_equal(to_host(out["layout_range"]), ref["layout_range"])
+    q, sc = to_host(out["recv_x"]), to_host(out["recv_scales"])
+    El = w.E // w.R
+    for d in range(w.R):
+        for j in range(El):
+            n = ref["recv_count"][d, j]
+            np.testing.assert_array_equal(q[d, j, :n], rq[d, j, :n])
+            np.testing.assert_array_equal(sc[d, j, :n], rs[d, j, :n])
+    y = oracle.dequant_rows(rq, rs)
+    co = ep.ep_ll_combine(to_dev(y), idd, to_dev(wts), out["ll_pos"], status=st)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_host(co), oracle.ll_combine(y, idx, wts, ref["ll_pos"]))
+
+
+def test_fp8_input_dispatch_r40_multiwarp():
+    w = Workload("f40", R=40, T=20, H=256, E=80, K=4, seed=73)
+    inp = make(w)
+    R, T, H = w.R, w.T, w.H
+    q = np.zeros((R, T, H), np.uint8)
+    sc = np.zeros((R, T, H // 128), np.float32)
+    for s in range(R):
+        for t in range(T):
+            q[s, t], sc[s, t] = oracle.quantize_row(inp["x"][s, t])
+    h = ep.ep_notify_dispatch(to_dev(inp["topk_idx"]), None, T, R, w.E)
+    st = ep.new_status()
+    rq, rs = ep.ep_dispatch_cached_fp8(to_dev(q), to_dev(sc), h["send_pos"], status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    eq, es = oracle.dispatch_rows_fp8(q, sc, to_host(h["send_pos"]))
+    rc = to_host(h["recv_count"])
+    for d in range(R):
+        np.testing.assert_array_equal(to_host(rq)[d, :rc[d]], eq[d, :rc[d]])
+        np.testing.assert_array_equal(to_host(rs)[d, :rc[d]], es[d, :rc[d]])
+
+
+def test_empty_inputs_everywhere():
+    R, H, E, K = 4, 256, 16, 2
+    x = torch.empty((R, 0, H), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((R, 0, K), dtype=torch.int64, device="cuda")
+    wt = torch.empty((R, 0, K), dtype=torch.float32, device="cuda")
+    ll = ep.ep_ll_dispatch(x, idx, E, use_fp8=True)
+    y = torch.empty((R, E // R, 0, H), dtype=torch.bfloat16, device="cuda")
+    co = ep.ep_ll_combine(y, idx, wt, ll["ll_pos"])
+    sp = torch.empty((R, 0, R), dtype=torch.int32, device="cuda")
+    rx = ep.ep_dispatch_cached(x, sp, capacity=0)
+    q = torch.empty((R, 0, H), dtype=torch.uint8, device="cuda")
+    s = torch.empty((R, 0, H // 128), dtype=torch.float32, device="cuda")
+    rq, rs = ep.ep_dispatch_cached_fp8(q, s, sp, capacity=0)
+    torch.cuda.synchronize()
+    assert (to_host(ll["recv_count"]) == 0).all() and (to_host(ll["layout_range"]) == 0).all()
+    assert co.numel() == 0 and rx.numel() == 0 and rq.numel() == 0
