@@ -263,11 +263,16 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
 // until its own bulk stores from that stage have finished reading it.
 // ---------------------------------------------------------------------------
 
-// Launch shape, chosen by a sweep on B200 at R=8, H=7168 (stages x chunk x
-// CTAs per SM): the row scatter is fastest with ~28 KB in flight per SM;
-// deeper pipelines oversubscribe HBM with this write-heavy mix and lose 5-7%.
+// Launch shape, from sweeps on B200 (stages x chunk x CTAs per SM), 2 CTAs
+// per SM in both cases:
+//  - rows > 8 KB (R=8, H=7168): ~3.5 KB chunks, 4 stages (~28 KB in flight per
+//    SM); deeper pipelines oversubscribe HBM with this write-heavy mix (-1..7%);
+//  - rows <= 8 KB (R=16, H=4096, skewed routing): one chunk per row, 8 stages;
+//    20% faster there than the long-row shape.
 constexpr int kCopyStages = 4;
+constexpr int kCopyStagesShort = 8;
 constexpr int kCopyChunkMax = 4096;
+constexpr int kCopyShortRow = 8192;
 constexpr int kCopyMaxCtasPerSm = 2;
 
 // bf16 rows only (the headline path): the row scatter described above.
@@ -644,7 +649,8 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
   a.cap = cap;
   a.num_tok = static_cast<long>(R) * T;
   a.row_bytes = row_bytes;
-  a.nchunks = (row_bytes + kCopyChunkMax - 1) / kCopyChunkMax;
+  const bool short_rows = row_bytes <= kCopyShortRow;
+  a.nchunks = short_rows ? 1 : (row_bytes + kCopyChunkMax - 1) / kCopyChunkMax;
   a.chunk_bytes = ((row_bytes + a.nchunks - 1) / a.nchunks + 15) & ~15;
   a.nblk = xs != nullptr ? nblk : 0;
   const int sc_bytes = a.nblk * 4;
@@ -661,22 +667,35 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
   a.stage_stride = (std::max(a.chunk_bytes, sc_bytes) + 127) & ~127;
   a.status = status;
   a.timeout_ns = wait_config().timeout_ns;
-  const size_t smem = 128 + static_cast<size_t>(kCopyStages) * a.stage_stride;
+  const int stages = short_rows ? kCopyStagesShort : kCopyStages;
+  const size_t smem = 128 + static_cast<size_t>(stages) * a.stage_stride;
   const int threads = 32 * ((R + 31) / 32);
-  const void *fn = xs != nullptr
-                       ? reinterpret_cast<const void *>(dispatch_copy_planes_kernel<kCopyStages, true>)
-                       : reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStages>);
+  const void *fn;
+  if (xs != nullptr)
+    fn = short_rows ? reinterpret_cast<const void *>(dispatch_copy_planes_kernel<kCopyStagesShort, true>)
+                    : reinterpret_cast<const void *>(dispatch_copy_planes_kernel<kCopyStages, true>);
+  else
+    fn = short_rows ? reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStagesShort>)
+                    : reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStages>);
   if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
   const long grid = std::min<long>(
       a.num_tok,
       static_cast<long>(std::min(kCopyMaxCtasPerSm, ctas_per_sm(fn, threads, smem))) * num_sms());
-  if (xs != nullptr)
-    dispatch_copy_planes_kernel<kCopyStages, true>
-        <<<static_cast<unsigned>(grid), threads, smem, stream>>>(a);
-  else
-    dispatch_copy_rows_kernel<kCopyStages><<<static_cast<unsigned>(grid), threads, smem, stream>>>(
+  const dim3 g(static_cast<unsigned>(grid)), b(threads);
+  if (xs != nullptr) {
+    if (short_rows)
+      dispatch_copy_planes_kernel<kCopyStagesShort, true><<<g, b, smem, stream>>>(a);
+    else
+      dispatch_copy_planes_kernel<kCopyStages, true><<<g, b, smem, stream>>>(a);
+  } else if (short_rows) {
+    dispatch_copy_rows_kernel<kCopyStagesShort><<<g, b, smem, stream>>>(
         a.x, a.send_pos, a.recv_x, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
         a.stage_stride, a.cap, a.status, a.timeout_ns);
+  } else {
+    dispatch_copy_rows_kernel<kCopyStages><<<g, b, smem, stream>>>(
+        a.x, a.send_pos, a.recv_x, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
+        a.stage_stride, a.cap, a.status, a.timeout_ns);
+  }
   return launch_status();
 }
 
