@@ -2,8 +2,10 @@
 """Benchmark: normal-mode MoE token routing (layout -> dispatch -> combine) on
 8 simulated ranks x 4096 tokens x 7168 hidden (bf16), top-8 of 256 experts.
 
-One step = ep_get_dispatch_layout + ep_dispatch + ep_combine over one batch of
-seeded synthetic input (identity experts: combine reads the dispatched rows).
+One step = ep_notify_dispatch with the fused layout (A1 + A2 in one kernel),
+ep_dispatch_cached (the row copy; notify + cached == ep_dispatch) and
+ep_combine, over one batch of seeded synthetic input (identity experts:
+combine reads the dispatched rows).
 Prints ONE JSON line (rank 0).  The headline value is algorithmic HBM GB/s of
 dispatch+combine (bytes the method must move, per step, divided by the step
 time); tokens/s and the share of 8 TB/s ride along.
@@ -456,16 +458,19 @@ def run_ours(args) -> None:
     wsp = torch.empty(ep.ep_dispatch_workspace_bytes(R, T, E), dtype=torch.uint8, device=device)
     status = ep.new_status(device)
 
+    out["num_tokens_per_rank"] = ntpr
+    out["num_tokens_per_expert"] = ntpe
+    out["is_token_in_rank"] = inr
+
     def step(ev=None):
-        # ep_dispatch == ep_notify_dispatch + ep_dispatch_cached; the two halves
-        # are called separately so that the row-copy kernel gets its own events
+        # layout (A1) is fused into the notify scan (A2): one kernel returns the
+        # layout and the handle.  ep_dispatch == ep_notify_dispatch +
+        # ep_dispatch_cached; the two halves are called separately so that the
+        # row-copy kernel gets its own events.
         if ev is not None:
             ev[0].record(stream)
-        ep.ep_get_dispatch_layout(idx, E, R, num_tokens_per_rank=ntpr, num_tokens_per_expert=ntpe,
-                                  is_token_in_rank=inr, status=status)
-        if ev is not None:
             ev[1].record(stream)
-        ep.ep_notify_dispatch(idx, wt, T, R, E, is_token_in_rank=inr, out=out, workspace=wsp,
+        ep.ep_notify_dispatch(idx, wt, T, R, E, with_layout=True, out=out, workspace=wsp,
                               status=status)
         if ev is not None:
             ev[2].record(stream)
@@ -504,7 +509,6 @@ def run_ours(args) -> None:
     barrier(device)
     clocks = sampler.stop()
     ms_local = t_start.elapsed_time(t_end) / args.steps
-    lay_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     notify_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     copy_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     comb_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
@@ -563,7 +567,7 @@ def run_ours(args) -> None:
                    "l2": "inputs larger than L2 (x 470 MB, recv_x 2.5 GB written); no flush"},
         "tokens_per_s": agg["tokens_per_s"],
         "pct_of_8TBps": 100.0 * agg["gbs"] / (SPEC_HBM_GBS * ws),
-        "phases_ms": {"layout": lay_ms, "dispatch": disp_ms, "dispatch_notify": notify_ms,
+        "phases_ms": {"dispatch": disp_ms, "dispatch_notify_with_layout": notify_ms,
                       "dispatch_copy": copy_ms, "combine": comb_ms},
         "bytes_per_step": {"dispatch": bytes_d, "combine": bytes_c, "copies": N},
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
@@ -573,7 +577,7 @@ def run_ours(args) -> None:
                      if peak_kind == "measured" else "fallback 6.65 TB/s"},
         "e2e": {"value": e2e["gbs"], "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e["ms_per_step"]},
-        "gpu_launches": 4 * args.steps,   # layout, scan, copy, combine per step
+        "gpu_launches": 4 * args.steps,   # scan (+layout), pad, copy, combine per step
         "clocks": clocks,
     }
     if ws == 1 and rank == 0 and not args.no_extra and T == CONFIGS["normal"].T:

@@ -42,7 +42,7 @@ _SIGS = {
     "ep_dispatch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                          _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P]),
     "ep_notify_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I,
-                                _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P]),
+                                _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P, _P]),
     "ep_dispatch_cached": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "ep_dispatch_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                  _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -229,9 +229,13 @@ def ep_notify_dispatch(topk_idx: Optional[torch.Tensor], topk_weights: Optional[
                        is_token_in_rank: Optional[torch.Tensor] = None,
                        expert_alignment: int = 1, capacity: Optional[int] = None,
                        out: Optional[dict] = None, with_metadata: bool = True,
+                       with_layout: bool = False,
                        workspace: Optional[torch.Tensor] = None, status=None,
                        stream=None) -> dict:
-    """The first half of ep_dispatch: handle + received metadata (no rows)."""
+    """The first half of ep_dispatch: handle + received metadata (no rows).
+    with_layout (routing from topk_idx only): also return the layout,
+    num_tokens_per_rank [R, R], num_tokens_per_expert [R, E],
+    is_token_in_rank bool [R, T, R], from the same kernel."""
     R, T = num_ranks, num_tokens
     src = topk_idx if topk_idx is not None else is_token_in_rank
     dev = src.device
@@ -256,6 +260,10 @@ def ep_notify_dispatch(topk_idx: Optional[torch.Tensor], topk_weights: Optional[
         get("num_recv_tokens_per_expert", (R, E // R), torch.int32)
         if topk_weights is not None:
             get("recv_topk_weights", (R, cap, K), torch.float32)
+    if with_layout:
+        get("num_tokens_per_rank", (R, R), torch.int32)
+        get("num_tokens_per_expert", (R, E), torch.int32)
+        get("is_token_in_rank", (R, T, R), torch.bool)
     if topk_idx is not None:
         _need(topk_idx, torch.int64, (R, T, K), "topk_idx")
     if topk_weights is not None:
@@ -271,6 +279,9 @@ def ep_notify_dispatch(topk_idx: Optional[torch.Tensor], topk_weights: Optional[
         _ptr(o.get("recv_topk_weights") if meta else None), _ptr(o["recv_src_idx"]),
         _ptr(o["rank_prefix_matrix"]), _ptr(o["recv_count"]),
         _ptr(o.get("num_recv_tokens_per_expert") if meta else None), _ptr(o["send_pos"]),
+        _ptr(o.get("num_tokens_per_rank") if with_layout else None),
+        _ptr(o.get("num_tokens_per_expert") if with_layout else None),
+        _ptr(o.get("is_token_in_rank") if with_layout else None),
         _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream))
     _check(rc, "ep_notify_dispatch")
     return o

@@ -41,8 +41,11 @@ struct DispatchScanParams {
   int32_t *P;
   int32_t *recv_count;
   int32_t *nrte;
+  int32_t *ntpr_out;     // optional layout outputs (routing from topk_idx only)
+  int32_t *ntpe_out;
+  uint8_t *in_rank_out;
   ScanHeader *head;
-  int32_t *expert_cnt;
+  int32_t *expert_cnt;   // [E] all sources, then [R][E] per source
   uint64_t *desc;
   int32_t *status;
   unsigned long long timeout_ns;
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const bool count_experts = p.nrte != nullptr;
+  const bool count_experts = p.nrte != nullptr || p.ntpe_out != nullptr;
 
   if (tid == 0) s_tile = static_cast<int>(atomicAdd(&p.head->ticket, 1u));
   if (count_experts)
@@ -163,6 +166,19 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
         if (count_experts) atomicAdd(&s_ehist[static_cast<int>(e)], 1);
       }
       if (bad) report(p.status, EP_STATUS_BAD_EXPERT);
+    }
+  }
+  // fused layout output: this token's row of is_token_in_rank
+  if (valid && p.in_rank_out != nullptr) {
+    uint8_t *row = p.in_rank_out + st * p.R;
+    if ((p.R & 3) == 0 && (reinterpret_cast<uintptr_t>(p.in_rank_out) & 3u) == 0) {
+      for (int d = 0; d < p.R; d += 4) {  // four 0/1 bytes per 32-bit store
+        const uint32_t b = my_mask[d >> 5] >> (d & 31);
+        reinterpret_cast<uint32_t *>(row)[d >> 2] =
+            (b & 1u) | ((b >> 1) & 1u) << 8 | ((b >> 2) & 1u) << 16 | ((b >> 3) & 1u) << 24;
+      }
+    } else {
+      for (int d = 0; d < p.R; ++d) row[d] = (my_mask[d >> 5] >> (d & 31)) & 1u;
     }
   }
   __syncthreads();
@@ -238,19 +254,30 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   }
   if (overflow) report(p.status, EP_STATUS_CAPACITY);
 
-  // ---- expert counts -> num_recv_tokens_per_expert ----------------------
+  // ---- expert counts -> num_recv_tokens_per_expert (+ fused layout) -------
   if (count_experts)
     for (int e = tid; e < p.E; e += kScanTile) {
       const int c = s_ehist[e];
-      if (c != 0) atomicAdd(&p.expert_cnt[e], c);
+      if (c != 0) {
+        atomicAdd(&p.expert_cnt[e], c);
+        if (p.ntpe_out != nullptr) atomicAdd(&p.expert_cnt[p.E + s * p.E + e], c);
+      }
     }
-  if (elect_last_cta(&p.head->done, static_cast<uint32_t>(p.num_tiles), &s_last) &&
-      count_experts) {
-    for (int e = tid; e < p.E; e += kScanTile) {
-      int n = __ldcg(&p.expert_cnt[e]);
-      if (p.align > 1) n = (n + p.align - 1) / p.align * p.align;
-      p.nrte[e] = n;
-    }
+  if (elect_last_cta(&p.head->done, static_cast<uint32_t>(p.num_tiles), &s_last)) {
+    if (p.nrte != nullptr)
+      for (int e = tid; e < p.E; e += kScanTile) {
+        int n = __ldcg(&p.expert_cnt[e]);
+        if (p.align > 1) n = (n + p.align - 1) / p.align * p.align;
+        p.nrte[e] = n;
+      }
+    if (p.ntpe_out != nullptr)
+      for (int i = tid; i < p.R * p.E; i += kScanTile)
+        p.ntpe_out[i] = __ldcg(&p.expert_cnt[p.E + i]);
+    if (p.ntpr_out != nullptr)  // tokens of s to d = P[s][d] - P[s-1][d]
+      for (int i = tid; i < p.R * p.R; i += kScanTile) {
+        const int prev = i >= p.R ? __ldcg(&p.P[i - p.R]) : 0;
+        p.ntpr_out[i] = __ldcg(&p.P[i]) - prev;
+      }
   }
 }
 
@@ -535,7 +562,8 @@ extern "C" EP_API size_t ep_dispatch_workspace_bytes(int num_ranks, int num_toke
   using namespace ep;
   if (num_ranks < 1 || num_tokens < 0 || num_experts < 0) return 0;
   const long tiles = static_cast<long>(num_ranks) * ((num_tokens + kScanTile - 1) / kScanTile);
-  return scan_workspace_bytes(tiles, num_ranks, num_experts);
+  // expert counters: all sources [E], then per source [R][E] (fused layout)
+  return scan_workspace_bytes(tiles, num_ranks, num_experts * (1 + num_ranks));
 }
 
 namespace ep {
@@ -568,9 +596,16 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
                 const uint8_t *is_token_in_rank, int R, int T, int K, int E, int align, int cap,
                 int64_t *recv_topk_idx, float *recv_topk_weights, int32_t *recv_src_idx,
                 int32_t *rank_prefix_matrix, int32_t *recv_count,
-                int32_t *num_recv_tokens_per_expert, int32_t *send_pos, void *workspace,
-                int32_t *status, cudaStream_t stream) {
+                int32_t *num_recv_tokens_per_expert, int32_t *send_pos, int32_t *ntpr_out,
+                int32_t *ntpe_out, uint8_t *in_rank_out, void *workspace, int32_t *status,
+                cudaStream_t stream) {
   if (T == 0) {  // nothing to route
+    if ((ntpr_out != nullptr &&
+         cudaMemsetAsync(ntpr_out, 0, sizeof(int32_t) * R * R, stream) != cudaSuccess) ||
+        (ntpe_out != nullptr &&
+         cudaMemsetAsync(ntpe_out, 0, sizeof(int32_t) * R * static_cast<size_t>(E), stream) !=
+             cudaSuccess))
+      return EP_ERR_CUDA;
     if (cudaMemsetAsync(rank_prefix_matrix, 0, sizeof(int32_t) * R * R, stream) != cudaSuccess ||
         cudaMemsetAsync(recv_count, 0, sizeof(int32_t) * R, stream) != cudaSuccess)
       return EP_ERR_CUDA;
@@ -612,10 +647,14 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   p.P = rank_prefix_matrix;
   p.recv_count = recv_count;
   p.nrte = num_recv_tokens_per_expert;
+  p.ntpr_out = ntpr_out;
+  p.ntpe_out = ntpe_out;
+  p.in_rank_out = in_rank_out;
   p.head = reinterpret_cast<ScanHeader *>(ws);
   p.expert_cnt = reinterpret_cast<int32_t *>(ws + sizeof(ScanHeader));
+  const int counters = Ectr * (1 + R);
   p.desc = reinterpret_cast<uint64_t *>(ws + sizeof(ScanHeader) +
-                                        static_cast<size_t>((Ectr + 3) & ~3) * 4);
+                                        static_cast<size_t>((counters + 3) & ~3) * 4);
   p.status = status;
   const WaitConfig wc = wait_config();
   p.timeout_ns = wc.timeout_ns;
@@ -751,9 +790,19 @@ extern "C" EP_API int ep_notify_dispatch(const int64_t *topk_idx, const float *t
                                          int32_t *recv_src_idx, int32_t *rank_prefix_matrix,
                                          int32_t *recv_count,
                                          int32_t *num_recv_tokens_per_expert, int32_t *send_pos,
-                                         void *workspace, size_t workspace_bytes,
-                                         int32_t *status, cudaStream_t stream) {
+                                         int32_t *num_tokens_per_rank,
+                                         int32_t *num_tokens_per_expert,
+                                         uint8_t *is_token_in_rank_out, void *workspace,
+                                         size_t workspace_bytes, int32_t *status,
+                                         cudaStream_t stream) {
   using namespace ep;
+  // the fused layout needs the routing to come from topk_idx
+  if ((num_tokens_per_rank != nullptr || num_tokens_per_expert != nullptr ||
+       is_token_in_rank_out != nullptr) &&
+      (topk_idx == nullptr || is_token_in_rank != nullptr || num_topk < 1 ||
+       num_topk > kMaxTopk || num_experts < 1 || num_experts > kMaxExperts ||
+       num_ranks < 1 || num_experts % num_ranks != 0))
+    return EP_ERR_INVALID_ARG;
   const int rc = check_notify_args(topk_idx, topk_weights, is_token_in_rank, num_ranks,
                                    num_tokens, num_topk, num_experts, expert_alignment, capacity,
                                    recv_topk_idx, recv_topk_weights, recv_src_idx,
@@ -763,7 +812,8 @@ extern "C" EP_API int ep_notify_dispatch(const int64_t *topk_idx, const float *t
   return notify_impl(topk_idx, topk_weights, is_token_in_rank, num_ranks, num_tokens, num_topk,
                      num_experts, expert_alignment, capacity, recv_topk_idx, recv_topk_weights,
                      recv_src_idx, rank_prefix_matrix, recv_count, num_recv_tokens_per_expert,
-                     send_pos, workspace, status, stream);
+                     send_pos, num_tokens_per_rank, num_tokens_per_expert, is_token_in_rank_out,
+                     workspace, status, stream);
 }
 
 extern "C" EP_API int ep_dispatch_cached(const void *x, const int32_t *send_pos, int num_ranks,
@@ -818,7 +868,7 @@ extern "C" EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
   rc = notify_impl(topk_idx, topk_weights, is_token_in_rank, num_ranks, num_tokens, num_topk,
                    num_experts, expert_alignment, capacity, recv_topk_idx, recv_topk_weights,
                    recv_src_idx, rank_prefix_matrix, recv_count, num_recv_tokens_per_expert,
-                   send_pos, workspace, status, stream);
+                   send_pos, nullptr, nullptr, nullptr, workspace, status, stream);
   if (rc != EP_OK) return rc;
   return copy_impl(x, nullptr, 0, 0, send_pos, num_ranks, num_tokens, hidden * 2, capacity,
                    recv_x, nullptr, status, stream);

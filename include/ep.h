@@ -179,6 +179,13 @@ EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
  * recv_x; it computes the handle (send_pos, rank_prefix_matrix, recv_count,
  * recv_src_idx), recv_topk_idx / recv_topk_weights and
  * num_recv_tokens_per_expert.
+ *
+ * Optionally, when the routing comes from topk_idx (is_token_in_rank NULL),
+ * the same kernel also returns the layout of ep_get_dispatch_layout for all
+ * R source ranks (A1 fused into A2): num_tokens_per_rank int32 [R, R],
+ * num_tokens_per_expert int32 [R, E], is_token_in_rank_out uint8 [R, T, R];
+ * each may be NULL.  Requesting them with is_token_in_rank given returns
+ * EP_ERR_INVALID_ARG.
  */
 EP_API int ep_notify_dispatch(const int64_t *topk_idx, const float *topk_weights,
                               const uint8_t *is_token_in_rank, int num_ranks,
@@ -188,7 +195,9 @@ EP_API int ep_notify_dispatch(const int64_t *topk_idx, const float *topk_weights
                               int32_t *recv_src_idx, int32_t *rank_prefix_matrix,
                               int32_t *recv_count,
                               int32_t *num_recv_tokens_per_expert,
-                              int32_t *send_pos, void *workspace,
+                              int32_t *send_pos, int32_t *num_tokens_per_rank,
+                              int32_t *num_tokens_per_expert,
+                              uint8_t *is_token_in_rank_out, void *workspace,
                               size_t workspace_bytes, int32_t *status,
                               cudaStream_t stream);
 

@@ -729,3 +729,33 @@ def test_empty_inputs_everywhere():
     torch.cuda.synchronize()
     assert (to_host(ll["recv_count"]) == 0).all() and (to_host(ll["layout_range"]) == 0).all()
     assert co.numel() == 0 and rx.numel() == 0 and rq.numel() == 0
+
+
+# ---------------------------------------------------------------------------
+# layout fused into the notify scan
+# ---------------------------------------------------------------------------
+
+FUSED_CASES = [
+    ("normal_like", Workload("fu1", R=8, T=300, H=64, E=256, K=8, seed=81)),
+    ("ragged_masked", Workload("fu2", R=5, T=129, H=64, E=40, K=3, masked_frac=0.2, seed=82)),
+    ("r40_unaligned", Workload("fu3", R=40, T=33, H=64, E=80, K=4, seed=83)),
+]
+
+
+@pytest.mark.parametrize("name,w", FUSED_CASES, ids=[c[0] for c in FUSED_CASES])
+def test_notify_with_fused_layout(name, w):
+    inp = make(w, with_x=False)
+    idx, wts = inp["topk_idx"], inp["topk_weights"]
+    lay = oracle.layout(idx, w.E, w.R)
+    pre = oracle.prefix(lay["is_token_in_rank"])
+    st = ep.new_status()
+    h = ep.ep_notify_dispatch(to_dev(idx), to_dev(wts), w.T, w.R, w.E, with_layout=True,
+                              status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(to_host(h["num_tokens_per_rank"]), lay["num_tokens_per_rank"])
+    np.testing.assert_array_equal(to_host(h["num_tokens_per_expert"]), lay["num_tokens_per_expert"])
+    np.testing.assert_array_equal(to_host(h["is_token_in_rank"]), lay["is_token_in_rank"])
+    np.testing.assert_array_equal(to_host(h["send_pos"]), pre["send_pos"])
+    np.testing.assert_array_equal(to_host(h["num_recv_tokens_per_expert"]),
+                                  oracle.expert_recv_counts(lay["num_tokens_per_expert"], w.R))
