@@ -55,14 +55,15 @@ struct DispatchScanParams {
 // Received top-k metadata of one copy held by a rank whose experts are
 // [lo, hi): local id for local slots, -1 / 0.0 otherwise.  16-byte stores
 // when K allows them (rows of K int64 / K fp32 are then 16-byte aligned).
+template <int MAXK>
 __device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, size_t row, int K,
-                                           int64_t lo, int64_t hi, const int64_t (&ek)[kMaxTopk],
-                                           const float (&wk)[kMaxTopk]) {
+                                           int64_t lo, int64_t hi, const int64_t (&ek)[MAXK],
+                                           const float (&wk)[MAXK]) {
   if (recv_idx != nullptr) {
     int64_t *dst = recv_idx + row * K;
     if ((K & 1) == 0) {
 #pragma unroll
-      for (int k = 0; k < kMaxTopk; k += 2) {
+      for (int k = 0; k < MAXK; k += 2) {
         if (k < K) {
           longlong2 v;
           v.x = (ek[k] >= lo && ek[k] < hi) ? ek[k] - lo : -1;
@@ -72,7 +73,7 @@ __device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, siz
       }
     } else {
 #pragma unroll
-      for (int k = 0; k < kMaxTopk; ++k)
+      for (int k = 0; k < MAXK; ++k)
         if (k < K) dst[k] = (ek[k] >= lo && ek[k] < hi) ? ek[k] - lo : -1;
     }
   }
@@ -80,7 +81,7 @@ __device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, siz
     float *dst = recv_w + row * K;
     if ((K & 3) == 0) {
 #pragma unroll
-      for (int k = 0; k < kMaxTopk; k += 4) {
+      for (int k = 0; k < MAXK; k += 4) {
         if (k < K) {
           float4 v;
           v.x = (ek[k] >= lo && ek[k] < hi) ? wk[k] : 0.f;
@@ -92,12 +93,14 @@ __device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, siz
       }
     } else {
 #pragma unroll
-      for (int k = 0; k < kMaxTopk; ++k)
+      for (int k = 0; k < MAXK; ++k)
         if (k < K) dst[k] = (ek[k] >= lo && ek[k] < hi) ? wk[k] : 0.f;
     }
   }
 }
 
+// MAXK: compile-time bound on the top-k slots (8 or 16), chosen per call.
+template <int MAXK>
 __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanParams p) {
   __shared__ int s_tile;
   __shared__ int s_last;
@@ -127,10 +130,10 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   const bool meta =
       valid && p.topk_idx != nullptr && (p.recv_idx != nullptr || p.recv_w != nullptr);
   const bool need_idx = valid && p.topk_idx != nullptr;
-  int64_t ek[kMaxTopk];
-  float wk[kMaxTopk];
+  int64_t ek[MAXK];
+  float wk[MAXK];
 #pragma unroll
-  for (int k = 0; k < kMaxTopk; ++k) {
+  for (int k = 0; k < MAXK; ++k) {
     ek[k] = -1;
     wk[k] = 0.f;
     if (need_idx && k < p.K) {
@@ -151,7 +154,7 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
     if (p.topk_idx != nullptr && (p.in_rank == nullptr || count_experts)) {
       bool bad = false;
 #pragma unroll
-      for (int k = 0; k < kMaxTopk; ++k) {
+      for (int k = 0; k < MAXK; ++k) {
         if (k >= p.K) break;
         const int64_t e = ek[k];
         if (e == -1) continue;
@@ -264,15 +267,39 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
       }
     }
   if (elect_last_cta(&p.head->done, static_cast<uint32_t>(p.num_tiles), &s_last)) {
+    // one CTA finalises: loads are issued in batches of 8 so that the loop
+    // does not wait one L2 round trip per element
+    constexpr int B = 8;
     if (p.nrte != nullptr)
-      for (int e = tid; e < p.E; e += kScanTile) {
-        int n = __ldcg(&p.expert_cnt[e]);
-        if (p.align > 1) n = (n + p.align - 1) / p.align * p.align;
-        p.nrte[e] = n;
+      for (int e0 = 0; e0 < p.E; e0 += kScanTile * B) {
+        int v[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const int e = e0 + b * kScanTile + tid;
+          v[b] = e < p.E ? __ldcg(&p.expert_cnt[e]) : 0;
+        }
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const int e = e0 + b * kScanTile + tid;
+          int n = v[b];
+          if (p.align > 1) n = (n + p.align - 1) / p.align * p.align;
+          if (e < p.E) p.nrte[e] = n;
+        }
       }
     if (p.ntpe_out != nullptr)
-      for (int i = tid; i < p.R * p.E; i += kScanTile)
-        p.ntpe_out[i] = __ldcg(&p.expert_cnt[p.E + i]);
+      for (int i0 = 0; i0 < p.R * p.E; i0 += kScanTile * B) {
+        int v[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const int i = i0 + b * kScanTile + tid;
+          v[b] = i < p.R * p.E ? __ldcg(&p.expert_cnt[p.E + i]) : 0;
+        }
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          const int i = i0 + b * kScanTile + tid;
+          if (i < p.R * p.E) p.ntpe_out[i] = v[b];
+        }
+      }
     if (p.ntpr_out != nullptr)  // tokens of s to d = P[s][d] - P[s-1][d]
       for (int i = tid; i < p.R * p.R; i += kScanTile) {
         const int prev = i >= p.R ? __ldcg(&p.P[i - p.R]) : 0;
@@ -659,7 +686,10 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   const WaitConfig wc = wait_config();
   p.timeout_ns = wc.timeout_ns;
   p.flags = wc.flags;
-  dispatch_scan_kernel<<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
+  if (topk_idx != nullptr && K > 8)
+    dispatch_scan_kernel<16><<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
+  else
+    dispatch_scan_kernel<8><<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
   if (launch_status() != EP_OK) return EP_ERR_CUDA;
   // rows past the receive count read -1 (fixed worst-case capacity)
   if (recv_topk_idx != nullptr && cap > 0) {

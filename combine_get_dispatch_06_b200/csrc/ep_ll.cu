@@ -45,6 +45,8 @@ struct LLScanParams {
   unsigned flags;
 };
 
+// MAXK: compile-time bound on the top-k slots (8 or 16), chosen per call.
+template <int MAXK>
 __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   __shared__ int s_tile;
   __shared__ uint32_t s_lanes[kScanWarps][kMaxExperts];  // lanes of the warp holding expert c
@@ -69,10 +71,10 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   // Distinct valid experts of this token (a repeated expert keeps only its
   // first slot in `col`; `ev` keeps every valid id).  Experts on a failed
   // rank are dropped.
-  int ev[kMaxTopk], col[kMaxTopk], rnk[kMaxTopk];
+  int ev[MAXK], col[MAXK], rnk[MAXK];
   bool bad = false;
 #pragma unroll
-  for (int k = 0; k < kMaxTopk; ++k) {
+  for (int k = 0; k < MAXK; ++k) {
     ev[k] = -1;
     col[k] = -1;
     rnk[k] = 0;
@@ -98,7 +100,7 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   // rank among the warp's tokens with that expert is then the number of
   // lower lanes in the word -- token order, whatever slot the expert is in.
 #pragma unroll
-  for (int k = 0; k < kMaxTopk; ++k) {
+  for (int k = 0; k < MAXK; ++k) {
     if (k < p.K) {
       const uint32_t peers = __match_any_sync(0xffffffffu, col[k]);
       if (col[k] >= 0 && lane == __ffs(peers) - 1) s_lanes[warp][col[k]] |= peers;
@@ -107,7 +109,7 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   }
   const uint32_t lt = lanemask_lt();
 #pragma unroll
-  for (int k = 0; k < kMaxTopk; ++k)
+  for (int k = 0; k < MAXK; ++k)
     if (col[k] >= 0) rnk[k] = __popc(s_lanes[warp][col[k]] & lt);
   __syncthreads();  // every warp's lane masks are complete before they are counted
   for (int c = tid; c < p.E; c += kScanTile)
@@ -140,10 +142,10 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   __syncthreads();
 
   if (valid) {
-    int pos[kMaxTopk];
+    int pos[MAXK];
     bool oob = false;
 #pragma unroll
-    for (int k = 0; k < kMaxTopk; ++k) {
+    for (int k = 0; k < MAXK; ++k) {
       pos[k] = -1;
       if (col[k] >= 0) {
         const int c = col[k];
@@ -157,12 +159,12 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
       }
     }
 #pragma unroll
-    for (int k = 0; k < kMaxTopk; ++k) {
+    for (int k = 0; k < MAXK; ++k) {
       if (k >= p.K) break;
       int v = pos[k];
       if (col[k] < 0 && ev[k] >= 0) {
 #pragma unroll
-        for (int k2 = 0; k2 < kMaxTopk; ++k2)
+        for (int k2 = 0; k2 < MAXK; ++k2)
           if (k2 < k && col[k2] == ev[k]) v = pos[k2];
       }
       p.ll_pos[st * p.K + k] = v;
@@ -547,7 +549,10 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   const WaitConfig wc = wait_config();
   p.timeout_ns = wc.timeout_ns;
   p.flags = wc.flags;
-  ll_scan_kernel<<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
+  if (K > 8)
+    ll_scan_kernel<16><<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
+  else
+    ll_scan_kernel<8><<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
   if (launch_status() != EP_OK) return EP_ERR_CUDA;
 
   const LLSmem plan = ll_smem_plan(H, use_fp8 != 0);
