@@ -24,6 +24,9 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ep_oracle.c")
 _LIB = os.path.join(_HERE, "libep_oracle.so")
+# The mutation test (tests/test_oracle_mutations.py) points this at a build of
+# a deliberately broken copy of ep_oracle.c to check that the pins fail.
+_LIB_OVERRIDE = os.environ.get("EP_ORACLE_LIB")
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -48,8 +51,11 @@ _lib = None
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        build()
-        L = ctypes.CDLL(_LIB)
+        if _LIB_OVERRIDE:
+            L = ctypes.CDLL(_LIB_OVERRIDE)
+        else:
+            build()
+            L = ctypes.CDLL(_LIB)
         L.orc_bf16_to_f32.restype = ctypes.c_float
         L.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
         L.orc_f32_to_bf16.restype = ctypes.c_uint16

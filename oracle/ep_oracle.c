@@ -539,22 +539,7 @@ void orc_quantize_row_ex(const uint16_t *x, int H, int round_scale, uint8_t *q,
 
 void orc_quantize_row(const uint16_t *x, int H, uint8_t *q, float *scales)
 {
-    for (int b = 0; b < H / 128; ++b) {
-        float amax = 0.0f;
-        for (int i = 0; i < 128; ++i) {
-            float a = fabsf(orc_bf16_to_f32(x[b * 128 + i]));
-            if (a > amax)
-                amax = a;
-        }
-        if (amax < 1e-4f)
-            amax = 1e-4f;
-        float inv = 448.0f / amax;
-        for (int i = 0; i < 128; ++i) {
-            float v = orc_bf16_to_f32(x[b * 128 + i]) * inv;
-            q[b * 128 + i] = orc_f32_to_e4m3(v);
-        }
-        scales[b] = amax / 448.0f;
-    }
+    orc_quantize_row_ex(x, H, 0, q, scales, NULL);
 }
 
 /*

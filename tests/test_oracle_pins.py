@@ -101,6 +101,28 @@ def test_golden_quant_block():
     assert s[0] == np.float32(1.0 / 224.0)
 
 
+def test_quant_zero_and_tiny_blocks():
+    # an all-zero block must quantise to zero codes with a finite positive
+    # scale (the amax floor keeps 448/amax finite); a block far below the
+    # floor keeps its signs and stays finite, and the round trip stays within
+    # the floor's quantum
+    x = np.zeros(256, np.float32)
+    x[128:] = np.where(np.arange(128) % 2 == 0, 1e-6, -1e-6)
+    for rs in (False, True):
+        q, s, _ = oracle.quantize_row_ex(f2b(x), round_scale=rs)
+        assert (q[:128] == 0).all()
+        assert np.isfinite(s).all() and (s > 0).all()
+        codes = oracle.e4m3_to_f32_array(q[128:])
+        assert np.isfinite(codes).all()
+        assert (np.sign(codes) == np.sign(x[128:])).all()
+        deq = codes.astype(np.float64) * s[1]
+        xv = b2f(f2b(x[128:])).astype(np.float64)
+        v = np.abs(xv) / s[1]
+        ulp = np.where(v < 2 ** -6, 2.0 ** -9,
+                       2.0 ** (np.floor(np.log2(np.maximum(v, 2 ** -6))) - 3))
+        assert (np.abs(deq - xv) <= 0.5 * ulp * s[1] * (1 + 1e-6)).all()
+
+
 def test_golden_quant_block_round_scale():
     g = gold("fp8_codes.json")["quant_block_round_scale"]
     x = np.zeros(128, np.float32)
