@@ -1,5 +1,6 @@
 // ep_api.cu -- host-side helpers of the C ABI: status text, version, the
 // process-wide limits of the bounded device waits, device properties.
+#include <algorithm>
 #include <atomic>
 #include <map>
 #include <mutex>
@@ -59,6 +60,22 @@ int ensure_dynamic_smem(const void *func, size_t bytes) {
     return EP_ERR_CUDA;
   cur = bytes;
   return EP_OK;
+}
+
+size_t spread_smem(size_t smem, int n) {
+  int dev = 0, per_sm = 0, reserved = 0;
+  if (n < 1 || cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
+          cudaSuccess)
+    return smem;
+  // n + 1 CTAs of (s + reserved) bytes overflow per_sm once s exceeds this
+  const long lo = static_cast<long>(per_sm) / (n + 1) - reserved + 16;
+  const size_t want = static_cast<size_t>((std::max<long>(lo, 0) + 15) & ~15L);
+  // only if n CTAs of that size still fit
+  if (static_cast<long>(n) * (static_cast<long>(want) + reserved) > per_sm) return smem;
+  return std::max(smem, want);
 }
 
 int ctas_per_sm(const void *func, int threads, size_t smem) {

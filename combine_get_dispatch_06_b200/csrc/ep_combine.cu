@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
                    const uint8_t *__restrict__ bias1, int R, long num_tok, int H, int K,
                    int cap, uint8_t *__restrict__ out, float *__restrict__ out_w,
                    int32_t *status) {
+  pdl_wait();
   extern __shared__ __align__(16) int64_t s_rows[];  // [warps][R] row indices d*cap + pos
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -144,7 +145,7 @@ extern "C" EP_API int ep_combine(const void *y, const float *recv_topk_weights,
   const long want = (num_tok + kCombineWarps - 1) / kCombineWarps;
   const long grid =
       std::min<long>(want, static_cast<long>(ctas_per_sm(fn, threads, smem)) * num_sms());
-  combine_kernel<<<static_cast<unsigned>(grid), threads, smem, stream>>>(
+  launch_pdl(combine_kernel, dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream,
       static_cast<const uint8_t *>(y), combined_topk_weights ? recv_topk_weights : nullptr,
       send_pos, static_cast<const uint8_t *>(bias_0), static_cast<const uint8_t *>(bias_1), R,
       num_tok, H, K, cap, static_cast<uint8_t *>(combined_x), combined_topk_weights, status);

@@ -39,6 +39,43 @@ int ensure_dynamic_smem(const void *func, size_t bytes);
 // dynamic shared memory (at least 1).  Cached per (function, device, smem).
 int ctas_per_sm(const void *func, int threads, size_t smem);
 
+// Dynamic shared memory to request so that at most `n` CTAs of a kernel fit
+// on one SM: max(smem, the smallest size of which n + 1 CTAs overflow the
+// SM).  A grid of n CTAs per SM then lands evenly on the SMs even when it is
+// scheduled while another kernel still holds part of them.
+size_t spread_smem(size_t smem, int n);
+
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialization.  It calls pdl_wait() before it reads
+// or writes any global memory: that waits until the previous grid in the
+// stream has completed and its writes are visible, so results keep stream
+// order.  It calls pdl_trigger() once its main work is issued: the next
+// kernel may then be scheduled (its CTAs start and block in their own
+// pdl_wait()), which hides its launch latency behind this kernel's tail.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void report(int32_t *status, int bits) {
   if (status != nullptr) atomicOr(status, bits);
 }

@@ -102,6 +102,7 @@ __device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, siz
 // MAXK: compile-time bound on the top-k slots (8 or 16), chosen per call.
 template <int MAXK>
 __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanParams p) {
+  pdl_wait();
   __shared__ int s_tile;
   __shared__ int s_last;
   __shared__ uint32_t s_mask[kScanTile * kMaskWords];
@@ -266,6 +267,7 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
         if (p.ntpe_out != nullptr) atomicAdd(&p.expert_cnt[p.E + s * p.E + e], c);
       }
     }
+  pdl_trigger();
   if (elect_last_cta(&p.head->done, static_cast<uint32_t>(p.num_tiles), &s_last)) {
     // one CTA finalises: loads are issued in batches of 8 so that the loop
     // does not wait one L2 round trip per element
@@ -336,6 +338,7 @@ __global__ void __launch_bounds__(kMaxRanks)
                          uint8_t *__restrict__ recv_x, int R, long num_tok, int row_bytes,
                          int chunk_bytes, int nchunks, int stage_stride, int cap,
                          int32_t *status, unsigned long long timeout_ns) {
+  pdl_wait();
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
   uint8_t *buf = smem + 128;
@@ -414,6 +417,7 @@ __global__ void __launch_bounds__(kMaxRanks)
       }
     }
   }
+  pdl_trigger();
   bulk_wait_all<0>();
   if (!all_ok) {
     report(status, EP_STATUS_WAIT_TIMEOUT);
@@ -451,6 +455,7 @@ struct CopyArgs {
 
 template <int S, bool kScales>
 __global__ void __launch_bounds__(kMaxRanks) dispatch_copy_planes_kernel(CopyArgs a) {
+  pdl_wait();
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
   uint8_t *buf = smem + 128;
@@ -569,6 +574,7 @@ __global__ void __launch_bounds__(kMaxRanks) dispatch_copy_planes_kernel(CopyArg
       if (i + S - 1 < nitems) sp[ps] = issue_next(ps);
     }
   }
+  pdl_trigger();
   bulk_wait_all<0>();
   if (!all_ok) {
     report(a.status, EP_STATUS_WAIT_TIMEOUT);
@@ -602,6 +608,8 @@ namespace {
 __global__ void __launch_bounds__(256)
     pad_recv_idx_kernel(const int32_t *__restrict__ recv_count, int cap, int K,
                         int64_t *__restrict__ recv_idx) {
+  pdl_wait();
+  pdl_trigger();
   const int d = blockIdx.y;
   const long first = min(max(recv_count[d], 0), cap);
   int64_t *base = recv_idx + static_cast<long>(d) * cap * K;
@@ -687,15 +695,18 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   p.timeout_ns = wc.timeout_ns;
   p.flags = wc.flags;
   if (topk_idx != nullptr && K > 8)
-    dispatch_scan_kernel<16><<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
+    launch_pdl(dispatch_scan_kernel<16>, dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
+        p);
   else
-    dispatch_scan_kernel<8><<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
+    launch_pdl(dispatch_scan_kernel<8>, dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
+        p);
   if (launch_status() != EP_OK) return EP_ERR_CUDA;
   // rows past the receive count read -1 (fixed worst-case capacity)
   if (recv_topk_idx != nullptr && cap > 0) {
     const long words = static_cast<long>(cap) * K / ((K & 1) == 0 ? 2 : 1);
     const int bx = static_cast<int>(std::min<long>((words + 255) / 256, 64));
-    pad_recv_idx_kernel<<<dim3(bx, R), 256, 0, stream>>>(recv_count, cap, K, recv_topk_idx);
+    launch_pdl(pad_recv_idx_kernel, dim3(bx, R), dim3(256), 0, stream,
+        recv_count, cap, K, recv_topk_idx);
     return launch_status();
   }
   return EP_OK;
@@ -737,7 +748,9 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
   a.status = status;
   a.timeout_ns = wait_config().timeout_ns;
   const int stages = short_rows ? kCopyStagesShort : kCopyStages;
-  const size_t smem = 128 + static_cast<size_t>(stages) * a.stage_stride;
+  // at most kCopyMaxCtasPerSm CTAs on an SM, also when scheduled early
+  const size_t smem =
+      spread_smem(128 + static_cast<size_t>(stages) * a.stage_stride, kCopyMaxCtasPerSm);
   const int threads = 32 * ((R + 31) / 32);
   const void *fn;
   if (xs != nullptr)
@@ -753,15 +766,17 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
   const dim3 g(static_cast<unsigned>(grid)), b(threads);
   if (xs != nullptr) {
     if (short_rows)
-      dispatch_copy_planes_kernel<kCopyStagesShort, true><<<g, b, smem, stream>>>(a);
+      launch_pdl(dispatch_copy_planes_kernel<kCopyStagesShort, true>, dim3(g), dim3(b), smem, stream,
+        a);
     else
-      dispatch_copy_planes_kernel<kCopyStages, true><<<g, b, smem, stream>>>(a);
+      launch_pdl(dispatch_copy_planes_kernel<kCopyStages, true>, dim3(g), dim3(b), smem, stream,
+        a);
   } else if (short_rows) {
-    dispatch_copy_rows_kernel<kCopyStagesShort><<<g, b, smem, stream>>>(
+    launch_pdl(dispatch_copy_rows_kernel<kCopyStagesShort>, dim3(g), dim3(b), smem, stream,
         a.x, a.send_pos, a.recv_x, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
         a.stage_stride, a.cap, a.status, a.timeout_ns);
   } else {
-    dispatch_copy_rows_kernel<kCopyStages><<<g, b, smem, stream>>>(
+    launch_pdl(dispatch_copy_rows_kernel<kCopyStages>, dim3(g), dim3(b), smem, stream,
         a.x, a.send_pos, a.recv_x, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
         a.stage_stride, a.cap, a.status, a.timeout_ns);
   }

@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(kLayoutTile)
     layout_kernel(const int64_t *__restrict__ topk_idx, int T, int K, int E, int R, int El,
                   int tiles_per_src, int32_t *__restrict__ ntpr, int32_t *__restrict__ ntpe,
                   uint8_t *__restrict__ in_rank, int32_t *status) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem[];
   int32_t *s_exp = reinterpret_cast<int32_t *>(smem);  // [E]
   uint8_t *s_row = smem + ((E * 4 + 15) & ~15);         // [tile, R]
@@ -115,7 +117,7 @@ extern "C" EP_API int ep_get_dispatch_layout(const int64_t *topk_idx, int num_sr
     return EP_ERR_CUDA;
   const long grid = static_cast<long>(S) * tiles_per_src;
   if (grid > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
-  layout_kernel<<<static_cast<unsigned>(grid), kLayoutTile, smem, stream>>>(
+  launch_pdl(layout_kernel, dim3(static_cast<unsigned>(grid)), dim3(kLayoutTile), smem, stream,
       topk_idx, T, K, E, R, E / R, tiles_per_src, num_tokens_per_rank, num_tokens_per_expert,
       is_token_in_rank, status);
   return launch_status();

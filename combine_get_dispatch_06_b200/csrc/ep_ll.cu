@@ -48,6 +48,8 @@ struct LLScanParams {
 // MAXK: compile-time bound on the top-k slots (8 or 16), chosen per call.
 template <int MAXK>
 __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
+  pdl_wait();
+  pdl_trigger();  // the next kernel may take the room this grid leaves
   __shared__ int s_tile;
   __shared__ uint32_t s_lanes[kScanWarps][kMaxExperts];  // lanes of the warp holding expert c
   __shared__ int s_whist[kScanWarps][kMaxExperts];
@@ -219,6 +221,8 @@ __global__ void __launch_bounds__(kLLThreads)
                        int cap, int round_scale, int ue8m0, LLSmem plan,
                        uint8_t *__restrict__ recv, void *__restrict__ scales_out,
                        int32_t *status, unsigned long long timeout_ns) {
+  pdl_wait();
+  pdl_trigger();  // the next kernel may take the room this grid leaves
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -392,6 +396,7 @@ __global__ void __launch_bounds__(kLLCombineWarps * 32)
                       const float *__restrict__ topk_w, const int32_t *__restrict__ ll_pos,
                       const int32_t *__restrict__ mask, long num_tok, int T, int H, int K, int E,
                       int cap, int nseg, uint8_t *__restrict__ out, int32_t *status) {
+  pdl_wait();
   __shared__ int64_t s_row[kLLCombineWarps][kMaxTopk];
   __shared__ float s_w[kLLCombineWarps][kMaxTopk];
   const int lane = threadIdx.x & 31;
@@ -550,14 +555,16 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   p.timeout_ns = wc.timeout_ns;
   p.flags = wc.flags;
   if (K > 8)
-    ll_scan_kernel<16><<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
+    launch_pdl(ll_scan_kernel<16>, dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
+        p);
   else
-    ll_scan_kernel<8><<<static_cast<unsigned>(num_tiles), kScanTile, 0, stream>>>(p);
+    launch_pdl(ll_scan_kernel<8>, dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
+        p);
   if (launch_status() != EP_OK) return EP_ERR_CUDA;
 
   const LLSmem plan = ll_smem_plan(H, use_fp8 != 0);
-  const size_t smem = static_cast<size_t>(plan.bytes);
-  if (smem > 227 * 1024) return EP_ERR_UNSUPPORTED;
+  if (plan.bytes > 227 * 1024) return EP_ERR_UNSUPPORTED;
+  const size_t smem = spread_smem(static_cast<size_t>(plan.bytes), kLLMaxCtasPerSm);
   const long num_tok = static_cast<long>(R) * T;
   const void *fn = use_fp8 ? reinterpret_cast<const void *>(ll_dispatch_kernel<true>)
                            : reinterpret_cast<const void *>(ll_dispatch_kernel<false>);
@@ -567,12 +574,12 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
       static_cast<long>(std::min(kLLMaxCtasPerSm, ctas_per_sm(fn, kLLThreads, smem))) *
           num_sms());
   if (use_fp8)
-    ll_dispatch_kernel<true><<<static_cast<unsigned>(grid), kLLThreads, smem, stream>>>(
+    launch_pdl(ll_dispatch_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
         static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, H, K, E,
         static_cast<int>(cap), round_scale, ue8m0, plan, static_cast<uint8_t *>(recv_x),
         recv_scales, status, wc.timeout_ns);
   else
-    ll_dispatch_kernel<false><<<static_cast<unsigned>(grid), kLLThreads, smem, stream>>>(
+    launch_pdl(ll_dispatch_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
         static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, H, K, E,
         static_cast<int>(cap), 0, 0, plan, static_cast<uint8_t *>(recv_x), nullptr, status,
         wc.timeout_ns);
@@ -607,7 +614,7 @@ extern "C" EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
   nseg = std::max(1, std::min(nseg, std::max(1, nvec / 32)));
   const long items = num_tok * nseg;
   const long grid = std::min<long>((items + kLLCombineWarps - 1) / kLLCombineWarps, resident);
-  ll_combine_kernel<<<static_cast<unsigned>(grid), threads, 0, stream>>>(
+  launch_pdl(ll_combine_kernel, dim3(static_cast<unsigned>(grid)), dim3(threads), 0, stream,
       static_cast<const uint8_t *>(y), topk_idx, topk_weights, ll_pos, rank_mask, num_tok, T, H,
       K, E, static_cast<int>(cap), nseg, static_cast<uint8_t *>(out), status);
   return launch_status();

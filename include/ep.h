@@ -15,6 +15,13 @@
  *   - Every call is asynchronous on `stream` and never synchronises the host.
  *     The caller orders calls with events.  Calls are stateless and may run
  *     concurrently if they use distinct output and workspace buffers.
+ *   - Kernels are launched with programmatic stream serialization
+ *     (programmatic dependent launch): each one waits for the previous grid
+ *     on the stream before it touches memory, and lets the next one be
+ *     scheduled early.  Ordinary launches, copies and events that follow on
+ *     the stream see every output as usual.  A kernel of the caller's that
+ *     follows with the same launch attribute must itself wait
+ *     (cudaGridDependencySynchronize) before it reads the outputs.
  *   - The return value is a host-side status (EP_OK ... EP_ERR_UNSUPPORTED).
  *     Argument checks happen before anything is launched; on an error nothing
  *     is launched and no output is touched.
