@@ -8,7 +8,9 @@ ep_combine, over one batch of seeded synthetic input (identity experts:
 combine reads the dispatched rows).
 Prints ONE JSON line (rank 0).  The headline value is algorithmic HBM GB/s of
 dispatch+combine (bytes the method must move, per step, divided by the step
-time); tokens/s and the share of 8 TB/s ride along.
+time); tokens/s and the share of 8 TB/s ride along.  The "e2e" figure is the
+same metric with every step's inputs uploaded from pinned host memory and its
+result downloaded, the copies of neighbouring steps overlapping the compute.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -260,8 +262,8 @@ def load_peak():
 
 # the source files each timed kernel is built from (for staleness checks)
 KERNEL_SOURCES = {
-    "dispatch_copy_kernel": ["ep_dispatch.cu", "ep_scan.cuh", "ep_common.cuh"],
-    "combine_kernel": ["ep_combine.cu", "ep_common.cuh"],
+    "dispatch_copy_rows_kernel": ["ep_dispatch.cu", "ep_scan.cuh", "ep_common.cuh", "ep_api.cu"],
+    "combine_kernel": ["ep_combine.cu", "ep_common.cuh", "ep_api.cu"],
 }
 
 
@@ -462,7 +464,9 @@ def run_ours(args) -> None:
     out["num_tokens_per_expert"] = ntpe
     out["is_token_in_rank"] = inr
 
-    def step(ev=None):
+    io0 = {"x": x, "idx": idx, "wt": wt, "cx": cx, "cw": cw}
+
+    def step(ev=None, io=io0):
         # layout (A1) is fused into the notify scan (A2): one kernel returns the
         # layout and the handle.  ep_dispatch == ep_notify_dispatch +
         # ep_dispatch_cached; the two halves are called separately so that the
@@ -470,15 +474,15 @@ def run_ours(args) -> None:
         if ev is not None:
             ev[0].record(stream)
             ev[1].record(stream)
-        ep.ep_notify_dispatch(idx, wt, T, R, E, with_layout=True, out=out, workspace=wsp,
-                              status=status)
+        ep.ep_notify_dispatch(io["idx"], io["wt"], T, R, E, with_layout=True, out=out,
+                              workspace=wsp, status=status)
         if ev is not None:
             ev[2].record(stream)
-        ep.ep_dispatch_cached(x, out["send_pos"], recv_x=out["recv_x"], status=status)
+        ep.ep_dispatch_cached(io["x"], out["send_pos"], recv_x=out["recv_x"], status=status)
         if ev is not None:
             ev[3].record(stream)
-        ep.ep_combine(out["recv_x"], out["send_pos"], out["recv_topk_weights"], combined_x=cx,
-                      combined_topk_weights=cw, status=status)
+        ep.ep_combine(out["recv_x"], out["send_pos"], out["recv_topk_weights"],
+                      combined_x=io["cx"], combined_topk_weights=io["cw"], status=status)
         if ev is not None:
             ev[4].record(stream)
 
@@ -518,38 +522,69 @@ def run_ours(args) -> None:
         raise RuntimeError(f"device status {int(status.item())} in the timed region")
 
     # ---- end to end: host inputs in, host result out, every step -----------
+    # Batches stream the way a serving loop feeds them: while step i computes,
+    # the inputs of step i+1 go up on one copy stream and the result of step
+    # i-1 comes down on another (the link is full duplex).  Two device sets of
+    # inputs and results alternate; events keep a set from being overwritten
+    # before the step or the copy that reads it is done.
     cx_h = torch.empty((R, T, H), dtype=torch.bfloat16).pin_memory()
     cw_h = torch.empty((R, T, K), dtype=torch.float32).pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
+    io1 = {k: torch.empty_like(v) for k, v in io0.items()}
+    ios = (io0, io1)
+    s_up = torch.cuda.Stream(device)
+    s_down = torch.cuda.Stream(device)
+    ev_up = [torch.cuda.Event() for _ in ios]
+    ev_done = [torch.cuda.Event() for _ in ios]
+    ev_down = [torch.cuda.Event() for _ in ios]
 
-    def e2e_step():
-        x.copy_(x_h, non_blocking=True)
-        idx.copy_(idx_h, non_blocking=True)
-        wt.copy_(w_h, non_blocking=True)
-        step()
-        cx_h.copy_(cx, non_blocking=True)
-        cw_h.copy_(cw, non_blocking=True)
+    def e2e_run(nsteps, start=None):
+        if start is not None:
+            s_up.wait_event(start)
+        for i in range(nsteps):
+            j = i % 2
+            io = ios[j]
+            with torch.cuda.stream(s_up):
+                if i >= 2:
+                    s_up.wait_event(ev_done[j])      # step i-2 has read this set
+                io["x"].copy_(x_h, non_blocking=True)
+                io["idx"].copy_(idx_h, non_blocking=True)
+                io["wt"].copy_(w_h, non_blocking=True)
+                ev_up[j].record(s_up)
+            stream.wait_event(ev_up[j])
+            if i >= 2:
+                stream.wait_event(ev_down[j])        # result of step i-2 is on the host
+            step(io=io)
+            ev_done[j].record(stream)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(ev_done[j])
+                cx_h.copy_(io["cx"], non_blocking=True)
+                cw_h.copy_(io["cw"], non_blocking=True)
+                ev_down[j].record(s_down)
+        stream.wait_stream(s_down)
 
-    for _ in range(2):
-        e2e_step()
+    e2e_run(2)
     barrier(device)
     torch.cuda.synchronize(device)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    e2e_run(e2e_steps, start=a)
     b.record(stream)
     torch.cuda.synchronize(device)
     barrier(device)
     e2e = aggregate(bytes_step, R * T, a.elapsed_time(b) / e2e_steps, device)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the end-to-end leg")
+    if not torch.equal(cx_h.view(torch.int16), cx.cpu().view(torch.int16)):
+        raise RuntimeError("end-to-end result differs from the device-resident step's")
     h2d = x_h.numel() * 2 + idx_h.numel() * 8 + w_h.numel() * 4
     d2h = cx_h.numel() * 2 + cw_h.numel() * 4
 
     peak, peak_kind = load_peak()
     bytes_copy = R * T * H * 2 + N * H * 2       # rows: read once, written per copy
     if copy_ms >= comb_ms:
-        dominant, dom_bytes, dom_ms = "dispatch_copy_kernel", bytes_copy, copy_ms
+        dominant, dom_bytes, dom_ms = "dispatch_copy_rows_kernel", bytes_copy, copy_ms
     else:
         dominant, dom_bytes, dom_ms = "combine_kernel", bytes_c, comb_ms
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9

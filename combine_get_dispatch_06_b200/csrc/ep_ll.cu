@@ -54,12 +54,15 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   __shared__ uint32_t s_lanes[kScanWarps][kMaxExperts];  // lanes of the warp holding expert c
   __shared__ int s_whist[kScanWarps][kMaxExperts];
   __shared__ int s_excl[kMaxExperts];
+  __shared__ int s_mask[kMaxRanks];  // failed ranks (non-zero), if a mask is given
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
   if (tid == 0) s_tile = static_cast<int>(atomicAdd(&p.head->ticket, 1u));
   for (int i = tid; i < kScanWarps * kMaxExperts; i += kScanTile) (&s_lanes[0][0])[i] = 0u;
+  if (p.mask != nullptr)
+    for (int i = tid; i < p.R; i += kScanTile) s_mask[i] = p.mask[i];
   __syncthreads();
 
   const int tile = s_tile;
@@ -68,7 +71,7 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   const bool valid = t < p.T;
   const size_t st = static_cast<size_t>(s) * p.T + t;
   // a failed (masked) source rank sends nothing
-  const bool src_ok = p.mask == nullptr || p.mask[s] == 0;
+  const bool src_ok = p.mask == nullptr || s_mask[s] == 0;
 
   // Distinct valid experts of this token (a repeated expert keeps only its
   // first slot in `col`; `ev` keeps every valid id).  Experts on a failed
@@ -83,7 +86,7 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
     if (valid && k < p.K) {
       const int64_t e = p.topk_idx[st * p.K + k];
       if (e >= 0 && e < p.E) {
-        if (!src_ok || (p.mask != nullptr && p.mask[static_cast<int>(e) / p.El] != 0)) continue;
+        if (!src_ok || (p.mask != nullptr && s_mask[static_cast<int>(e) / p.El] != 0)) continue;
         ev[k] = static_cast<int>(e);
         bool dup = false;
 #pragma unroll
@@ -121,24 +124,44 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
 
   const bool publish = (p.flags & EP_DEBUG_SUPPRESS_PUBLISH) == 0;
   const bool first_of_src = (tile % p.tiles_per_src) == 0;
-  for (int c = tid; c < p.E; c += kScanTile) {
-    int run = 0;
+  // The tile's count of every column is published before any column looks
+  // back, so no tile waits for a predecessor that is still busy with its
+  // other columns.
+  constexpr int kCols = kMaxExperts / kScanTile;
+  int runs[kCols];
 #pragma unroll
-    for (int w = 0; w < kScanWarps; ++w) {
-      const int n = s_whist[w][c];
-      s_whist[w][c] = run;
-      run += n;
+  for (int i = 0; i < kCols; ++i) {
+    const int c = tid + i * kScanTile;
+    runs[i] = 0;
+    if (c < p.E) {
+      int run = 0;
+#pragma unroll
+      for (int w = 0; w < kScanWarps; ++w) {
+        const int n = s_whist[w][c];
+        s_whist[w][c] = run;
+        run += n;
+      }
+      runs[i] = run;
+      if (publish) publish_aggregate(p.desc, tile, p.E, c, static_cast<uint32_t>(run));
     }
-    const uint32_t excl = lookback_window<1, 16>(p.desc, tile, p.E, c, static_cast<uint32_t>(run),
-                                                 publish, p.timeout_ns, p.status);
+  }
+#pragma unroll
+  for (int i = 0; i < kCols; ++i) {
+    const int c = tid + i * kScanTile;
+    if (c >= p.E) break;
+    const int run = runs[i];
+    const uint32_t excl = lookback_window<1, 32>(p.desc, tile, p.E, c, static_cast<uint32_t>(run),
+                                                 publish, p.timeout_ns, p.status, true);
     s_excl[c] = static_cast<int>(excl);
     const size_t o = (static_cast<size_t>(c) * p.R + s) * 2;
     if (first_of_src) p.layout_range[o] = static_cast<int>(excl);
-    // rows source s owns: the tiles of s add their counts (zeroed on the host)
-    if (run != 0) {
+    // rows source s owns: its only tile stores the count; several tiles add
+    // theirs (zeroed on the host)
+    if (p.tiles_per_src == 1)
+      p.layout_range[o + 1] = run;
+    else if (run != 0)
       atomicAdd(&p.layout_range[o + 1], run);
-      if (p.stats != nullptr) atomicAdd(&p.stats[c], run);
-    }
+    if (run != 0 && p.stats != nullptr) atomicAdd(&p.stats[c], run);
     if (tile == p.num_tiles - 1) p.recv_count[c] = static_cast<int>(excl) + run;
   }
   __syncthreads();
@@ -209,21 +232,26 @@ __host__ __device__ inline LLSmem ll_smem_plan(int H, bool fp8) {
   return m;
 }
 
-// One CTA per token at a time, tokens strided over the grid.  Thread 0 keeps
-// kLLInStages bulk loads of upcoming rows in flight; all 256 threads quantise
-// the current row (16 consecutive threads per 128-channel block, amax by
-// xor-shuffles); then warp 0's lanes, one per distinct expert of the token,
-// send the e4m3 row and its scales with bulk shared->global stores.
+// One CTA per token at a time.  Tokens are claimed from a shared counter
+// (`claim`, zeroed with the workspace), so CTAs that run faster take more of
+// them and the grid finishes together.  Thread 0 keeps kLLInStages claimed
+// rows in flight as bulk loads and claims one more token ahead, to hide the
+// atomic's round trip; warp 0 loads the next token's slots one token ahead.
+// All 256 threads quantise the current row (16 consecutive threads per
+// 128-channel block, amax by xor-shuffles); then warp 0's lanes, one per
+// distinct expert of the token, send the e4m3 row and its scales with bulk
+// shared->global stores.
 template <bool kFP8>
 __global__ void __launch_bounds__(kLLThreads)
     ll_dispatch_kernel(const uint8_t *__restrict__ x, const int64_t *__restrict__ topk_idx,
                        const int32_t *__restrict__ ll_pos, long num_tok, int H, int K, int E,
                        int cap, int round_scale, int ue8m0, LLSmem plan,
                        uint8_t *__restrict__ recv, void *__restrict__ scales_out,
-                       int32_t *status, unsigned long long timeout_ns) {
+                       uint32_t *claim, int32_t *status, unsigned long long timeout_ns) {
   pdl_wait();
   pdl_trigger();  // the next kernel may take the room this grid leaves
   extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ long s_tok[kLLInStages];  // token in each input stage, -1 = none
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
@@ -237,44 +265,57 @@ __global__ void __launch_bounds__(kLLThreads)
   const bool bulk_scales = (sc_bytes & 15) == 0;
   float *scales = static_cast<float *>(scales_out);
   uint8_t *scales8 = static_cast<uint8_t *>(scales_out);
-  const long n = static_cast<long>(blockIdx.x) < num_tok
-                     ? (num_tok - 1 - blockIdx.x) / gridDim.x + 1
-                     : 0;
 
-  if (tid == 0) {
-#pragma unroll
-    for (int i = 0; i < kLLInStages; ++i) mbar_init(&bars[i], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  auto issue = [&](long i) {  // thread 0
-    const int stg = static_cast<int>(i % kLLInStages);
-    const long u = static_cast<long>(blockIdx.x) + i * gridDim.x;
+  auto take = [&]() -> long {  // thread 0: the next unclaimed token, or -1
+    const uint32_t c = atomicAdd(claim, 1u);
+    return static_cast<long>(c) < num_tok ? static_cast<long>(c) : -1L;
+  };
+  auto issue = [&](int stg, long u) {  // thread 0
+    s_tok[stg] = u;
+    if (u < 0) return;
     mbar_arrive_expect_tx(&bars[stg], static_cast<uint32_t>(row_in));
     bulk_g2s_hint(inb + stg * plan.in_stride, x + u * row_in, static_cast<uint32_t>(row_in),
                   &bars[stg], l2_evict_first_policy());
   };
-  if (tid == 0)
-    for (long i = 0; i < kLLInStages && i < n; ++i) issue(i);
+  // slot `lane` of token u: its expert (or -1) and its slab row
+  auto slots = [&](long u, int &e, int &pos) {
+    e = -1;
+    pos = -1;
+    if (u >= 0 && lane < K) {
+      const int64_t ee = topk_idx[u * K + lane];
+      if (ee >= 0 && ee < E) {
+        e = static_cast<int>(ee);
+        pos = ll_pos[u * K + lane];
+      }
+    }
+  };
+
+  long ahead = -1;  // thread 0: the token claimed for the next issue
+  if (tid == 0) {
+#pragma unroll
+    for (int i = 0; i < kLLInStages; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+#pragma unroll
+    for (int i = 0; i < kLLInStages; ++i) issue(i, take());
+    ahead = take();
+  }
+  __syncthreads();
+  int e_next = -1, pos_next = -1;
+  if (tid < 32) slots(s_tok[0], e_next, pos_next);
 
   bool all_ok = true;
-  long stop = n;
-  for (long i = 0; i < n; ++i) {
+  long stop = -1;
+  for (long i = 0;; ++i) {
     const int stg = static_cast<int>(i % kLLInStages);
-    const long u = static_cast<long>(blockIdx.x) + i * gridDim.x;
+    const long u = s_tok[stg];
+    if (u < 0) break;  // claims are ordered: every later stage is empty too
     uint8_t *in = inb + stg * plan.in_stride;
 
     // destination of slot `lane` (warp 0): one row per distinct expert
     long dst = -1;
     if (tid < 32) {
-      int e = -1, pos = -1;
-      if (lane < K) {
-        const int64_t ee = topk_idx[u * K + lane];
-        if (ee >= 0 && ee < E) {
-          e = static_cast<int>(ee);
-          pos = ll_pos[u * K + lane];
-        }
-      }
+      const int e = e_next, pos = pos_next;
+      slots(s_tok[(i + 1) % kLLInStages], e_next, pos_next);  // used next token
       bool dup = false;
       for (int k2 = 0; k2 < K; ++k2) {
         const int e2 = __shfl_sync(0xffffffffu, e, k2);
@@ -321,8 +362,8 @@ __global__ void __launch_bounds__(kLLThreads)
         uint32_t ebits = 0;
         if (round_scale) {
           // smallest power of two >= amax / 448, and its exact reciprocal
-          const uint32_t u = __float_as_uint(__fdiv_rn(amax, 448.0f));
-          ebits = (u >> 23) + ((u & 0x7FFFFFu) != 0u ? 1u : 0u);
+          const uint32_t b = __float_as_uint(__fdiv_rn(amax, 448.0f));
+          ebits = (b >> 23) + ((b & 0x7FFFFFu) != 0u ? 1u : 0u);
           scale = __uint_as_float(ebits << 23);
           inv = __uint_as_float((254u - ebits) << 23);
         } else {
@@ -366,19 +407,22 @@ __global__ void __launch_bounds__(kLLThreads)
     }
     if (!kFP8) __syncthreads();
     // `in` is free: quantised (FP8) or read by the stores (bf16)
-    if (tid == 0 && i + kLLInStages < n) {
+    if (tid == 0) {
       fence_proxy_async_smem();
-      issue(i + kLLInStages);
+      const long next = ahead;
+      ahead = next >= 0 ? take() : -1L;
+      issue(stg, next);
     }
   }
   if (tid < 32) bulk_wait_all<0>();
   if (!all_ok) {
     report(status, EP_STATUS_WAIT_TIMEOUT);
     if (tid == 0) {
-      const long end = min(n, stop + kLLInStages);
-      for (long k = stop; k < end; ++k)
-        (void)mbar_wait_bounded(&bars[k % kLLInStages],
-                                static_cast<uint32_t>((k / kLLInStages) & 1), timeout_ns);
+      // drain the loads still in flight before the CTA's shared memory goes away
+      for (long k = stop; k < stop + kLLInStages; ++k)
+        if (s_tok[k % kLLInStages] >= 0)
+          (void)mbar_wait_bounded(&bars[k % kLLInStages],
+                                  static_cast<uint32_t>((k / kLLInStages) & 1), timeout_ns);
     }
   }
 }
@@ -526,7 +570,9 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   const int tiles_per_src = (T + kScanTile - 1) / kScanTile;
   const long num_tiles = static_cast<long>(R) * tiles_per_src;
   if (cap > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
-  if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess ||
+  if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return EP_ERR_CUDA;
+  // several tiles per source add up their counts; a single tile stores them
+  if (tiles_per_src > 1 &&
       cudaMemsetAsync(layout_range, 0, sizeof(int32_t) * 2 * static_cast<size_t>(E) * R,
                       stream) != cudaSuccess)
     return EP_ERR_CUDA;
@@ -577,12 +623,12 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
     launch_pdl(ll_dispatch_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
         static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, H, K, E,
         static_cast<int>(cap), round_scale, ue8m0, plan, static_cast<uint8_t *>(recv_x),
-        recv_scales, status, wc.timeout_ns);
+        recv_scales, &p.head->claim, status, wc.timeout_ns);
   else
     launch_pdl(ll_dispatch_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
         static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, H, K, E,
-        static_cast<int>(cap), 0, 0, plan, static_cast<uint8_t *>(recv_x), nullptr, status,
-        wc.timeout_ns);
+        static_cast<int>(cap), 0, 0, plan, static_cast<uint8_t *>(recv_x), nullptr,
+        &p.head->claim, status, wc.timeout_ns);
   return launch_status();
 }
 

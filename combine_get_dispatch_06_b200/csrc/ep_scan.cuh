@@ -22,7 +22,8 @@ constexpr int kScanWarps = kScanTile / 32;
 struct ScanHeader {
   uint32_t ticket;  // next tile number
   uint32_t done;    // tiles finished
-  uint32_t pad[2];
+  uint32_t claim;   // work counter of a kernel that runs after the scan
+  uint32_t pad;
 };
 
 // Workspace: header, then `counters` int32 (rounded to 4), then the
@@ -34,6 +35,13 @@ __host__ __device__ inline size_t scan_workspace_bytes(long num_tiles, int colum
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
+// Publishes the tile's own count of column `c` (an inclusive prefix for tile 0).
+__device__ __forceinline__ void publish_aggregate(uint64_t *desc, int tile, int columns, int c,
+                                                  uint32_t agg) {
+  st_relaxed_gpu(desc + static_cast<size_t>(tile) * columns + c,
+                 ((tile == 0 ? 2ull : 1ull) << 32) | agg);
+}
+
 // Windowed look-back for column `c` of tile `tile`, run by an aligned group of
 // G lanes (G a power of two <= 32; all G lanes call it with the same
 // arguments).  Each round the group reads a window of G*U predecessor
@@ -43,11 +51,13 @@ __host__ __device__ inline size_t scan_workspace_bytes(long num_tiles, int colum
 // is not yet published makes the group re-read the window, at most
 // `timeout_ns` in total.  Returns the exclusive prefix to every lane of the
 // group and publishes the tile's inclusive prefix (lane 0 of the group).
+// `agg_published`: the caller has already published the tile's own count
+// with publish_aggregate().
 template <int G, int U>
 __device__ __forceinline__ uint32_t lookback_window(uint64_t *desc, int tile, int columns, int c,
                                                     uint32_t agg, bool publish,
                                                     unsigned long long timeout_ns,
-                                                    int32_t *status) {
+                                                    int32_t *status, bool agg_published = false) {
   static_assert(G >= 1 && G <= 32 && (G & (G - 1)) == 0, "G must be a power of two");
   constexpr int W = G * U;
   const int lane = threadIdx.x & 31;
@@ -56,10 +66,10 @@ __device__ __forceinline__ uint32_t lookback_window(uint64_t *desc, int tile, in
   const uint32_t gmask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << gbase);
   uint64_t *mine = desc + static_cast<size_t>(tile) * columns + c;
   if (tile == 0) {
-    if (publish && gl == 0) st_relaxed_gpu(mine, (2ull << 32) | agg);
+    if (publish && !agg_published && gl == 0) st_relaxed_gpu(mine, (2ull << 32) | agg);
     return 0u;
   }
-  if (publish && gl == 0) st_relaxed_gpu(mine, (1ull << 32) | agg);
+  if (publish && !agg_published && gl == 0) st_relaxed_gpu(mine, (1ull << 32) | agg);
 
   uint32_t excl = 0;
   int base = tile - 1;
