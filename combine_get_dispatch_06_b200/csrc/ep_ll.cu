@@ -38,18 +38,25 @@ struct LLScanParams {
   int32_t *recv_src_info;
   int32_t *layout_range;
   int32_t *recv_count;
-  ScanHeader *head;
+  ScanHeader *head;      // head->done counts the tiles whose results are out
   uint64_t *desc;
+  uint32_t *tile_ready;  // [num_tiles] set once a tile's results are out
   int32_t *status;
   unsigned long long timeout_ns;
   unsigned flags;
 };
 
 // MAXK: compile-time bound on the top-k slots (8 or 16), chosen per call.
+//
+// The dispatch kernel that follows runs concurrently with this one: it is
+// scheduled once every tile has passed pdl_trigger(), which comes after
+// pdl_wait(), so everything before this kernel in the stream is complete by
+// then; it takes each token's slab rows once the token's tile has published
+// them (tile_ready, release/acquire).
 template <int MAXK>
 __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   pdl_wait();
-  pdl_trigger();  // the next kernel may take the room this grid leaves
+  pdl_trigger();  // after the wait: see above
   __shared__ int s_tile;
   __shared__ uint32_t s_lanes[kScanWarps][kMaxExperts];  // lanes of the warp holding expert c
   __shared__ int s_whist[kScanWarps][kMaxExperts];
@@ -196,6 +203,12 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
     }
     if (oob) report(p.status, EP_STATUS_BAD_POSITION);
   }
+  // every result of the tile is written: publish it to the dispatch kernel
+  __syncthreads();
+  if (tid == 0) {
+    st_release_gpu(p.tile_ready + tile, 1u);
+    red_release_gpu_add(&p.head->done, 1u);
+  }
 
 }
 
@@ -232,23 +245,43 @@ __host__ __device__ inline LLSmem ll_smem_plan(int H, bool fp8) {
   return m;
 }
 
+// Waits, by all 32 lanes of a warp, until *flag is non-zero; every lane
+// observes it with acquire semantics.  False when `timeout_ns` ran out.
+__device__ __forceinline__ bool warp_wait_flag(const uint32_t *flag,
+                                               unsigned long long timeout_ns) {
+  uint64_t t0 = 0;
+  while (true) {
+    if (__all_sync(0xffffffffu, ld_acquire_gpu(flag) != 0u)) return true;
+    const uint64_t now = __shfl_sync(0xffffffffu, globaltimer(), 0);
+    if (t0 == 0) t0 = now;
+    if (now - t0 > timeout_ns) return false;
+    __nanosleep(64);
+  }
+}
+
 // One CTA per token at a time.  Tokens are claimed from a shared counter
 // (`claim`, zeroed with the workspace), so CTAs that run faster take more of
 // them and the grid finishes together.  Thread 0 keeps kLLInStages claimed
 // rows in flight as bulk loads and claims one more token ahead, to hide the
-// atomic's round trip; warp 0 loads the next token's slots one token ahead.
-// All 256 threads quantise the current row (16 consecutive threads per
-// 128-channel block, amax by xor-shuffles); then warp 0's lanes, one per
-// distinct expert of the token, send the e4m3 row and its scales with bulk
-// shared->global stores.
+// atomic's round trip.  All 256 threads quantise the current row (16
+// consecutive threads per 128-channel block, amax by xor-shuffles); then warp
+// 0's lanes, one per distinct expert of the token, send the e4m3 row and its
+// scales with bulk shared->global stores.
+//
+// The kernel runs concurrently with ll_scan_kernel (see there): rows and
+// expert ids are inputs and are read at once; a token's slab rows (ll_pos)
+// are read once its tile is out (tile_ready), and, after every tile is out
+// (tiles_done == num_tiles), a token ahead.  The kernel waits for the scan
+// grid to complete before it exits, so later work in the stream sees both.
 template <bool kFP8>
 __global__ void __launch_bounds__(kLLThreads)
     ll_dispatch_kernel(const uint8_t *__restrict__ x, const int64_t *__restrict__ topk_idx,
-                       const int32_t *__restrict__ ll_pos, long num_tok, int H, int K, int E,
+                       const int32_t *ll_pos, long num_tok, int T, int H, int K, int E,
                        int cap, int round_scale, int ue8m0, LLSmem plan,
                        uint8_t *__restrict__ recv, void *__restrict__ scales_out,
-                       uint32_t *claim, int32_t *status, unsigned long long timeout_ns) {
-  pdl_wait();
+                       uint32_t *claim, const uint32_t *tile_ready, const uint32_t *tiles_done,
+                       int tiles_per_src, int num_tiles, int32_t *status,
+                       unsigned long long timeout_ns) {
   pdl_trigger();  // the next kernel may take the room this grid leaves
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ long s_tok[kLLInStages];  // token in each input stage, -1 = none
@@ -277,17 +310,13 @@ __global__ void __launch_bounds__(kLLThreads)
     bulk_g2s_hint(inb + stg * plan.in_stride, x + u * row_in, static_cast<uint32_t>(row_in),
                   &bars[stg], l2_evict_first_policy());
   };
-  // slot `lane` of token u: its expert (or -1) and its slab row
-  auto slots = [&](long u, int &e, int &pos) {
-    e = -1;
-    pos = -1;
-    if (u >= 0 && lane < K) {
-      const int64_t ee = topk_idx[u * K + lane];
-      if (ee >= 0 && ee < E) {
-        e = static_cast<int>(ee);
-        pos = ll_pos[u * K + lane];
-      }
-    }
+  auto expert_of = [&](long u) -> int {  // expert of slot `lane` of token u, or -1
+    if (u < 0 || lane >= K) return -1;
+    const int64_t ee = __ldg(topk_idx + u * K + lane);
+    return (ee >= 0 && ee < E) ? static_cast<int>(ee) : -1;
+  };
+  auto tile_of = [&](long u) -> int {
+    return static_cast<int>((u / T) * tiles_per_src + (u % T) / kScanTile);
   };
 
   long ahead = -1;  // thread 0: the token claimed for the next issue
@@ -300,8 +329,10 @@ __global__ void __launch_bounds__(kLLThreads)
     ahead = take();
   }
   __syncthreads();
+  // warp 0: the next token's experts and (once every tile is out) its rows
   int e_next = -1, pos_next = -1;
-  if (tid < 32) slots(s_tok[0], e_next, pos_next);
+  bool pos_next_ok = false, all_out = false, failed = false;
+  if (tid < 32) e_next = expert_of(s_tok[0]);
 
   bool all_ok = true;
   long stop = -1;
@@ -311,22 +342,18 @@ __global__ void __launch_bounds__(kLLThreads)
     if (u < 0) break;  // claims are ordered: every later stage is empty too
     uint8_t *in = inb + stg * plan.in_stride;
 
-    // destination of slot `lane` (warp 0): one row per distinct expert
-    long dst = -1;
+    // warp 0: this token's experts (and rows, if read a token ahead); start
+    // reading the next token's experts
+    int e = -1, pos = -1;
+    bool have_pos = false;
+    long un = -1;
     if (tid < 32) {
-      const int e = e_next, pos = pos_next;
-      slots(s_tok[(i + 1) % kLLInStages], e_next, pos_next);  // used next token
-      bool dup = false;
-      for (int k2 = 0; k2 < K; ++k2) {
-        const int e2 = __shfl_sync(0xffffffffu, e, k2);
-        dup |= (k2 < lane && e2 == e);
-      }
-      if (e >= 0 && !dup) {  // pos -1: the slot was dropped (failed rank)
-        if (pos >= 0 && pos < cap)
-          dst = static_cast<long>(e) * cap + pos;
-        else if (pos != -1)
-          report(status, EP_STATUS_BAD_POSITION);
-      }
+      e = e_next;
+      pos = pos_next;
+      have_pos = pos_next_ok;
+      un = s_tok[(i + 1) % kLLInStages];
+      e_next = expert_of(un);
+      pos_next_ok = false;
       // FP8: the output buffer of token i - 2 must have been read by its stores
       if (kFP8) bulk_wait_read<1>();
     }
@@ -390,6 +417,35 @@ __global__ void __launch_bounds__(kLLThreads)
       src = q;
     }
     if (tid < 32) {
+      // slab rows of this token: wait for its tile if they were not read ahead
+      if (!have_pos && !failed) {
+        if (all_out || warp_wait_flag(tile_ready + tile_of(u), timeout_ns)) {
+          pos = lane < K ? ld_relaxed_gpu(ll_pos + u * K + lane) : -1;
+        } else {
+          failed = true;  // later tokens are dropped too: no wait per token
+          if (lane == 0) report(status, EP_STATUS_WAIT_TIMEOUT);
+        }
+      }
+      if (!all_out && !failed)
+        all_out = __all_sync(0xffffffffu,
+                             ld_acquire_gpu(tiles_done) >= static_cast<uint32_t>(num_tiles));
+      if (all_out && un >= 0) {  // every tile is out: read the next token's rows now
+        if (lane < K) pos_next = ld_relaxed_gpu(ll_pos + un * K + lane);
+        pos_next_ok = true;
+      }
+      // one row per distinct expert
+      bool dup = false;
+      for (int k2 = 0; k2 < K; ++k2) {
+        const int e2 = __shfl_sync(0xffffffffu, e, k2);
+        dup |= (k2 < lane && e2 == e);
+      }
+      long dst = -1;
+      if (!failed && e >= 0 && !dup) {  // pos -1: the slot was dropped (failed rank)
+        if (pos >= 0 && pos < cap)
+          dst = static_cast<long>(e) * cap + pos;
+        else if (pos != -1)
+          report(status, EP_STATUS_BAD_POSITION);
+      }
       if (dst >= 0) {
         bulk_s2g(recv + dst * pay, src, static_cast<uint32_t>(pay));
         if constexpr (kFP8) {
@@ -425,6 +481,8 @@ __global__ void __launch_bounds__(kLLThreads)
                                   static_cast<uint32_t>((k / kLLInStages) & 1), timeout_ns);
     }
   }
+  // the scan grid completes before this one does
+  pdl_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -519,11 +577,22 @@ __global__ void __launch_bounds__(kLLCombineWarps * 32)
 }  // namespace
 }  // namespace ep
 
+namespace ep {
+namespace {
+// LL workspace: scan header, descriptors [tiles][E] (64-bit), then one
+// tile-ready word per tile.
+size_t ll_ready_offset(long tiles, int E) {
+  return sizeof(ScanHeader) + static_cast<size_t>(tiles) * E * sizeof(uint64_t);
+}
+}  // namespace
+}  // namespace ep
+
 extern "C" EP_API size_t ep_ll_workspace_bytes(int num_ranks, int num_tokens, int num_experts) {
   using namespace ep;
   if (num_ranks < 1 || num_tokens < 0 || num_experts < 1) return 0;
   const long tiles = static_cast<long>(num_ranks) * ((num_tokens + kScanTile - 1) / kScanTile);
-  return scan_workspace_bytes(tiles, num_experts, 0);
+  const size_t bytes = ll_ready_offset(tiles, num_experts) + static_cast<size_t>(tiles) * 4;
+  return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
 extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
@@ -596,6 +665,7 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   p.recv_count = recv_count;
   p.head = reinterpret_cast<ScanHeader *>(ws);
   p.desc = reinterpret_cast<uint64_t *>(ws + sizeof(ScanHeader));
+  p.tile_ready = reinterpret_cast<uint32_t *>(ws + ll_ready_offset(num_tiles, E));
   p.status = status;
   const WaitConfig wc = wait_config();
   p.timeout_ns = wc.timeout_ns;
@@ -621,14 +691,16 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
           num_sms());
   if (use_fp8)
     launch_pdl(ll_dispatch_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
-        static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, H, K, E,
+        static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, T, H, K, E,
         static_cast<int>(cap), round_scale, ue8m0, plan, static_cast<uint8_t *>(recv_x),
-        recv_scales, &p.head->claim, status, wc.timeout_ns);
+        recv_scales, &p.head->claim, p.tile_ready, &p.head->done, tiles_per_src,
+        static_cast<int>(num_tiles), status, wc.timeout_ns);
   else
     launch_pdl(ll_dispatch_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
-        static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, H, K, E,
+        static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, T, H, K, E,
         static_cast<int>(cap), 0, 0, plan, static_cast<uint8_t *>(recv_x), nullptr,
-        &p.head->claim, status, wc.timeout_ns);
+        &p.head->claim, p.tile_ready, &p.head->done, tiles_per_src,
+        static_cast<int>(num_tiles), status, wc.timeout_ns);
   return launch_status();
 }
 
