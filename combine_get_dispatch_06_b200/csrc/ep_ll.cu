@@ -38,9 +38,9 @@ struct LLScanParams {
   int32_t *recv_src_info;
   int32_t *layout_range;
   int32_t *recv_count;
-  ScanHeader *head;      // head->done counts the tiles whose results are out
+  ScanHeader *head;
   uint64_t *desc;
-  uint32_t *tile_ready;  // [num_tiles] set once a tile's results are out
+  int32_t *pos_mirror;  // [R*T][K] ll_pos + 2 (0 = not written yet), for the dispatch kernel
   int32_t *status;
   unsigned long long timeout_ns;
   unsigned flags;
@@ -51,8 +51,9 @@ struct LLScanParams {
 // The dispatch kernel that follows runs concurrently with this one: it is
 // scheduled once every tile has passed pdl_trigger(), which comes after
 // pdl_wait(), so everything before this kernel in the stream is complete by
-// then; it takes each token's slab rows once the token's tile has published
-// them (tile_ready, release/acquire).
+// then.  It takes each token's slab rows from a mirror of ll_pos in the
+// workspace, zeroed before this kernel and written here as ll_pos + 2, so
+// that a non-zero word is its own proof of being written.
 template <int MAXK>
 __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   pdl_wait();
@@ -200,14 +201,9 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
           if (k2 < k && col[k2] == ev[k]) v = pos[k2];
       }
       p.ll_pos[st * p.K + k] = v;
+      st_relaxed_gpu(p.pos_mirror + st * p.K + k, v + 2);
     }
     if (oob) report(p.status, EP_STATUS_BAD_POSITION);
-  }
-  // every result of the tile is written: publish it to the dispatch kernel
-  __syncthreads();
-  if (tid == 0) {
-    st_release_gpu(p.tile_ready + tile, 1u);
-    red_release_gpu_add(&p.head->done, 1u);
   }
 
 }
@@ -215,7 +211,7 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
 // ---------------------------------------------------------------------------
 
 constexpr int kLLThreads = 256;  // 8 warps quantise one token row together
-constexpr int kLLInStages = 3;
+constexpr int kLLInStages = 2;
 constexpr int kLLMaxCtasPerSm = 3;
 
 __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float d) {
@@ -245,20 +241,6 @@ __host__ __device__ inline LLSmem ll_smem_plan(int H, bool fp8) {
   return m;
 }
 
-// Waits, by all 32 lanes of a warp, until *flag is non-zero; every lane
-// observes it with acquire semantics.  False when `timeout_ns` ran out.
-__device__ __forceinline__ bool warp_wait_flag(const uint32_t *flag,
-                                               unsigned long long timeout_ns) {
-  uint64_t t0 = 0;
-  while (true) {
-    if (__all_sync(0xffffffffu, ld_acquire_gpu(flag) != 0u)) return true;
-    const uint64_t now = __shfl_sync(0xffffffffu, globaltimer(), 0);
-    if (t0 == 0) t0 = now;
-    if (now - t0 > timeout_ns) return false;
-    __nanosleep(64);
-  }
-}
-
 // One CTA per token at a time.  Tokens are claimed from a shared counter
 // (`claim`, zeroed with the workspace), so CTAs that run faster take more of
 // them and the grid finishes together.  Thread 0 keeps kLLInStages claimed
@@ -269,18 +251,16 @@ __device__ __forceinline__ bool warp_wait_flag(const uint32_t *flag,
 // scales with bulk shared->global stores.
 //
 // The kernel runs concurrently with ll_scan_kernel (see there): rows and
-// expert ids are inputs and are read at once; a token's slab rows (ll_pos)
-// are read once its tile is out (tile_ready), and, after every tile is out
-// (tiles_done == num_tiles), a token ahead.  The kernel waits for the scan
-// grid to complete before it exits, so later work in the stream sees both.
+// expert ids are inputs and are read at once; a token's slab rows come from
+// the scan's mirror of ll_pos, read a token ahead and read again while a
+// word is still zero (not written yet).  The kernel waits for the scan grid
+// to complete before it exits, so later work in the stream sees both.
 template <bool kFP8>
 __global__ void __launch_bounds__(kLLThreads)
     ll_dispatch_kernel(const uint8_t *__restrict__ x, const int64_t *__restrict__ topk_idx,
-                       const int32_t *ll_pos, long num_tok, int T, int H, int K, int E,
-                       int cap, int round_scale, int ue8m0, LLSmem plan,
-                       uint8_t *__restrict__ recv, void *__restrict__ scales_out,
-                       uint32_t *claim, const uint32_t *tile_ready, const uint32_t *tiles_done,
-                       int tiles_per_src, int num_tiles, int32_t *status,
+                       const int32_t *pos_mirror, long num_tok, int H, int K, int E, int cap,
+                       int round_scale, int ue8m0, LLSmem plan, uint8_t *__restrict__ recv,
+                       void *__restrict__ scales_out, uint32_t *claim, int32_t *status,
                        unsigned long long timeout_ns) {
   pdl_trigger();  // the next kernel may take the room this grid leaves
   extern __shared__ __align__(128) uint8_t smem[];
@@ -315,8 +295,9 @@ __global__ void __launch_bounds__(kLLThreads)
     const int64_t ee = __ldg(topk_idx + u * K + lane);
     return (ee >= 0 && ee < E) ? static_cast<int>(ee) : -1;
   };
-  auto tile_of = [&](long u) -> int {
-    return static_cast<int>((u / T) * tiles_per_src + (u % T) / kScanTile);
+  auto mirror_of = [&](long u) -> int32_t {  // slot `lane` of token u: ll_pos + 2, 0 = not yet
+    if (u < 0 || lane >= K) return 1;          // no slot: reads as ll_pos -1
+    return ld_relaxed_gpu(pos_mirror + u * K + lane);
   };
 
   long ahead = -1;  // thread 0: the token claimed for the next issue
@@ -329,10 +310,14 @@ __global__ void __launch_bounds__(kLLThreads)
     ahead = take();
   }
   __syncthreads();
-  // warp 0: the next token's experts and (once every tile is out) its rows
-  int e_next = -1, pos_next = -1;
-  bool pos_next_ok = false, all_out = false, failed = false;
-  if (tid < 32) e_next = expert_of(s_tok[0]);
+  // warp 0: the next token's experts and mirrored slab rows
+  int e_next = -1;
+  int32_t m_next = 0;
+  bool failed = false;
+  if (tid < 32) {
+    e_next = expert_of(s_tok[0]);
+    m_next = mirror_of(s_tok[0]);
+  }
 
   bool all_ok = true;
   long stop = -1;
@@ -342,18 +327,16 @@ __global__ void __launch_bounds__(kLLThreads)
     if (u < 0) break;  // claims are ordered: every later stage is empty too
     uint8_t *in = inb + stg * plan.in_stride;
 
-    // warp 0: this token's experts (and rows, if read a token ahead); start
-    // reading the next token's experts
-    int e = -1, pos = -1;
-    bool have_pos = false;
-    long un = -1;
+    // warp 0: this token's experts and rows (read a token ahead); start
+    // reading the next token's
+    int e = -1;
+    int32_t m = 0;
     if (tid < 32) {
       e = e_next;
-      pos = pos_next;
-      have_pos = pos_next_ok;
-      un = s_tok[(i + 1) % kLLInStages];
+      m = m_next;
+      const long un = s_tok[(i + 1) % kLLInStages];
       e_next = expert_of(un);
-      pos_next_ok = false;
+      m_next = mirror_of(un);
       // FP8: the output buffer of token i - 2 must have been read by its stores
       if (kFP8) bulk_wait_read<1>();
     }
@@ -417,22 +400,23 @@ __global__ void __launch_bounds__(kLLThreads)
       src = q;
     }
     if (tid < 32) {
-      // slab rows of this token: wait for its tile if they were not read ahead
-      if (!have_pos && !failed) {
-        if (all_out || warp_wait_flag(tile_ready + tile_of(u), timeout_ns)) {
-          pos = lane < K ? ld_relaxed_gpu(ll_pos + u * K + lane) : -1;
-        } else {
-          failed = true;  // later tokens are dropped too: no wait per token
-          if (lane == 0) report(status, EP_STATUS_WAIT_TIMEOUT);
+      // slab rows of this token: words still zero are read again (bounded);
+      // after a wait ran out, this and later tokens are dropped
+      if (!failed) {
+        uint64_t t0 = 0;
+        while (!__all_sync(0xffffffffu, m != 0)) {
+          const uint64_t now = __shfl_sync(0xffffffffu, globaltimer(), 0);
+          if (t0 == 0) t0 = now;
+          if (now - t0 > timeout_ns) {
+            failed = true;
+            if (lane == 0) report(status, EP_STATUS_WAIT_TIMEOUT);
+            break;
+          }
+          __nanosleep(64);
+          if (m == 0) m = mirror_of(u);
         }
       }
-      if (!all_out && !failed)
-        all_out = __all_sync(0xffffffffu,
-                             ld_acquire_gpu(tiles_done) >= static_cast<uint32_t>(num_tiles));
-      if (all_out && un >= 0) {  // every tile is out: read the next token's rows now
-        if (lane < K) pos_next = ld_relaxed_gpu(ll_pos + un * K + lane);
-        pos_next_ok = true;
-      }
+      const int pos = m - 2;
       // one row per distinct expert
       bool dup = false;
       for (int k2 = 0; k2 < K; ++k2) {
@@ -579,9 +563,9 @@ __global__ void __launch_bounds__(kLLCombineWarps * 32)
 
 namespace ep {
 namespace {
-// LL workspace: scan header, descriptors [tiles][E] (64-bit), then one
-// tile-ready word per tile.
-size_t ll_ready_offset(long tiles, int E) {
+// LL workspace: scan header, descriptors [tiles][E] (64-bit), then the
+// position mirror [R*T][K] int32 (room for K up to kMaxTopk).
+size_t ll_mirror_offset(long tiles, int E) {
   return sizeof(ScanHeader) + static_cast<size_t>(tiles) * E * sizeof(uint64_t);
 }
 }  // namespace
@@ -591,7 +575,8 @@ extern "C" EP_API size_t ep_ll_workspace_bytes(int num_ranks, int num_tokens, in
   using namespace ep;
   if (num_ranks < 1 || num_tokens < 0 || num_experts < 1) return 0;
   const long tiles = static_cast<long>(num_ranks) * ((num_tokens + kScanTile - 1) / kScanTile);
-  const size_t bytes = ll_ready_offset(tiles, num_experts) + static_cast<size_t>(tiles) * 4;
+  const size_t bytes = ll_mirror_offset(tiles, num_experts) +
+                       static_cast<size_t>(num_ranks) * num_tokens * kMaxTopk * sizeof(int32_t);
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
@@ -638,8 +623,10 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   const long cap = static_cast<long>(R) * T;
   const int tiles_per_src = (T + kScanTile - 1) / kScanTile;
   const long num_tiles = static_cast<long>(R) * tiles_per_src;
-  if (cap > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
-  if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return EP_ERR_CUDA;
+  if (cap > 0x7ffffffdL) return EP_ERR_UNSUPPORTED;  // mirror words hold ll_pos + 2
+  // header, descriptors and the mirror words this call uses start at zero
+  const size_t used = ll_mirror_offset(num_tiles, E) + static_cast<size_t>(cap) * K * sizeof(int32_t);
+  if (cudaMemsetAsync(workspace, 0, used, stream) != cudaSuccess) return EP_ERR_CUDA;
   // several tiles per source add up their counts; a single tile stores them
   if (tiles_per_src > 1 &&
       cudaMemsetAsync(layout_range, 0, sizeof(int32_t) * 2 * static_cast<size_t>(E) * R,
@@ -665,7 +652,7 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   p.recv_count = recv_count;
   p.head = reinterpret_cast<ScanHeader *>(ws);
   p.desc = reinterpret_cast<uint64_t *>(ws + sizeof(ScanHeader));
-  p.tile_ready = reinterpret_cast<uint32_t *>(ws + ll_ready_offset(num_tiles, E));
+  p.pos_mirror = reinterpret_cast<int32_t *>(ws + ll_mirror_offset(num_tiles, E));
   p.status = status;
   const WaitConfig wc = wait_config();
   p.timeout_ns = wc.timeout_ns;
@@ -691,16 +678,14 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
           num_sms());
   if (use_fp8)
     launch_pdl(ll_dispatch_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
-        static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, T, H, K, E,
+        static_cast<const uint8_t *>(x), topk_idx, p.pos_mirror, num_tok, H, K, E,
         static_cast<int>(cap), round_scale, ue8m0, plan, static_cast<uint8_t *>(recv_x),
-        recv_scales, &p.head->claim, p.tile_ready, &p.head->done, tiles_per_src,
-        static_cast<int>(num_tiles), status, wc.timeout_ns);
+        recv_scales, &p.head->claim, status, wc.timeout_ns);
   else
     launch_pdl(ll_dispatch_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
-        static_cast<const uint8_t *>(x), topk_idx, ll_pos, num_tok, T, H, K, E,
+        static_cast<const uint8_t *>(x), topk_idx, p.pos_mirror, num_tok, H, K, E,
         static_cast<int>(cap), 0, 0, plan, static_cast<uint8_t *>(recv_x), nullptr,
-        &p.head->claim, p.tile_ready, &p.head->done, tiles_per_src,
-        static_cast<int>(num_tiles), status, wc.timeout_ns);
+        &p.head->claim, status, wc.timeout_ns);
   return launch_status();
 }
 
