@@ -14,7 +14,7 @@
 //                         top-k metadata, P, recv_count; expert counts are
 //                         reduced with shared + global atomics and finalised
 //                         by the last CTA.  Small (a few MB of traffic).
-//   dispatch_copy_kernel  the data movement: each token row is read ONCE from
+//   dispatch_copy_rows_kernel  the data movement: each token row is read ONCE from
 //                         HBM into shared memory by a bulk (TMA) copy and
 //                         written to each destination by bulk shared->global
 //                         copies, S stages deep.  HBM-bound: R*T*H*2 bytes

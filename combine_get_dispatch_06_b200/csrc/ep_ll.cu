@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
 // ---------------------------------------------------------------------------
 
 constexpr int kLLThreads = 256;  // 8 warps quantise one token row together
-constexpr int kLLInStages = 2;
+constexpr int kLLInStages = 2;  // >= 2: warp 0 reads the next stage's token ahead
 constexpr int kLLMaxCtasPerSm = 3;
 
 __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float d) {
@@ -221,6 +221,9 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float 
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
+
+static_assert(kLLInStages >= 2, "the next token must sit in another stage");
+constexpr int kLLMaxDynSmem = 227 * 1024 - 1024;  // the CTA's limit, less its static arrays
 
 // Shared-memory plan of one CTA: 128 bytes of mbarriers, kLLInStages input
 // rows (bf16, filled by bulk copies), then (FP8 only) two e4m3 output rows
@@ -666,7 +669,7 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   if (launch_status() != EP_OK) return EP_ERR_CUDA;
 
   const LLSmem plan = ll_smem_plan(H, use_fp8 != 0);
-  if (plan.bytes > 227 * 1024) return EP_ERR_UNSUPPORTED;
+  if (plan.bytes > kLLMaxDynSmem) return EP_ERR_UNSUPPORTED;
   const size_t smem = spread_smem(static_cast<size_t>(plan.bytes), kLLMaxCtasPerSm);
   const long num_tok = static_cast<long>(R) * T;
   const void *fn = use_fp8 ? reinterpret_cast<const void *>(ll_dispatch_kernel<true>)

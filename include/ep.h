@@ -346,8 +346,9 @@ EP_API size_t ep_ll_workspace_bytes(int num_ranks, int num_tokens,
  *   cumulative_local_expert_recv_stats  int32 [R, E_l] or NULL: each call adds
  *                  its recv_count (the pages' cumulative per-expert counter)
  *   workspace      ep_ll_workspace_bytes(R, T, E) bytes, any content
- * H is limited by shared memory (three staged input rows per CTA): FP8 needs
- * H <= 28672 and bf16 H <= 38720; larger returns EP_ERR_UNSUPPORTED.
+ * H is limited by shared memory (two staged input rows per CTA, plus two
+ * e4m3 rows for FP8): FP8 needs H <= 38016 and bf16 H <= 57792; larger
+ * returns EP_ERR_UNSUPPORTED.
  */
 EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
                           const int32_t *rank_mask, int num_ranks,
