@@ -343,6 +343,9 @@ LL_CASES = [
     ("h128_halfwarp", Workload("l3", R=3, T=40, H=128, E=9, K=3, seed=3), True),
     ("h640_scales_unaligned", Workload("l4", R=2, T=130, H=640, E=8, K=2, seed=4), True),
     ("pr1_shape", Workload("l5", R=4, T=64, H=256, E=16, K=2, seed=0), True),
+    # 96 scan tiles (6 per source) against ~440 dispatch CTAs: most tokens'
+    # rows are read while the scan that writes their positions still runs
+    ("many_tiles", Workload("l6", R=16, T=700, H=256, E=64, K=8, masked_frac=0.05, seed=6), True),
 ]
 
 
