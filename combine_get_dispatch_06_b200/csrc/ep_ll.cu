@@ -282,9 +282,12 @@ __global__ void __launch_bounds__(kLLThreads)
   float *scales = static_cast<float *>(scales_out);
   uint8_t *scales8 = static_cast<uint8_t *>(scales_out);
 
+  // Token blockIdx.x is this CTA's first (the grid is at most num_tok wide),
+  // so every CTA starts on the earliest tokens, whose positions the scan
+  // writes first; the rest are claimed from the counter, past the grid.
   auto take = [&]() -> long {  // thread 0: the next unclaimed token, or -1
-    const uint32_t c = atomicAdd(claim, 1u);
-    return static_cast<long>(c) < num_tok ? static_cast<long>(c) : -1L;
+    const long c = static_cast<long>(atomicAdd(claim, 1u)) + gridDim.x;
+    return c < num_tok ? c : -1L;
   };
   auto issue = [&](int stg, long u) {  // thread 0
     s_tok[stg] = u;
@@ -309,7 +312,7 @@ __global__ void __launch_bounds__(kLLThreads)
     for (int i = 0; i < kLLInStages; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
 #pragma unroll
-    for (int i = 0; i < kLLInStages; ++i) issue(i, take());
+    for (int i = 0; i < kLLInStages; ++i) issue(i, i == 0 ? static_cast<long>(blockIdx.x) : take());
     ahead = take();
   }
   __syncthreads();
