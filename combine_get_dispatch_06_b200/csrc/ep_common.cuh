@@ -76,6 +76,26 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// n / d by one multiply-high, for 0 <= n and n * d < 2^32 (expert ids and
+// experts per rank are at most 512).  m = ceil(2^32 / d) exceeds 2^32 / d by
+// less than 1, so n * m / 2^32 = n / d + err with 0 <= err < n / 2^32 < 1 / d:
+// never enough to reach the next integer.  d == 1 has no 32-bit m.
+struct FastDiv {
+  uint32_t m;
+  int d;
+};
+
+inline FastDiv make_fastdiv(int d) {
+  FastDiv f;
+  f.d = d;
+  f.m = d > 1 ? static_cast<uint32_t>((0x100000000ull + static_cast<uint64_t>(d) - 1) / d) : 0u;
+  return f;
+}
+
+__device__ __forceinline__ int fastdiv(int n, FastDiv f) {
+  return f.d == 1 ? n : static_cast<int>(__umulhi(static_cast<uint32_t>(n), f.m));
+}
+
 __device__ __forceinline__ void report(int32_t *status, int bits) {
   if (status != nullptr) atomicOr(status, bits);
 }

@@ -34,6 +34,7 @@ struct DispatchScanParams {
   const float *topk_w;
   const uint8_t *in_rank;
   int R, T, K, E, El, cap, align, tiles_per_src, num_tiles, W;
+  FastDiv el_div;  // division by El
   int32_t *send_pos;
   int32_t *recv_src_idx;
   int64_t *recv_idx;
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
           continue;
         }
         if (p.in_rank == nullptr) {
-          const int d = static_cast<int>(e) / p.El;
+          const int d = fastdiv(static_cast<int>(e), p.el_div);
           my_mask[d >> 5] |= 1u << (d & 31);
         }
         if (count_experts) atomicAdd(&s_ehist[static_cast<int>(e)], 1);
@@ -670,6 +671,7 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   p.K = K;
   p.E = E;
   p.El = topk_idx != nullptr ? E / R : 1;
+  p.el_div = make_fastdiv(p.El);
   p.cap = cap;
   p.align = align;
   p.tiles_per_src = tiles_per_src;

@@ -26,7 +26,7 @@ __device__ __forceinline__ int warp_sum(int v) {
 }
 
 __global__ void __launch_bounds__(kLayoutTile)
-    layout_kernel(const int64_t *__restrict__ topk_idx, int T, int K, int E, int R, int El,
+    layout_kernel(const int64_t *__restrict__ topk_idx, int T, int K, int E, int R, FastDiv El,
                   int tiles_per_src, int32_t *__restrict__ ntpr, int32_t *__restrict__ ntpe,
                   uint8_t *__restrict__ in_rank, int32_t *status) {
   pdl_wait();
@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(kLayoutTile)
         bad = true;
         continue;
       }
-      s_row[tid * R + static_cast<int>(e) / El] = 1;
+      s_row[tid * R + fastdiv(static_cast<int>(e), El)] = 1;
       atomicAdd(&s_exp[static_cast<int>(e)], 1);
     }
     if (bad) report(status, EP_STATUS_BAD_EXPERT);
@@ -118,7 +118,8 @@ extern "C" EP_API int ep_get_dispatch_layout(const int64_t *topk_idx, int num_sr
   const long grid = static_cast<long>(S) * tiles_per_src;
   if (grid > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
   launch_pdl(layout_kernel, dim3(static_cast<unsigned>(grid)), dim3(kLayoutTile), smem, stream,
-      topk_idx, T, K, E, R, E / R, tiles_per_src, num_tokens_per_rank, num_tokens_per_expert,
+      topk_idx, T, K, E, R, make_fastdiv(E / R), tiles_per_src, num_tokens_per_rank,
+      num_tokens_per_expert,
       is_token_in_rank, status);
   return launch_status();
 }

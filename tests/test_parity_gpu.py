@@ -48,6 +48,9 @@ LAYOUT_CASES = [
     ("r64", Workload("r64", R=64, T=130, H=0, E=128, K=8, seed=7)),
     ("r384", Workload("r384", R=384, T=3, H=0, E=384, K=16, seed=9)),
     ("e512_k16", Workload("e512", R=16, T=257, H=0, E=512, K=16, seed=11)),
+    # experts per rank not a power of two (the expert -> rank division)
+    ("el7", Workload("el7", R=6, T=200, H=0, E=42, K=5, seed=13)),
+    ("el511", Workload("el511", R=1, T=150, H=0, E=511, K=9, seed=15)),
 ]
 
 
@@ -126,6 +129,7 @@ PARITY_CASES = [
     ("r64_multiwarp", Workload("r64", R=64, T=40, H=64, E=128, K=8, seed=6), 1),
     ("k1", Workload("k1", R=3, T=257, H=8, E=3, K=1, seed=8), 1),
     ("big_row_chunks", Workload("br", R=3, T=70, H=12288, E=12, K=3, seed=10), 1),
+    ("el3_align4", Workload("e3", R=5, T=150, H=64, E=15, K=4, masked_frac=0.05, seed=14), 4),
 ]
 
 
