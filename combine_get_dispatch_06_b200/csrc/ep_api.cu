@@ -38,10 +38,6 @@ int num_sms() {
   return g_sms[dev];
 }
 
-int launch_status() {
-  return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ERR_CUDA;
-}
-
 namespace {
 std::mutex g_attr_mu;
 std::map<std::pair<const void *, int>, size_t> g_smem_set;
@@ -62,14 +58,32 @@ int ensure_dynamic_smem(const void *func, size_t bytes) {
   return EP_OK;
 }
 
+namespace {
+std::mutex g_smem_attr_mu;
+int g_smem_per_sm[kMaxDevices] = {0};
+int g_smem_reserved[kMaxDevices] = {0};
+}  // namespace
+
 size_t spread_smem(size_t smem, int n) {
-  int dev = 0, per_sm = 0, reserved = 0;
-  if (n < 1 || cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
-          cudaSuccess ||
-      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
-          cudaSuccess)
-    return smem;
+  int dev = 0;
+  if (n < 1 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return smem;
+  int per_sm, reserved;
+  {
+    std::lock_guard<std::mutex> lk(g_smem_attr_mu);
+    if (g_smem_per_sm[dev] == 0) {
+      int a = 0, b = 0;
+      if (cudaDeviceGetAttribute(&a, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+              cudaSuccess ||
+          cudaDeviceGetAttribute(&b, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
+              cudaSuccess ||
+          a <= 0)
+        return smem;
+      g_smem_per_sm[dev] = a;
+      g_smem_reserved[dev] = b;
+    }
+    per_sm = g_smem_per_sm[dev];
+    reserved = g_smem_reserved[dev];
+  }
   // n + 1 CTAs of (s + reserved) bytes overflow per_sm once s exceeds this
   const long lo = static_cast<long>(per_sm) / (n + 1) - reserved + 16;
   const size_t want = static_cast<size_t>((std::max<long>(lo, 0) + 15) & ~15L);

@@ -145,9 +145,10 @@ extern "C" EP_API int ep_combine(const void *y, const float *recv_topk_weights,
   const long want = (num_tok + kCombineWarps - 1) / kCombineWarps;
   const long grid =
       std::min<long>(want, static_cast<long>(ctas_per_sm(fn, threads, smem)) * num_sms());
-  launch_pdl(combine_kernel, dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream,
+  const cudaError_t launched = launch_pdl(combine_kernel,
+      dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream,
       static_cast<const uint8_t *>(y), combined_topk_weights ? recv_topk_weights : nullptr,
       send_pos, static_cast<const uint8_t *>(bias_0), static_cast<const uint8_t *>(bias_1), R,
       num_tok, H, K, cap, static_cast<uint8_t *>(combined_x), combined_topk_weights, status);
-  return launch_status();
+  return launch_status(launched);
 }

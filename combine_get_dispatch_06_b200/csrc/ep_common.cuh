@@ -28,8 +28,12 @@ WaitConfig wait_config();
 // Number of SMs of the current device (cached per device).
 int num_sms();
 
-// Returns EP_ERR_CUDA if the last launch failed.
-int launch_status();
+// EP_OK for a launch that returned cudaSuccess, else EP_ERR_CUDA.  The
+// launch's own return value is used, not cudaGetLastError(), which would
+// also report (and clear) an error some other code left behind.
+inline int launch_status(cudaError_t launched) {
+  return launched == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
 
 // Raise the dynamic shared-memory limit of `func` on the current device to at
 // least `bytes` (needed above 48 KiB).  Cached per (function, device).

@@ -696,20 +696,23 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   const WaitConfig wc = wait_config();
   p.timeout_ns = wc.timeout_ns;
   p.flags = wc.flags;
+  cudaError_t launched;
   if (topk_idx != nullptr && K > 8)
-    launch_pdl(dispatch_scan_kernel<16>, dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
+    launched = launch_pdl(dispatch_scan_kernel<16>,
+        dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
         p);
   else
-    launch_pdl(dispatch_scan_kernel<8>, dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
+    launched = launch_pdl(dispatch_scan_kernel<8>,
+        dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
         p);
-  if (launch_status() != EP_OK) return EP_ERR_CUDA;
+  if (launch_status(launched) != EP_OK) return EP_ERR_CUDA;
   // rows past the receive count read -1 (fixed worst-case capacity)
   if (recv_topk_idx != nullptr && cap > 0) {
     const long words = static_cast<long>(cap) * K / ((K & 1) == 0 ? 2 : 1);
     const int bx = static_cast<int>(std::min<long>((words + 255) / 256, 64));
-    launch_pdl(pad_recv_idx_kernel, dim3(bx, R), dim3(256), 0, stream,
+    launched = launch_pdl(pad_recv_idx_kernel, dim3(bx, R), dim3(256), 0, stream,
         recv_count, cap, K, recv_topk_idx);
-    return launch_status();
+    return launch_status(launched);
   }
   return EP_OK;
 }
@@ -766,23 +769,27 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
       a.num_tok,
       static_cast<long>(std::min(kCopyMaxCtasPerSm, ctas_per_sm(fn, threads, smem))) * num_sms());
   const dim3 g(static_cast<unsigned>(grid)), b(threads);
+  cudaError_t launched;
   if (xs != nullptr) {
     if (short_rows)
-      launch_pdl(dispatch_copy_planes_kernel<kCopyStagesShort, true>, dim3(g), dim3(b), smem, stream,
+      launched = launch_pdl(dispatch_copy_planes_kernel<kCopyStagesShort, true>,
+          dim3(g), dim3(b), smem, stream,
         a);
     else
-      launch_pdl(dispatch_copy_planes_kernel<kCopyStages, true>, dim3(g), dim3(b), smem, stream,
+      launched = launch_pdl(dispatch_copy_planes_kernel<kCopyStages, true>,
+          dim3(g), dim3(b), smem, stream,
         a);
   } else if (short_rows) {
-    launch_pdl(dispatch_copy_rows_kernel<kCopyStagesShort>, dim3(g), dim3(b), smem, stream,
+    launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStagesShort>,
+        dim3(g), dim3(b), smem, stream,
         a.x, a.send_pos, a.recv_x, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
         a.stage_stride, a.cap, a.status, a.timeout_ns);
   } else {
-    launch_pdl(dispatch_copy_rows_kernel<kCopyStages>, dim3(g), dim3(b), smem, stream,
+    launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStages>, dim3(g), dim3(b), smem, stream,
         a.x, a.send_pos, a.recv_x, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
         a.stage_stride, a.cap, a.status, a.timeout_ns);
   }
-  return launch_status();
+  return launch_status(launched);
 }
 
 // Checks shared by ep_dispatch and ep_notify_dispatch.

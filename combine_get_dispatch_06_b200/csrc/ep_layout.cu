@@ -117,9 +117,10 @@ extern "C" EP_API int ep_get_dispatch_layout(const int64_t *topk_idx, int num_sr
     return EP_ERR_CUDA;
   const long grid = static_cast<long>(S) * tiles_per_src;
   if (grid > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
-  launch_pdl(layout_kernel, dim3(static_cast<unsigned>(grid)), dim3(kLayoutTile), smem, stream,
+  const cudaError_t launched = launch_pdl(layout_kernel,
+      dim3(static_cast<unsigned>(grid)), dim3(kLayoutTile), smem, stream,
       topk_idx, T, K, E, R, make_fastdiv(E / R), tiles_per_src, num_tokens_per_rank,
       num_tokens_per_expert,
       is_token_in_rank, status);
-  return launch_status();
+  return launch_status(launched);
 }

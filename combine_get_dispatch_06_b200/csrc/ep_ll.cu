@@ -663,13 +663,16 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   const WaitConfig wc = wait_config();
   p.timeout_ns = wc.timeout_ns;
   p.flags = wc.flags;
+  cudaError_t launched;
   if (K > 8)
-    launch_pdl(ll_scan_kernel<16>, dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
+    launched = launch_pdl(ll_scan_kernel<16>,
+        dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
         p);
   else
-    launch_pdl(ll_scan_kernel<8>, dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
+    launched = launch_pdl(ll_scan_kernel<8>,
+        dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
         p);
-  if (launch_status() != EP_OK) return EP_ERR_CUDA;
+  if (launch_status(launched) != EP_OK) return EP_ERR_CUDA;
 
   const LLSmem plan = ll_smem_plan(H, use_fp8 != 0);
   if (plan.bytes > kLLMaxDynSmem) return EP_ERR_UNSUPPORTED;
@@ -683,16 +686,18 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
       static_cast<long>(std::min(kLLMaxCtasPerSm, ctas_per_sm(fn, kLLThreads, smem))) *
           num_sms());
   if (use_fp8)
-    launch_pdl(ll_dispatch_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
+    launched = launch_pdl(ll_dispatch_kernel<true>,
+        dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
         static_cast<const uint8_t *>(x), topk_idx, p.pos_mirror, num_tok, H, K, E,
         static_cast<int>(cap), round_scale, ue8m0, plan, static_cast<uint8_t *>(recv_x),
         recv_scales, &p.head->claim, status, wc.timeout_ns);
   else
-    launch_pdl(ll_dispatch_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
+    launched = launch_pdl(ll_dispatch_kernel<false>,
+        dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
         static_cast<const uint8_t *>(x), topk_idx, p.pos_mirror, num_tok, H, K, E,
         static_cast<int>(cap), 0, 0, plan, static_cast<uint8_t *>(recv_x), nullptr,
         &p.head->claim, status, wc.timeout_ns);
-  return launch_status();
+  return launch_status(launched);
 }
 
 extern "C" EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
@@ -723,8 +728,9 @@ extern "C" EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
   nseg = std::max(1, std::min(nseg, std::max(1, nvec / 32)));
   const long items = num_tok * nseg;
   const long grid = std::min<long>((items + kLLCombineWarps - 1) / kLLCombineWarps, resident);
-  launch_pdl(ll_combine_kernel, dim3(static_cast<unsigned>(grid)), dim3(threads), 0, stream,
+  const cudaError_t launched = launch_pdl(ll_combine_kernel,
+      dim3(static_cast<unsigned>(grid)), dim3(threads), 0, stream,
       static_cast<const uint8_t *>(y), topk_idx, topk_weights, ll_pos, rank_mask, num_tok, T, H,
       K, E, static_cast<int>(cap), nseg, static_cast<uint8_t *>(out), status);
-  return launch_status();
+  return launch_status(launched);
 }
