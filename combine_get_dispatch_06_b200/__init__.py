@@ -12,6 +12,7 @@ Layouts and semantics are those of ``include/ep.h``.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 from typing import Optional
 
@@ -81,6 +82,8 @@ def _ptr(t: Optional[torch.Tensor]):
         return None
     if not t.is_cuda:
         raise EPError("all tensors passed to libep must be CUDA tensors")
+    if t.device.index != torch.cuda.current_device():
+        raise EPError("all tensors of one call must be on the same CUDA device")
     if not t.is_contiguous():
         raise EPError("all tensors passed to libep must be contiguous")
     return t.data_ptr()
@@ -90,6 +93,20 @@ def _stream(stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream()
     return stream.cuda_stream
+
+
+def _on_tensor_device(fn):
+    """Run a wrapper with the device of its first CUDA tensor argument
+    current, so that allocations, the default stream and the library's
+    per-device settings all refer to that device."""
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        for a in list(args) + list(kwargs.values()):
+            if isinstance(a, torch.Tensor) and a.is_cuda:
+                with torch.cuda.device(a.device):
+                    return fn(*args, **kwargs)
+        return fn(*args, **kwargs)
+    return wrapper
 
 
 def _need(t: torch.Tensor, dtype, shape, name):
@@ -125,6 +142,7 @@ def new_status(device=None) -> torch.Tensor:
 # A1
 # ---------------------------------------------------------------------------
 
+@_on_tensor_device
 def ep_get_dispatch_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, *,
                            num_tokens_per_rank=None, num_tokens_per_expert=None,
                            is_token_in_rank=None, status=None, stream=None):
@@ -170,6 +188,7 @@ def ep_dispatch_workspace_bytes(num_ranks: int, num_tokens: int, num_experts: in
     return int(_lib.ep_dispatch_workspace_bytes(num_ranks, num_tokens, num_experts))
 
 
+@_on_tensor_device
 def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor],
                 topk_weights: Optional[torch.Tensor], num_experts: int, *,
                 is_token_in_rank: Optional[torch.Tensor] = None, expert_alignment: int = 1,
@@ -224,6 +243,7 @@ def ep_dispatch(x: torch.Tensor, topk_idx: Optional[torch.Tensor],
     return o
 
 
+@_on_tensor_device
 def ep_notify_dispatch(topk_idx: Optional[torch.Tensor], topk_weights: Optional[torch.Tensor],
                        num_tokens: int, num_ranks: int, num_experts: int, *,
                        is_token_in_rank: Optional[torch.Tensor] = None,
@@ -287,6 +307,7 @@ def ep_notify_dispatch(topk_idx: Optional[torch.Tensor], topk_weights: Optional[
     return o
 
 
+@_on_tensor_device
 def ep_dispatch_cached(x: torch.Tensor, send_pos: torch.Tensor, *, capacity: Optional[int] = None,
                        recv_x: Optional[torch.Tensor] = None, status=None,
                        stream=None) -> torch.Tensor:
@@ -304,6 +325,7 @@ def ep_dispatch_cached(x: torch.Tensor, send_pos: torch.Tensor, *, capacity: Opt
     return recv_x
 
 
+@_on_tensor_device
 def ep_dispatch_cached_fp8(x_e4m3: torch.Tensor, x_scales: torch.Tensor, send_pos: torch.Tensor,
                            *, scales_col_major: bool = False, capacity: Optional[int] = None,
                            recv_x: Optional[torch.Tensor] = None,
@@ -331,6 +353,7 @@ def ep_dispatch_cached_fp8(x_e4m3: torch.Tensor, x_scales: torch.Tensor, send_po
     return recv_x, recv_scales
 
 
+@_on_tensor_device
 def ep_dispatch_noalloc(x: torch.Tensor, topk_idx: Optional[torch.Tensor],
                         topk_weights: Optional[torch.Tensor], num_experts: int, *,
                         is_token_in_rank: Optional[torch.Tensor] = None,
@@ -374,6 +397,7 @@ def ep_dispatch_noalloc(x: torch.Tensor, topk_idx: Optional[torch.Tensor],
 # A4
 # ---------------------------------------------------------------------------
 
+@_on_tensor_device
 def ep_combine(y: torch.Tensor, send_pos: torch.Tensor,
                recv_topk_weights: Optional[torch.Tensor] = None, *,
                bias: Optional[tuple] = None,
@@ -417,6 +441,7 @@ def ep_ll_workspace_bytes(num_ranks: int, num_tokens: int, num_experts: int) -> 
     return int(_lib.ep_ll_workspace_bytes(num_ranks, num_tokens, num_experts))
 
 
+@_on_tensor_device
 def ep_ll_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int, *,
                    use_fp8: bool = True, round_scale: bool = False, use_ue8m0: bool = False,
                    rank_mask: Optional[torch.Tensor] = None,
@@ -469,6 +494,7 @@ def ep_ll_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, num_experts: int, *,
     return o
 
 
+@_on_tensor_device
 def ep_ll_combine(y: torch.Tensor, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
                   ll_pos: torch.Tensor, *, rank_mask: Optional[torch.Tensor] = None,
                   out: Optional[torch.Tensor] = None, status=None,
