@@ -16,12 +16,16 @@
 //     rounding at the end.
 //
 // Kernels:
-//   ll_scan_kernel      positions, recv_src_info, layout_range, counts
-//   ll_dispatch_kernel  one warp per token: read the row once, quantise in
-//                       registers (16 lanes per 128-channel block, amax by
-//                       xor-shuffles), stage it in shared memory, then one
-//                       bulk (TMA) store per destination slab row
-//   ll_combine_kernel   one warp per token, up to 16 rows in flight per lane
+//   ll_scan_kernel      positions, recv_src_info, layout_range, counts, and
+//                       a mirror of the positions for the dispatch kernel
+//   ll_dispatch_kernel  runs concurrently with the scan; one CTA per token at
+//                       a time (tokens claimed from a counter): read the row
+//                       once by a bulk copy, quantise it (16 threads per
+//                       128-channel block, amax by xor-shuffles) into shared
+//                       memory, then one bulk (TMA) store per destination
+//                       slab row once the scan has written its position
+//   ll_combine_kernel   one warp per (token, channel segment), up to 8 rows
+//                       in flight per lane
 #include <algorithm>
 
 #include "ep_scan.cuh"
