@@ -64,7 +64,7 @@ extern "C" {
 #define EP_OK               0  /* launched                                   */
 #define EP_ERR_INVALID_ARG  1  /* a size, pointer or alignment check failed  */
 #define EP_ERR_CUDA         2  /* the CUDA runtime reported a launch error   */
-#define EP_ERR_UNSUPPORTED  3  /* valid call, shape this build cannot run    */
+#define EP_ERR_UNSUPPORTED  3  /* valid call, shape the library cannot run   */
 
 /* Device-side status bits, OR-ed into `status`. */
 #define EP_STATUS_BAD_EXPERT       1  /* a top-k id outside [-1, E); slot ignored      */
