@@ -130,6 +130,8 @@ PARITY_CASES = [
     ("k1", Workload("k1", R=3, T=257, H=8, E=3, K=1, seed=8), 1),
     ("big_row_chunks", Workload("br", R=3, T=70, H=12288, E=12, K=3, seed=10), 1),
     ("el3_align4", Workload("e3", R=5, T=150, H=64, E=15, K=4, masked_frac=0.05, seed=14), 4),
+    # the largest rank count (12 warps per copy CTA, 384-bit routing masks)
+    ("r384_max", Workload("r384", R=384, T=3, H=64, E=384, K=4, seed=16), 1),
 ]
 
 
@@ -702,6 +704,34 @@ def test_ll_k16_e512():
     co = ep.ep_ll_combine(to_dev(y), idd, to_dev(wts), out["ll_pos"], status=st)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(to_host(co), oracle.ll_combine(y, idx, wts, ref["ll_pos"]))
+
+
+@pytest.mark.parametrize("fp8,H_max,H_over", [(True, 38016, 38144), (False, 57792, 57800)])
+def test_ll_largest_hidden_and_one_past(fp8, H_max, H_over):
+    """LL rows are staged whole in shared memory: the largest hidden size the
+    header states runs bit-exact, the next step is refused before launch."""
+    w = Workload("llh", R=2, T=5, H=H_max, E=4, K=2, seed=74)
+    inp = make(w)
+    x, idx = inp["x"], inp["topk_idx"]
+    ref = oracle.ll_layout(idx, w.E)
+    rq, rs = oracle.ll_dispatch_rows(x, idx, ref["ll_pos"], w.E, use_fp8=fp8)
+    st = ep.new_status()
+    out = ep.ep_ll_dispatch(to_dev(x), to_dev(idx), w.E, use_fp8=fp8, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(to_host(out["ll_pos"]), ref["ll_pos"])
+    q = to_host(out["recv_x"])
+    sc = to_host(out["recv_scales"]) if fp8 else None
+    for d in range(w.R):
+        for j in range(w.E // w.R):
+            n = ref["recv_count"][d, j]
+            np.testing.assert_array_equal(q[d, j, :n], rq[d, j, :n])
+            if fp8:
+                np.testing.assert_array_equal(sc[d, j, :n], rs[d, j, :n])
+    w2 = Workload("llh2", R=2, T=5, H=H_over, E=4, K=2, seed=75)
+    inp2 = make(w2)
+    with pytest.raises(ep.EPError, match="unsupported"):
+        ep.ep_ll_dispatch(to_dev(inp2["x"]), to_dev(inp2["topk_idx"]), w2.E, use_fp8=fp8)
 
 
 def test_fp8_input_dispatch_r40_multiwarp():
