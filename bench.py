@@ -422,10 +422,10 @@ def run_ours(args) -> None:
     import torch.distributed as dist
 
     ws, rank, local = dist_env()
-    if ws > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
+    torch.cuda.set_device(device)  # before the process group: NCCL binds this device
+    if ws > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     import combine_get_dispatch_06_b200 as ep  # fails loudly without libep.so
 
     w = CONFIGS["normal"]
