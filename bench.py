@@ -355,17 +355,17 @@ def extra_configs(device, ep) -> dict:
     x = to_dev_bf16(inp["x"], device)
     idx = torch.from_numpy(inp["topk_idx"]).to(device)
     wt = torch.from_numpy(inp["topk_weights"]).to(device)
-    a, b, c = ep.ep_get_dispatch_layout(idx, w.E, w.R)
-    d = ep.ep_dispatch(x, idx, wt, w.E, is_token_in_rank=c)
+    # the same call sequence as the headline step: layout fused into notify
+    d = ep.ep_notify_dispatch(idx, wt, w.T, w.R, w.E, with_layout=True)
+    d["recv_x"] = ep.ep_dispatch_cached(x, d["send_pos"])
     cx, cw = ep.ep_combine(d["recv_x"], d["send_pos"], d["recv_topk_weights"])
     wsp = torch.empty(ep.ep_dispatch_workspace_bytes(w.R, w.T, w.E), dtype=torch.uint8,
                       device=device)
     buf = {"d": d}
 
     def sk():
-        ep.ep_get_dispatch_layout(idx, w.E, w.R, num_tokens_per_rank=a, num_tokens_per_expert=b,
-                                  is_token_in_rank=c)
-        ep.ep_dispatch(x, idx, wt, w.E, is_token_in_rank=c, out=d, workspace=wsp)
+        ep.ep_notify_dispatch(idx, wt, w.T, w.R, w.E, with_layout=True, out=d, workspace=wsp)
+        ep.ep_dispatch_cached(x, d["send_pos"], recv_x=d["recv_x"])
         ep.ep_combine(d["recv_x"], d["send_pos"], d["recv_topk_weights"], combined_x=cx,
                       combined_topk_weights=cw)
     ms = timeit(sk, iters=20)
@@ -373,7 +373,7 @@ def extra_configs(device, ep) -> dict:
     nb = dispatch_bytes(w.R, w.T, w.H, w.K, N) + combine_bytes(w.R, w.T, w.H, w.K, N)
     out["skewed"] = {"ms": ms, "gbs": nb / (ms * 1e-3) / 1e9, "copies": N,
                      "tokens_per_s": w.R * w.T / (ms * 1e-3)}
-    del x, idx, wt, buf, d, cx, cw, a, b, c, wsp
+    del x, idx, wt, buf, d, cx, cw, wsp
     torch.cuda.empty_cache()
 
     # low latency: FP8 dispatch + weighted combine
