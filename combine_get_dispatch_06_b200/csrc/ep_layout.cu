@@ -12,6 +12,15 @@
 // bin, and the byte matrix is written out with 16-byte stores.  Integer
 // atomics make the result independent of the order in which tiles finish.
 // Bound: latency (the whole input of the 4096 x 8 case is 256 KiB).
+//
+// Up to 4096 tokens per source rank and 32 ranks, one thread-block cluster of
+// 8 CTAs (512 tokens each) takes a whole source rank instead: each CTA counts
+// its tokens in shared memory, adds the counts into CTA 0's shared memory
+// through the cluster's distributed shared memory, and CTA 0 stores every
+// count of the source rank -- no global atomics and no zeroing of the outputs
+// beforehand.
+#include <cooperative_groups.h>
+
 #include "ep_common.cuh"
 
 namespace ep {
@@ -89,6 +98,80 @@ __global__ void __launch_bounds__(kLayoutTile)
   }
 }
 
+constexpr int kClusterCtas = 8;
+constexpr int kClusterThreads = 512;                            // one token per thread
+constexpr int kClusterTokens = kClusterCtas * kClusterThreads;  // per source rank
+constexpr int kClusterMaxRanks = 32;                            // rank set in one word
+
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterThreads)
+    layout_cluster_kernel(const int64_t *__restrict__ topk_idx, int T, int K, int E, int R,
+                          FastDiv El, int32_t *__restrict__ ntpr, int32_t *__restrict__ ntpe,
+                          uint8_t *__restrict__ in_rank, int32_t *status) {
+  namespace cg = cooperative_groups;
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int s_exp[kMaxExperts];         // this CTA's counts; CTA 0: the source's
+  __shared__ int s_rank[kClusterMaxRanks];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = static_cast<int>(cluster.block_rank());
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int s = blockIdx.x / kClusterCtas;
+  const int t = crank * kClusterThreads + tid;
+
+  for (int i = tid; i < E; i += kClusterThreads) s_exp[i] = 0;
+  if (tid < R) s_rank[tid] = 0;
+  cluster.sync();  // CTA 0's counters are zero before any CTA adds to them
+
+  uint32_t ranks = 0;  // bit d: the token goes to rank d
+  if (t < T) {
+    const int64_t *idx = topk_idx + (static_cast<size_t>(s) * T + t) * K;
+    int64_t ek[kMaxTopk];
+#pragma unroll
+    for (int k = 0; k < kMaxTopk; ++k) ek[k] = k < K ? __ldg(idx + k) : -1;
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < kMaxTopk; ++k) {
+      const int64_t e = ek[k];
+      if (k >= K || e == -1) continue;
+      if (e < -1 || e >= E) {
+        bad = true;
+        continue;
+      }
+      ranks |= 1u << fastdiv(static_cast<int>(e), El);
+      atomicAdd(&s_exp[static_cast<int>(e)], 1);
+    }
+    if (bad) report(status, EP_STATUS_BAD_EXPERT);
+    uint8_t *row = in_rank + (static_cast<size_t>(s) * T + t) * R;
+    if ((R & 3) == 0 && (reinterpret_cast<uintptr_t>(in_rank) & 3u) == 0) {
+      for (int d = 0; d < R; d += 4) {  // four 0/1 bytes per 32-bit store
+        const uint32_t b = ranks >> d;
+        reinterpret_cast<uint32_t *>(row)[d >> 2] =
+            (b & 1u) | ((b >> 1) & 1u) << 8 | ((b >> 2) & 1u) << 16 | ((b >> 3) & 1u) << 24;
+      }
+    } else {
+      for (int d = 0; d < R; ++d) row[d] = (ranks >> d) & 1u;
+    }
+  }
+  for (int d = 0; d < R; ++d) {  // tokens per rank, a warp at a time
+    const int c = __popc(__ballot_sync(0xffffffffu, (ranks >> d) & 1u));
+    if (lane == 0 && c != 0) atomicAdd(&s_rank[d], c);
+  }
+  __syncthreads();
+  if (crank != 0) {  // into CTA 0's shared memory
+    int *r_exp = cluster.map_shared_rank(s_exp, 0);
+    int *r_rank = cluster.map_shared_rank(s_rank, 0);
+    for (int e = tid; e < E; e += kClusterThreads)
+      if (s_exp[e] != 0) atomicAdd(&r_exp[e], s_exp[e]);
+    if (tid < R && s_rank[tid] != 0) atomicAdd(&r_rank[tid], s_rank[tid]);
+  }
+  cluster.sync();  // every CTA's counts are in CTA 0
+  if (crank == 0) {
+    for (int e = tid; e < E; e += kClusterThreads) ntpe[static_cast<size_t>(s) * E + e] = s_exp[e];
+    if (tid < R) ntpr[static_cast<size_t>(s) * R + tid] = s_rank[tid];
+  }
+}
+
 }  // namespace
 }  // namespace ep
 
@@ -106,6 +189,15 @@ extern "C" EP_API int ep_get_dispatch_layout(const int64_t *topk_idx, int num_sr
   if (num_tokens_per_rank == nullptr || num_tokens_per_expert == nullptr)
     return EP_ERR_INVALID_ARG;
   if (T > 0 && (topk_idx == nullptr || is_token_in_rank == nullptr)) return EP_ERR_INVALID_ARG;
+  if (T > 0 && T <= kClusterTokens && R <= kClusterMaxRanks) {
+    // one cluster per source rank; it stores every count, nothing to zero
+    if (static_cast<long>(S) * kClusterCtas > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
+    const cudaError_t launched = launch_pdl(layout_cluster_kernel,
+        dim3(static_cast<unsigned>(S) * kClusterCtas), dim3(kClusterThreads), 0, stream,
+        topk_idx, T, K, E, R, make_fastdiv(E / R), num_tokens_per_rank, num_tokens_per_expert,
+        is_token_in_rank, status);
+    return launch_status(launched);
+  }
   if (cudaMemsetAsync(num_tokens_per_rank, 0, sizeof(int32_t) * S * R, stream) != cudaSuccess ||
       cudaMemsetAsync(num_tokens_per_expert, 0, sizeof(int32_t) * static_cast<size_t>(S) * E,
                       stream) != cudaSuccess)

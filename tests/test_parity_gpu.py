@@ -51,6 +51,9 @@ LAYOUT_CASES = [
     # experts per rank not a power of two (the expert -> rank division)
     ("el7", Workload("el7", R=6, T=200, H=0, E=42, K=5, seed=13)),
     ("el511", Workload("el511", R=1, T=150, H=0, E=511, K=9, seed=15)),
+    # past one 8-CTA cluster per source rank (4096 tokens): the tile kernel
+    ("t5000_tiles", Workload("t5k", R=8, T=5000, H=0, E=64, K=6, masked_frac=0.05, seed=17)),
+    ("r33_tiles", Workload("r33", R=33, T=300, H=0, E=66, K=4, seed=18)),
 ]
 
 
@@ -68,9 +71,10 @@ def test_layout_parity(name, w):
     assert int(st.item()) == 0
 
 
-def test_layout_bad_ids_and_duplicates():
+@pytest.mark.parametrize("T", [150, 4200], ids=["cluster", "tiles"])
+def test_layout_bad_ids_and_duplicates(T):
     rng = np.random.default_rng(1)
-    R, T, K, E = 4, 150, 4, 16
+    R, K, E = 4, 4, 16
     idx = rng.integers(0, E, size=(R, T, K)).astype(np.int64)
     idx[:, ::7, 1] = idx[:, ::7, 0]          # repeated experts
     idx[:, ::5, 2] = -1
