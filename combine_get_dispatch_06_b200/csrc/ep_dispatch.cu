@@ -53,12 +53,13 @@ struct DispatchScanParams {
   unsigned flags;
 };
 
-// Received top-k metadata of one copy held by a rank whose experts are
-// [lo, hi): local id for local slots, -1 / 0.0 otherwise.  16-byte stores
-// when K allows them (rows of K int64 / K fp32 are then 16-byte aligned).
+// Received top-k metadata of the copy held by rank d: the local id of every
+// slot whose expert lives on d (dk[k] == d, lk[k] its local id), -1 and 0.0
+// for the others.  32-bit compares and selects; 16-byte stores when K allows
+// them (rows of K int64 / K fp32 are then 16-byte aligned).
 template <int MAXK>
 __device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, size_t row, int K,
-                                           int64_t lo, int64_t hi, const int64_t (&ek)[MAXK],
+                                           int d, const int (&dk)[MAXK], const int (&lk)[MAXK],
                                            const float (&wk)[MAXK]) {
   if (recv_idx != nullptr) {
     int64_t *dst = recv_idx + row * K;
@@ -67,15 +68,15 @@ __device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, siz
       for (int k = 0; k < MAXK; k += 2) {
         if (k < K) {
           longlong2 v;
-          v.x = (ek[k] >= lo && ek[k] < hi) ? ek[k] - lo : -1;
-          v.y = (ek[k + 1] >= lo && ek[k + 1] < hi) ? ek[k + 1] - lo : -1;
+          v.x = dk[k] == d ? static_cast<int64_t>(lk[k]) : -1ll;
+          v.y = dk[k + 1] == d ? static_cast<int64_t>(lk[k + 1]) : -1ll;
           *reinterpret_cast<longlong2 *>(dst + k) = v;
         }
       }
     } else {
 #pragma unroll
       for (int k = 0; k < MAXK; ++k)
-        if (k < K) dst[k] = (ek[k] >= lo && ek[k] < hi) ? ek[k] - lo : -1;
+        if (k < K) dst[k] = dk[k] == d ? static_cast<int64_t>(lk[k]) : -1ll;
     }
   }
   if (recv_w != nullptr) {
@@ -85,17 +86,17 @@ __device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, siz
       for (int k = 0; k < MAXK; k += 4) {
         if (k < K) {
           float4 v;
-          v.x = (ek[k] >= lo && ek[k] < hi) ? wk[k] : 0.f;
-          v.y = (ek[k + 1] >= lo && ek[k + 1] < hi) ? wk[k + 1] : 0.f;
-          v.z = (ek[k + 2] >= lo && ek[k + 2] < hi) ? wk[k + 2] : 0.f;
-          v.w = (ek[k + 3] >= lo && ek[k + 3] < hi) ? wk[k + 3] : 0.f;
+          v.x = dk[k] == d ? wk[k] : 0.f;
+          v.y = dk[k + 1] == d ? wk[k + 1] : 0.f;
+          v.z = dk[k + 2] == d ? wk[k + 2] : 0.f;
+          v.w = dk[k + 3] == d ? wk[k + 3] : 0.f;
           *reinterpret_cast<float4 *>(dst + k) = v;
         }
       }
     } else {
 #pragma unroll
       for (int k = 0; k < MAXK; ++k)
-        if (k < K) dst[k] = (ek[k] >= lo && ek[k] < hi) ? wk[k] : 0.f;
+        if (k < K) dst[k] = dk[k] == d ? wk[k] : 0.f;
     }
   }
 }
@@ -144,6 +145,16 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
     }
   }
 
+  // destination rank and local id of every valid slot (-1: none)
+  int dk[MAXK], lk[MAXK];
+#pragma unroll
+  for (int k = 0; k < MAXK; ++k) {
+    const int64_t e = ek[k];
+    const bool ok = k < p.K && e >= 0 && e < p.E;
+    dk[k] = ok ? fastdiv(static_cast<int>(e), p.el_div) : -1;
+    lk[k] = ok ? static_cast<int>(e) - dk[k] * p.El : 0;
+  }
+
   // ---- routing bits of this token --------------------------------------
   uint32_t *my_mask = s_mask + tid * p.W;
   for (int w = 0; w < p.W; ++w) my_mask[w] = 0u;
@@ -164,10 +175,7 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
           bad = true;
           continue;
         }
-        if (p.in_rank == nullptr) {
-          const int d = fastdiv(static_cast<int>(e), p.el_div);
-          my_mask[d >> 5] |= 1u << (d & 31);
-        }
+        if (p.in_rank == nullptr) my_mask[dk[k] >> 5] |= 1u << (dk[k] & 31);
         if (count_experts) atomicAdd(&s_ehist[static_cast<int>(e)], 1);
       }
       if (bad) report(p.status, EP_STATUS_BAD_EXPERT);
@@ -253,8 +261,7 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
       }
       const size_t row = static_cast<size_t>(d) * p.cap + pos;
       p.recv_src_idx[row] = t;
-      if (meta) write_meta(p.recv_idx, p.recv_w, row, p.K, static_cast<int64_t>(d) * p.El,
-                           static_cast<int64_t>(d + 1) * p.El, ek, wk);
+      if (meta) write_meta(p.recv_idx, p.recv_w, row, p.K, d, dk, lk, wk);
     }
   }
   if (overflow) report(p.status, EP_STATUS_CAPACITY);
