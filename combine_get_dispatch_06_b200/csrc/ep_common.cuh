@@ -53,9 +53,11 @@ size_t spread_smem(size_t smem, int n);
 // with programmatic stream serialization.  It calls pdl_wait() before it reads
 // or writes any global memory: that waits until the previous grid in the
 // stream has completed and its writes are visible, so results keep stream
-// order.  It calls pdl_trigger() once its main work is issued: the next
-// kernel may then be scheduled (its CTAs start and block in their own
-// pdl_wait()), which hides its launch latency behind this kernel's tail.
+// order.  (One exception, argued where it is made: the LL dispatch kernel runs
+// alongside the LL scan and waits for it only before it exits.)  It calls
+// pdl_trigger() once its main work is issued: the next kernel may then be
+// scheduled (its CTAs start and block in their own pdl_wait()), which hides
+// its launch latency behind this kernel's tail.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, Args &&...args) {
