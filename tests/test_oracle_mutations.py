@@ -69,6 +69,24 @@ MUTANTS = [
     ("ll_mask_ignores_destination",
      "                if (mask && (mask[s] || mask[e / El])) {\n                    ll_pos[st * K + k] = -1;",
      "                if (mask && mask[s]) {\n                    ll_pos[st * K + k] = -1;"),
+    ("expert_counts_aligned_down",
+     "                n = (n + align - 1) / align * align;",
+     "                n = n / align * align;"),
+    ("handle_stores_source_rank",
+     "                    recv_src_idx[(size_t)d * cap + row] = t;",
+     "                    recv_src_idx[(size_t)d * cap + row] = s;"),
+    ("dispatch_copies_neighbour_row",
+     "                   x + (size_t)st * H, sizeof(uint16_t) * (size_t)H);",
+     "                   x + (size_t)(st + (st + 1 < (long)R * T)) * H, sizeof(uint16_t) * (size_t)H);"),
+    ("combined_weights_last_copy_only",
+     "                    acc = acc + recv_w[((size_t)d * cap + row) * K + k];",
+     "                    acc = recv_w[((size_t)d * cap + row) * K + k];"),
+    ("ll_range_begin_after_source",
+     "        for (int e = 0; e < E; ++e)\n            layout_range[((size_t)e * R + s) * 2 + 0] = count[e];\n        for (int t = 0; t < T; ++t) {",
+     "        for (int t = 0; t < T; ++t) {"),
+    ("dequant_by_inverse_scale",
+     "            float v = orc_e4m3_to_f32(q[(size_t)r * H + h]) *\n                      scales[(size_t)r * (H / 128) + h / 128];",
+     "            float v = orc_e4m3_to_f32(q[(size_t)r * H + h]) /\n                      scales[(size_t)r * (H / 128) + h / 128];"),
 ]
 
 
@@ -85,6 +103,7 @@ def test_pins_fail_on_mutant(name, find, repl, tmp_path):
                            "-o", str(lib), str(csrc), "-lm"])
     env = dict(os.environ, EP_ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests",
-                        "test_oracle_pins.py"), "-x", "-q", "-p", "no:cacheprovider"],
+                        "test_oracle_pins.py"), "-x", "-q", "-p", "no:cacheprovider",
+                        f"--basetemp={tmp_path / 'inner'}"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-1500:]}"
