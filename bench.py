@@ -213,6 +213,17 @@ def cpu_baseline(w: Workload, T_sample: int = 2048, reps: int = 3) -> dict:
             "tokens_per_s": ntok / dt, "seconds": dt}
 
 
+def workload_config(T: int, ws: int) -> dict:
+    """The `config` of the JSON line, the same for both arms."""
+    w = CONFIGS["normal"]
+    return {"workload": f"normal: R={w.R} simulated ranks x T={T} tokens x H={w.H} bf16, "
+                        f"E={w.E} experts, top-{w.K} distinct uniform, fp32 softmax weights, "
+                        "identity experts",
+            "global_batch": w.R * T * ws, "seq_len": None,
+            "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
+            "l2": "inputs larger than L2 (x 470 MB, recv_x 2.5 GB written); no flush"}
+
+
 def run_reference(args) -> None:
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -235,11 +246,11 @@ def run_reference(args) -> None:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "normal: R=8 x T=4096 x H=7168 bf16, E=256, top-8 (oracle on a "
-                               f"sample of {T_sample} tokens per source rank)",
-                   "global_batch": w.R * T_sample, "seq_len": None, "parallelism": "replicas"},
+        "config": workload_config(w.T, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"first {T_sample} tokens of each of the 8 source ranks per step"},
+                         "sample": (f"each step runs the C oracle single-threaded on the first "
+                                    f"{T_sample} of {w.T} tokens of each of the {w.R} source "
+                                    "ranks (bytes and tokens counted for that sample)")},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "tokens_per_s": tot_tok / dt,
     }
@@ -594,12 +605,7 @@ def run_ours(args) -> None:
         "metric": METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": agg["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"normal: R=8 simulated ranks x T={T} tokens x H=7168 bf16, "
-                               "E=256 experts, top-8 distinct uniform, fp32 softmax weights, "
-                               "identity experts",
-                   "global_batch": R * T * ws, "seq_len": None,
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (x 470 MB, recv_x 2.5 GB written); no flush"},
+        "config": workload_config(T, ws),
         "tokens_per_s": agg["tokens_per_s"],
         "pct_of_8TBps": 100.0 * agg["gbs"] / (SPEC_HBM_GBS * ws),
         "phases_ms": {"dispatch": disp_ms, "dispatch_notify_with_layout": notify_ms,
