@@ -199,6 +199,25 @@ def oracle_pass(sample: dict, w: Workload):
     return dt, nbytes, R * T
 
 
+def host_cpu() -> dict:
+    """The host's CPU model and core counts (the CPU baseline runs on one core)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    nproc = os.cpu_count()
+    try:
+        avail = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        avail = nproc
+    return {"cpu_model": model, "nproc": nproc, "cores_available": avail}
+
+
 def cpu_baseline(w: Workload, T_sample: int = 2048, reps: int = 3) -> dict:
     sample = sample_workload(w, T_sample)
     times = []
@@ -206,7 +225,9 @@ def cpu_baseline(w: Workload, T_sample: int = 2048, reps: int = 3) -> dict:
         dt, nbytes, ntok = oracle_pass(sample, w)
         times.append(dt)
     dt = statistics.median(times)
+    host = host_cpu()
     return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "cores_used": f"1 of {host['cores_available']} cores", **host,
             "sample": (f"first {T_sample} of {w.T} tokens of each of the {w.R} source ranks "
                        f"(same seeded workload), layout+prefix+dispatch+combine, median of "
                        f"{reps} single-threaded runs of the C oracle"),
@@ -241,13 +262,20 @@ def run_reference(args) -> None:
         tot_tok += nt
     dt = time.perf_counter() - t0
     value = tot_bytes / dt / 1e9
+    host = host_cpu()
+    config = workload_config(w.T, 1)
+    # the CPU arm times a sample of the workload; the rate is per byte and per
+    # token of that sample
+    config["sample"] = {"tokens_per_rank": T_sample, "of_tokens_per_rank": w.T,
+                        "source_ranks": w.R, "global_batch_timed": w.R * T_sample}
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": workload_config(w.T, 1),
+        "config": config,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "cores_used": f"1 of {host['cores_available']} cores", **host,
                          "sample": (f"each step runs the C oracle single-threaded on the first "
                                     f"{T_sample} of {w.T} tokens of each of the {w.R} source "
                                     "ranks (bytes and tokens counted for that sample)")},
@@ -428,6 +456,62 @@ def extra_configs(device, ep) -> dict:
     return out
 
 
+def routing_step(ep, io: dict, out: dict, wsp, status, R: int, T: int, E: int, stream=None,
+                 ev=None) -> None:
+    """One step of the timed path.
+
+    The layout (A1) is fused into the notify scan (A2): ep_notify_dispatch with
+    the layout outputs returns the layout, the handle and the received top-k
+    metadata from one kernel.  ep_dispatch_cached moves the rows (ep_dispatch
+    == ep_notify_dispatch + ep_dispatch_cached; the halves are called apart so
+    that the row copy gets its own events), and ep_combine reduces them back
+    with identity experts (y = recv_x).  io: inputs x, idx, wt and combined
+    outputs cx, cw; out: handle, layout and receive buffers; ev: five events
+    recorded around the phases, or None."""
+    if ev is not None:
+        ev[0].record(stream)
+        ev[1].record(stream)
+    ep.ep_notify_dispatch(io["idx"], io["wt"], T, R, E, with_layout=True, out=out,
+                          workspace=wsp, status=status, stream=stream)
+    if ev is not None:
+        ev[2].record(stream)
+    ep.ep_dispatch_cached(io["x"], out["send_pos"], recv_x=out["recv_x"], status=status,
+                          stream=stream)
+    if ev is not None:
+        ev[3].record(stream)
+    ep.ep_combine(out["recv_x"], out["send_pos"], out["recv_topk_weights"],
+                  combined_x=io["cx"], combined_topk_weights=io["cw"], status=status,
+                  stream=stream)
+    if ev is not None:
+        ev[4].record(stream)
+
+
+def step_buffers(R: int, T: int, H: int, E: int, K: int, device) -> tuple:
+    """Device buffers of routing_step: (out, cx, cw, workspace, status)."""
+    import torch
+
+    import combine_get_dispatch_06_b200 as ep
+
+    cap = R * T
+    out = {
+        "recv_x": torch.empty((R, cap, H), dtype=torch.bfloat16, device=device),
+        "recv_topk_idx": torch.empty((R, cap, K), dtype=torch.int64, device=device),
+        "recv_topk_weights": torch.empty((R, cap, K), dtype=torch.float32, device=device),
+        "recv_src_idx": torch.empty((R, cap), dtype=torch.int32, device=device),
+        "rank_prefix_matrix": torch.empty((R, R), dtype=torch.int32, device=device),
+        "recv_count": torch.empty((R,), dtype=torch.int32, device=device),
+        "num_recv_tokens_per_expert": torch.empty((R, E // R), dtype=torch.int32, device=device),
+        "send_pos": torch.empty((R, T, R), dtype=torch.int32, device=device),
+        "num_tokens_per_rank": torch.empty((R, R), dtype=torch.int32, device=device),
+        "num_tokens_per_expert": torch.empty((R, E), dtype=torch.int32, device=device),
+        "is_token_in_rank": torch.empty((R, T, R), dtype=torch.bool, device=device),
+    }
+    cx = torch.empty((R, T, H), dtype=torch.bfloat16, device=device)
+    cw = torch.empty((R, T, K), dtype=torch.float32, device=device)
+    wsp = torch.empty(ep.ep_dispatch_workspace_bytes(R, T, E), dtype=torch.uint8, device=device)
+    return out, cx, cw, wsp, ep.new_status(device)
+
+
 def run_ours(args) -> None:
     import torch
     import torch.distributed as dist
@@ -452,50 +536,12 @@ def run_ours(args) -> None:
     idx = idx_h.to(device)
     wt = w_h.to(device)
 
-    cap = R * T
-    out = {
-        "recv_x": torch.empty((R, cap, H), dtype=torch.bfloat16, device=device),
-        "recv_topk_idx": torch.empty((R, cap, K), dtype=torch.int64, device=device),
-        "recv_topk_weights": torch.empty((R, cap, K), dtype=torch.float32, device=device),
-        "recv_src_idx": torch.empty((R, cap), dtype=torch.int32, device=device),
-        "rank_prefix_matrix": torch.empty((R, R), dtype=torch.int32, device=device),
-        "recv_count": torch.empty((R,), dtype=torch.int32, device=device),
-        "num_recv_tokens_per_expert": torch.empty((R, E // R), dtype=torch.int32, device=device),
-        "send_pos": torch.empty((R, T, R), dtype=torch.int32, device=device),
-    }
-    ntpr = torch.empty((R, R), dtype=torch.int32, device=device)
-    ntpe = torch.empty((R, E), dtype=torch.int32, device=device)
-    inr = torch.empty((R, T, R), dtype=torch.bool, device=device)
-    cx = torch.empty((R, T, H), dtype=torch.bfloat16, device=device)
-    cw = torch.empty((R, T, K), dtype=torch.float32, device=device)
-    wsp = torch.empty(ep.ep_dispatch_workspace_bytes(R, T, E), dtype=torch.uint8, device=device)
-    status = ep.new_status(device)
-
-    out["num_tokens_per_rank"] = ntpr
-    out["num_tokens_per_expert"] = ntpe
-    out["is_token_in_rank"] = inr
+    out, cx, cw, wsp, status = step_buffers(R, T, H, E, K, device)
 
     io0 = {"x": x, "idx": idx, "wt": wt, "cx": cx, "cw": cw}
 
     def step(ev=None, io=io0):
-        # layout (A1) is fused into the notify scan (A2): one kernel returns the
-        # layout and the handle.  ep_dispatch == ep_notify_dispatch +
-        # ep_dispatch_cached; the two halves are called separately so that the
-        # row-copy kernel gets its own events.
-        if ev is not None:
-            ev[0].record(stream)
-            ev[1].record(stream)
-        ep.ep_notify_dispatch(io["idx"], io["wt"], T, R, E, with_layout=True, out=out,
-                              workspace=wsp, status=status)
-        if ev is not None:
-            ev[2].record(stream)
-        ep.ep_dispatch_cached(io["x"], out["send_pos"], recv_x=out["recv_x"], status=status)
-        if ev is not None:
-            ev[3].record(stream)
-        ep.ep_combine(out["recv_x"], out["send_pos"], out["recv_topk_weights"],
-                      combined_x=io["cx"], combined_topk_weights=io["cw"], status=status)
-        if ev is not None:
-            ev[4].record(stream)
+        routing_step(ep, io, out, wsp, status, R, T, E, stream, ev)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -631,6 +677,112 @@ def run_ours(args) -> None:
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------------------
+# profiling cases: one entry point of the path, looped, on a named workload
+# ---------------------------------------------------------------------------
+
+# Sized for ncu captures: the "_small" and "_scan" cases hold at most ~2 GB on
+# the device (inputs still larger than L2 where the kernel streams rows); the
+# full-size cases are for the single-pass launch list only.
+PROFILE_CASES = {
+    "notify_normal": (Workload("normal_routing", R=8, T=4096, H=0, E=256, K=8), "notify"),
+    "notify_skewed": (Workload("skewed_routing", R=16, T=2048, H=0, E=128, K=6, routing="zipf",
+                               zipf_s=1.2, masked_frac=0.1), "notify"),
+    "layout": (CONFIGS["layout"], "layout"),
+    "copy_normal_small": (Workload("normal_small", R=8, T=1536, H=7168, E=256, K=8), "copy"),
+    "combine_normal_small": (Workload("normal_small", R=8, T=1536, H=7168, E=256, K=8),
+                             "combine"),
+    "step_skewed_small": (Workload("skewed_small", R=16, T=1024, H=4096, E=128, K=6,
+                                   routing="zipf", zipf_s=1.2, masked_frac=0.1), "step"),
+    "step_skewed": (CONFIGS["skewed"], "step"),
+    "ll_dispatch_small": (Workload("ll_small", R=8, T=512, H=7168, E=64, K=8), "ll_dispatch"),
+    "ll_scan": (Workload("ll_routing", R=32, T=128, H=128, E=256, K=8), "ll_dispatch"),
+    "ll_dispatch": (CONFIGS["ll"], "ll_dispatch"),
+    "ll_combine_small": (Workload("ll_small", R=8, T=256, H=7168, E=64, K=8), "ll_combine"),
+}
+
+
+def run_profile(args) -> None:
+    """Loop one entry point on a PROFILE_CASES workload (warm-up, then
+    --steps calls) and print its mean time per call as one JSON line."""
+    import dataclasses
+
+    import torch
+
+    import combine_get_dispatch_06_b200 as ep
+
+    w, what = PROFILE_CASES[args.profile]
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    inp = make(w)
+    R, T, H, E, K = w.R, w.T, w.H, w.E, w.K
+    idx = torch.from_numpy(inp["topk_idx"]).to(device)
+    wt = torch.from_numpy(inp["topk_weights"]).to(device)
+    x = to_dev_bf16(inp["x"], device) if "x" in inp else None
+    status = ep.new_status(device)
+    stream = torch.cuda.current_stream(device)
+    if what == "layout":
+        idx1 = idx[0]
+        o = ep.ep_get_dispatch_layout(idx1, E, R, status=status)
+
+        def call():
+            ep.ep_get_dispatch_layout(idx1, E, R, num_tokens_per_rank=o[0],
+                                      num_tokens_per_expert=o[1], is_token_in_rank=o[2],
+                                      status=status)
+    elif what in ("notify", "copy", "combine", "step"):
+        out, cx, cw, wsp, _ = step_buffers(R, T, max(H, 8), E, K, device)
+        ep.ep_notify_dispatch(idx, wt, T, R, E, with_layout=True, out=out, workspace=wsp,
+                              status=status)
+        if x is not None:
+            ep.ep_dispatch_cached(x, out["send_pos"], recv_x=out["recv_x"], status=status)
+        io = {"x": x, "idx": idx, "wt": wt, "cx": cx, "cw": cw}
+
+        def call():
+            if what == "notify":
+                ep.ep_notify_dispatch(idx, wt, T, R, E, with_layout=True, out=out,
+                                      workspace=wsp, status=status)
+            elif what == "copy":
+                ep.ep_dispatch_cached(x, out["send_pos"], recv_x=out["recv_x"], status=status)
+            elif what == "combine":
+                ep.ep_combine(out["recv_x"], out["send_pos"], out["recv_topk_weights"],
+                              combined_x=cx, combined_topk_weights=cw, status=status)
+            else:
+                routing_step(ep, io, out, wsp, status, R, T, E, stream)
+    elif what in ("ll_dispatch", "ll_combine"):
+        ws = torch.empty(ep.ep_ll_workspace_bytes(R, T, E), dtype=torch.uint8, device=device)
+        d = ep.ep_ll_dispatch(x, idx, E, use_fp8=True, workspace=ws, status=status)
+        if what == "ll_combine":
+            del d["recv_x"], d["recv_scales"]
+            g = torch.Generator(device=device).manual_seed(1)
+            y = torch.randn((R, E // R, R * T, H), generator=g, device=device,
+                            dtype=torch.bfloat16)
+            out_c = torch.empty((R, T, H), dtype=torch.bfloat16, device=device)
+
+            def call():
+                ep.ep_ll_combine(y, idx, wt, d["ll_pos"], out=out_c, status=status)
+        else:
+            def call():
+                ep.ep_ll_dispatch(x, idx, E, use_fp8=True, out=d, workspace=ws, status=status)
+    else:
+        raise ValueError(what)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(device)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())}")
+    print(json.dumps({"profile": args.profile, "entry": what,
+                      "us_per_call": a.elapsed_time(b) / args.steps * 1e3,
+                      "steps": args.steps, "warmup": args.warmup,
+                      "workload": dataclasses.asdict(w)}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -641,10 +793,14 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per source rank (default 4096; smaller only for profiling)")
+    ap.add_argument("--profile", choices=sorted(PROFILE_CASES), default=None,
+                    help="loop one entry point on a named small workload (for ncu captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile is not None:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

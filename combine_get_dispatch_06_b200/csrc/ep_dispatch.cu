@@ -604,7 +604,8 @@ extern "C" EP_API size_t ep_dispatch_workspace_bytes(int num_ranks, int num_toke
   if (num_ranks < 1 || num_tokens < 0 || num_experts < 0) return 0;
   const long tiles = static_cast<long>(num_ranks) * ((num_tokens + kScanTile - 1) / kScanTile);
   // expert counters: all sources [E], then per source [R][E] (fused layout)
-  return scan_workspace_bytes(tiles, num_ranks, num_experts * (1 + num_ranks));
+  return scan_workspace_bytes(tiles, num_ranks,
+                              static_cast<long>(num_experts) * (1L + num_ranks));
 }
 
 namespace ep {
@@ -799,13 +800,13 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
   return launch_status(launched);
 }
 
-// Checks shared by ep_dispatch and ep_notify_dispatch.
-int check_notify_args(const int64_t *topk_idx, const float *topk_weights,
-                      const uint8_t *is_token_in_rank, int R, int T, int K, int E, int align,
-                      int cap, const int64_t *recv_topk_idx, const float *recv_topk_weights,
-                      const int32_t *recv_src_idx, const int32_t *rank_prefix_matrix,
-                      const int32_t *recv_count, const int32_t *nrte, const int32_t *send_pos,
-                      const void *workspace, size_t workspace_bytes) {
+// Checks shared by ep_dispatch, ep_notify_dispatch and ep_dispatch_noalloc,
+// except the workspace (check_workspace).
+int check_notify_shape(const int64_t *topk_idx, const float *topk_weights,
+                       const uint8_t *is_token_in_rank, int R, int T, int K, int E, int align,
+                       int cap, const int64_t *recv_topk_idx, const float *recv_topk_weights,
+                       const int32_t *recv_src_idx, const int32_t *rank_prefix_matrix,
+                       const int32_t *recv_count, const int32_t *nrte, const int32_t *send_pos) {
   if (R < 1 || R > kMaxRanks || T < 0 || cap < 0 || align < 1) return EP_ERR_INVALID_ARG;
   if (rank_prefix_matrix == nullptr || recv_count == nullptr) return EP_ERR_INVALID_ARG;
   const bool meta = recv_topk_idx != nullptr || recv_topk_weights != nullptr || nrte != nullptr;
@@ -821,11 +822,31 @@ int check_notify_args(const int64_t *topk_idx, const float *topk_weights,
   if (static_cast<long>(R) * ((T + kScanTile - 1) / kScanTile) > 0x7fffffffL ||
       static_cast<long>(R) * T > 0x7fffffffL)
     return EP_ERR_UNSUPPORTED;
+  return EP_OK;
+}
+
+// The caller's workspace of a call that passed check_notify_shape.
+int check_workspace(const int64_t *topk_idx, int R, int T, int E, const void *workspace,
+                    size_t workspace_bytes) {
+  if (T == 0) return EP_OK;
   const size_t need = ep_dispatch_workspace_bytes(R, T, topk_idx != nullptr ? E : 0);
   if (workspace == nullptr || workspace_bytes < need ||
       (reinterpret_cast<uintptr_t>(workspace) & 15u))
     return EP_ERR_INVALID_ARG;
   return EP_OK;
+}
+
+int check_notify_args(const int64_t *topk_idx, const float *topk_weights,
+                      const uint8_t *is_token_in_rank, int R, int T, int K, int E, int align,
+                      int cap, const int64_t *recv_topk_idx, const float *recv_topk_weights,
+                      const int32_t *recv_src_idx, const int32_t *rank_prefix_matrix,
+                      const int32_t *recv_count, const int32_t *nrte, const int32_t *send_pos,
+                      const void *workspace, size_t workspace_bytes) {
+  const int rc = check_notify_shape(topk_idx, topk_weights, is_token_in_rank, R, T, K, E, align,
+                                    cap, recv_topk_idx, recv_topk_weights, recv_src_idx,
+                                    rank_prefix_matrix, recv_count, nrte, send_pos);
+  if (rc != EP_OK) return rc;
+  return check_workspace(topk_idx, R, T, E, workspace, workspace_bytes);
 }
 
 int check_copy_args(const void *x, const int32_t *send_pos, int R, int T, int H, int cap,
@@ -946,12 +967,17 @@ extern "C" EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
 // kNoAllocScratchBytes, which every GPU that loads this library holds until
 // the process exits.  It allocates nothing and calls nothing that allocates.
 //
-// Set-up: the first call on a device (with that device current) looks up the
-// array's device address with cudaGetSymbolAddress and caches it; make that
-// first call before any stream capture.  The array is shared by every call on
-// a device and keeps the last call's contents; ep_dispatch clears the part it
-// uses on the stream before its kernels run, so calls on one stream are safe,
-// but calls that overlap on the GPU (other streams, other threads) race on it.
+// The array's name is only a host-side stand-in in host code; the kernels get
+// its device address, looked up with cudaGetSymbolAddress with the device
+// current.  The first call on a device does that set-up (make it before any
+// stream capture).  Later calls made outside stream capture look the address
+// up again, so a device reset (after which the module, and the array, may
+// load elsewhere) is harmless; a call made while its stream is capturing uses
+// the address of the last call outside capture.  The array is shared by every
+// call on a device and keeps the last call's contents; ep_dispatch clears the
+// part it uses on the stream before its kernels run, so calls on one stream
+// are safe, but calls that overlap on the GPU (other streams, other threads)
+// race on it.
 // ---------------------------------------------------------------------------
 
 namespace ep {
@@ -965,14 +991,19 @@ void *g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
 std::mutex g_noalloc_mu;
 
 // Device address of the scratch array on the current device, or nullptr.
-void *noalloc_scratch() {
+void *noalloc_scratch(cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  const bool capturing =
+      cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  if (!capturing || g_noalloc_ptr[dev] == nullptr) {
     void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      g_noalloc_ptr[dev] = nullptr;
       return nullptr;
+    }
     g_noalloc_ptr[dev] = p;
   }
   return g_noalloc_ptr[dev];
@@ -989,15 +1020,25 @@ extern "C" EP_API int ep_dispatch_noalloc(
     int32_t *recv_count, int32_t *num_recv_tokens_per_expert, int32_t *send_pos,
     int32_t *status, cudaStream_t stream) {
   using namespace ep;
-  if (num_ranks < 1 || num_tokens < 0 || num_experts < 0) return EP_ERR_INVALID_ARG;
+  // ep_dispatch's argument checks first: an invalid call is reported as
+  // invalid whatever its size
+  int rc = check_notify_shape(topk_idx, topk_weights, is_token_in_rank, num_ranks, num_tokens,
+                              num_topk, num_experts, expert_alignment, capacity, recv_topk_idx,
+                              recv_topk_weights, recv_src_idx, rank_prefix_matrix, recv_count,
+                              num_recv_tokens_per_expert, send_pos);
+  if (rc != EP_OK) return rc;
+  rc = check_copy_args(x, send_pos, num_ranks, num_tokens, hidden, capacity, recv_x);
+  if (rc != EP_OK) return rc;
   const size_t need =
       ep_dispatch_workspace_bytes(num_ranks, num_tokens, topk_idx != nullptr ? num_experts : 0);
   if (need > kNoAllocScratchBytes) return EP_ERR_UNSUPPORTED;  // beyond the static scratch
-  void *scratch = noalloc_scratch();
+  void *scratch = noalloc_scratch(stream);
   if (scratch == nullptr) return EP_ERR_CUDA;
-  return ep_dispatch(x, topk_idx, topk_weights, is_token_in_rank, num_ranks, num_tokens, hidden,
-                     num_topk, num_experts, expert_alignment, capacity, recv_x, recv_topk_idx,
-                     recv_topk_weights, recv_src_idx, rank_prefix_matrix, recv_count,
-                     num_recv_tokens_per_expert, send_pos, scratch, kNoAllocScratchBytes,
-                     status, stream);
+  rc = notify_impl(topk_idx, topk_weights, is_token_in_rank, num_ranks, num_tokens, num_topk,
+                   num_experts, expert_alignment, capacity, recv_topk_idx, recv_topk_weights,
+                   recv_src_idx, rank_prefix_matrix, recv_count, num_recv_tokens_per_expert,
+                   send_pos, nullptr, nullptr, nullptr, scratch, status, stream);
+  if (rc != EP_OK) return rc;
+  return copy_impl(x, nullptr, 0, 0, send_pos, num_ranks, num_tokens, hidden * 2, capacity,
+                   recv_x, nullptr, status, stream);
 }

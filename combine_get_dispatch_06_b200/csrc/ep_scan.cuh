@@ -29,7 +29,7 @@ struct ScanHeader {
 // Workspace: header, then `counters` int32 (rounded to 4), then the
 // descriptors [num_tiles][columns] uint64.
 __host__ __device__ inline size_t scan_workspace_bytes(long num_tiles, int columns,
-                                                       int counters) {
+                                                       long counters) {
   const size_t head = sizeof(ScanHeader) + static_cast<size_t>((counters + 3) & ~3) * 4;
   const size_t bytes = head + static_cast<size_t>(num_tiles) * columns * sizeof(uint64_t);
   return (bytes + 255) & ~static_cast<size_t>(255);

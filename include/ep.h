@@ -253,16 +253,21 @@ EP_API int ep_dispatch_cached_fp8(const void *x_e4m3, const float *x_scales,
  * another allocator, or a latency-critical loop that cannot afford
  * cudaMalloc/cudaFree (they can synchronise the device).
  *
- * Arguments, outputs and results are those of ep_dispatch.  The scratch lives
- * in a 2 MiB static device array inside the library, held on every GPU that
- * loads the library until the process exits; this call allocates nothing.
- * Calls needing more than that (ep_dispatch_workspace_bytes(R, T, E) >
- * 2 MiB, with E = 0 when topk_idx is NULL) return EP_ERR_UNSUPPORTED.
+ * Arguments, outputs and results are those of ep_dispatch; its argument
+ * checks come first (an invalid call returns EP_ERR_INVALID_ARG whatever its
+ * size).  The scratch lives in a 2 MiB static device array inside the
+ * library, held on every GPU that loads the library until the process exits;
+ * this call allocates nothing.  Calls needing more than that
+ * (ep_dispatch_workspace_bytes(R, T, E) > 2 MiB, with E = 0 when topk_idx is
+ * NULL) return EP_ERR_UNSUPPORTED.
  * The first call on a device, with that device current, looks up the array's
  * device address (cudaGetSymbolAddress); make that first call before any
- * stream capture.  Every call on a device shares the array and it keeps the
- * last call's contents (the call clears what it uses on `stream` first): calls
- * that overlap on the GPU, e.g. on two streams at once, race on it.
+ * stream capture.  Later calls outside stream capture look it up again (so a
+ * device reset, after which the array may sit elsewhere, does no harm); a call
+ * whose stream is capturing uses the address of the last call outside capture.
+ * Every call on a device shares the array and it keeps the last call's
+ * contents (the call clears what it uses on `stream` first): calls that
+ * overlap on the GPU, e.g. on two streams at once, race on it.
  */
 EP_API int ep_dispatch_noalloc(const void *x, const int64_t *topk_idx,
                                const float *topk_weights,
