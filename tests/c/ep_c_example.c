@@ -1,8 +1,9 @@
 /*
  * A plain C caller of libep: the hand-worked 2-rank, 3-token routing example
  * (tests/golden/routing_tiny.json) through ep_get_dispatch_layout,
- * ep_dispatch and ep_combine, with device buffers from cudaMalloc and the
- * default stream.  The example's rows have 2 channels; the library moves rows
+ * ep_dispatch and ep_combine, then through the low-latency pair
+ * ep_ll_dispatch (bf16 payload) and ep_ll_combine with identity experts, with
+ * device buffers from cudaMalloc and the default stream.  The example's rows have 2 channels; the library moves rows
  * of a multiple of 8 channels (16 bytes), so each row is zero-padded to 8
  * channels and only the example's 2 are printed.  Prints every output as
  * "name v0 v1 ..." lines for the test to compare with the fixture.
@@ -22,6 +23,7 @@
 #define HX 2 /* the example's channels */
 #define H 8  /* channels per row as stored (zero-padded) */
 #define CAP (R * T)
+#define EL (E / R)
 
 #define CK(x)                                                                  \
   do {                                                                         \
@@ -150,6 +152,58 @@ int main(void) {
     }
   printf("\ncombined_topk_weights");
   for (int i = 0; i < R * T * K; ++i) printf(" %.9g", cw_h[i]);
+  printf("\n");
+
+  /* low latency: bf16 slabs [R, E_l, R*T, H], then the weighted combine of
+     the slab rows as they are (identity experts) */
+  void *slab, *lout, *lws;
+  int *lrc, *lrsi, *llr, *lpos;
+  const size_t lwsb = ep_ll_workspace_bytes(R, T, E);
+  CK(cudaMalloc(&slab, (size_t)R * EL * CAP * H * 2));
+  CK(cudaMalloc(&lout, R * T * H * 2));
+  CK(cudaMalloc(&lws, lwsb));
+  CK(cudaMalloc((void **)&lrc, R * EL * 4));
+  CK(cudaMalloc((void **)&lrsi, R * EL * CAP * 4));
+  CK(cudaMalloc((void **)&llr, R * EL * R * 2 * 4));
+  CK(cudaMalloc((void **)&lpos, R * T * K * 4));
+  EK(ep_ll_dispatch(x, idx, NULL, R, T, H, K, E, 0, slab, NULL, lrc, lrsi, llr, lpos, NULL, lws,
+                    lwsb, st, 0));
+  EK(ep_ll_combine(slab, idx, w, lpos, NULL, R, T, H, K, E, lout, st, 0));
+  CK(cudaDeviceSynchronize());
+  int lrc_h[R * EL], lrsi_h[R * EL * CAP], llr_h[R * EL * R * 2], lpos_h[R * T * K];
+  unsigned short slab_h[R * EL * CAP * H], lout_h[R * T * H];
+  CK(cudaMemcpy(lrc_h, lrc, sizeof lrc_h, cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(lrsi_h, lrsi, sizeof lrsi_h, cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(llr_h, llr, sizeof llr_h, cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(lpos_h, lpos, sizeof lpos_h, cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(slab_h, slab, sizeof slab_h, cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(lout_h, lout, sizeof lout_h, cudaMemcpyDeviceToHost));
+  CK(cudaMemcpy(&st_h, st, 4, cudaMemcpyDeviceToHost));
+  print_i32("ll_status", &st_h, 1);
+  print_i32("ll_recv_count", lrc_h, R * EL);
+  print_i32("ll_layout_range", llr_h, R * EL * R * 2);
+  print_i32("ll_pos", lpos_h, R * T * K);
+  for (int e = 0; e < R * EL; ++e) {
+    printf("ll_recv_src_info_%d_%d", e / EL, e % EL);
+    for (int r = 0; r < lrc_h[e]; ++r) printf(" %d", lrsi_h[e * CAP + r]);
+    printf("\nll_slab_%d_%d", e / EL, e % EL);
+    for (int r = 0; r < lrc_h[e]; ++r)
+      for (int c = 0; c < HX; ++c) {
+        unsigned int u = (unsigned int)slab_h[(e * CAP + r) * H + c] << 16;
+        float f;
+        memcpy(&f, &u, 4);
+        printf(" %.9g", f);
+      }
+    printf("\n");
+  }
+  printf("ll_combined_x");
+  for (int t = 0; t < R * T; ++t)
+    for (int c = 0; c < HX; ++c) {
+      unsigned int u = (unsigned int)lout_h[t * H + c] << 16;
+      float f;
+      memcpy(&f, &u, 4);
+      printf(" %.9g", f);
+    }
   printf("\n");
   return 0;
 }

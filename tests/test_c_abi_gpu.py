@@ -1,6 +1,7 @@
 """The C ABI from C: tests/c/ep_c_example.c, compiled against include/ep.h and
 libep.so, runs the hand-worked golden example through layout, dispatch and
-combine; its printed outputs must equal the fixture."""
+combine, and through low-latency dispatch (bf16 slabs) and the weighted
+low-latency combine; its printed outputs must equal the fixture."""
 import json
 import os
 import subprocess
@@ -42,3 +43,23 @@ def test_c_caller_reproduces_the_golden_example(tmp_path):
         assert got[f"recv_src_idx_{d}"] == flat(g["recv_src_idx"][d])
         assert got[f"recv_topk_idx_{d}"] == flat(g["recv_topk_idx"][d])
         assert got[f"recv_topk_weights_{d}"] == flat(g["recv_topk_weights"][d])
+    # low latency (legacy-test analysis page: the low_latency_dispatch call,
+    # its handle (recv_src_info, recv_layout_range) and per-expert counts, and
+    # the low_latency_combine check against x times the masked weight sum)
+    assert got["ll_status"] == [0.0]
+    assert got["ll_recv_count"] == flat(g["ll_recv_count"])
+    assert got["ll_layout_range"] == flat(g["ll_layout_range"])
+    assert got["ll_pos"] == flat(g["ll_pos"])
+    assert got["ll_combined_x"] == flat(g["ll_combined_x"])
+    R, El, T = g["R"], g["E"] // g["R"], g["T"]
+    x = np.array(g["x"], np.float64)
+    for d in range(R):
+        for j in range(El):
+            assert got[f"ll_recv_src_info_{d}_{j}"] == flat(g["ll_recv_src_info"][d][j])
+            # slab rows: the rows of their source tokens, source rank by source rank
+            rows = []
+            for s in range(R):
+                begin, n = g["ll_layout_range"][d][j][s]
+                for r in range(begin, begin + n):
+                    rows.append(x[s, g["ll_recv_src_info"][d][j][r]])
+            assert got[f"ll_slab_{d}_{j}"] == flat(rows), (d, j)

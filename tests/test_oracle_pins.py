@@ -79,6 +79,10 @@ def test_golden_tiny_low_latency():
         for j in range(g["E"] // g["R"]):
             n = g["ll_recv_count"][d][j]
             np.testing.assert_array_equal(ll["recv_src_info"][d, j, :n], g["ll_recv_src_info"][d][j])
+    # identity experts: the bf16 slab rows go back unchanged
+    slab, _ = oracle.ll_dispatch_rows(f2b(g["x"]), idx, ll["ll_pos"], g["E"], use_fp8=False)
+    out = oracle.ll_combine(slab, idx, np.array(g["topk_weights"], np.float32), ll["ll_pos"])
+    np.testing.assert_array_equal(b2f(out), np.array(g["ll_combined_x"], np.float32))
 
 
 def test_golden_fp8_and_bf16_codes():

@@ -115,9 +115,9 @@ def test_noalloc_routing_from_is_token_in_rank_only():
 def test_noalloc_near_the_limit_runs_and_past_it_is_refused():
     import combine_get_dispatch_06_b200 as ep
 
-    # 384 ranks, one scan tile per source, 384 experts: 88% of the array
+    # 384 ranks, one scan tile per source, 384 experts: 84% of the array
     near = Workload("near", R=384, T=128, H=8, E=384, K=4, seed=36)
-    assert 0.85 * SCRATCH_BYTES < ep.ep_dispatch_workspace_bytes(384, 128, 384) <= SCRATCH_BYTES
+    assert 0.8 * SCRATCH_BYTES < ep.ep_dispatch_workspace_bytes(384, 128, 384) <= SCRATCH_BYTES
     _run_pair(ep, near, align=1)
     # one token more per source: two tiles per source, past the array
     over = Workload("over", R=384, T=129, H=8, E=384, K=4, seed=37)
