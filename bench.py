@@ -678,6 +678,142 @@ def run_ours(args) -> None:
 
 
 # ---------------------------------------------------------------------------
+# one rank per GPU (--mode sharded)
+# ---------------------------------------------------------------------------
+
+def shard_bytes(R, T, H, K, N):
+    """Algorithmic bytes of one rank's dispatch + combine: its T rows read
+    once, its N copies written, its ids and weights read, per-copy metadata
+    written, its layout / positions; combine reads the N rows back, writes T
+    rows, weights and positions."""
+    disp = T * H * 2 + N * H * 2 + T * K * 12 + N * (K * 12 + 4) + T * K * 8 + 2 * T * R + T * R * 4
+    comb = N * H * 2 + T * H * 2 + N * K * 4 + T * K * 4 + T * R * 4
+    return disp, comb
+
+
+def run_sharded(args) -> None:
+    """The normal workload with one rank per GPU: rank r holds its own T
+    tokens, writes their rows into the destination GPUs' receive buffers
+    through peer pointers (CUDA IPC over NVLink) and gathers them back at
+    combine; the notify counts travel by an NCCL all-gather and the phases
+    are ordered by stream-ordered NCCL all-reduces (no host round trip).
+    R = number of GPUs, 32 experts per rank unless 256 divides evenly."""
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29533")
+    dist.init_process_group("nccl", rank=rank, world_size=ws,
+                            timeout=datetime.timedelta(seconds=120))
+    from combine_get_dispatch_06_b200.shard import ShardedBuffer  # fails loudly without libep.so
+
+    w0 = CONFIGS["normal"]
+    R, T, H, K = ws, (args.tokens or w0.T), w0.H, w0.K
+    E = w0.E if w0.E % R == 0 else 32 * R
+    w = Workload("normal_sharded", R=R, T=T, H=H, E=E, K=K, seed=w0.seed)
+    inp = make(w, ranks=[rank])
+    x = to_dev_bf16(inp["x"][0], device)
+    idx = torch.from_numpy(inp["topk_idx"][0]).to(device)
+    wt = torch.from_numpy(inp["topk_weights"][0]).to(device)
+    cx = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+    cw = torch.empty((T, K), dtype=torch.float32, device=device)
+    buf = ShardedBuffer(dist.group.WORLD, T, H, K, E, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        buf.dispatch(x, idx, wt)
+        buf.combine(combined_x=cx, combined_topk_weights=cw)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    if int(buf.status.item()) != 0:
+        raise RuntimeError(f"device status {int(buf.status.item())} during warm-up")
+    sp = buf.send_pos
+    N = int((sp >= 0).sum().item())
+    remote = torch.ones(R, dtype=torch.bool, device=device)
+    remote[rank] = False
+    N_remote = int(((sp >= 0) & remote[None, :]).sum().item())
+    bd, bc = shard_bytes(R, T, H, K, N)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clocks = sampler.stop()
+    ms_local = a.elapsed_time(b) / args.steps
+    agg = aggregate(bd + bc, T, ms_local, device)
+    if int(buf.status.item()) != 0:
+        raise RuntimeError(f"device status {int(buf.status.item())} in the timed region")
+    # rows crossing NVLink per step (each way): copies to other ranks, then read back
+    link = reduce_max(N_remote * H * 2 * 2, device)
+
+    # end to end: this step's inputs up from pinned host memory, its result down
+    x_h = torch.from_numpy(inp["x"][0].view(np.int16)).view(torch.bfloat16).pin_memory()
+    idx_h = torch.from_numpy(inp["topk_idx"][0]).pin_memory()
+    w_h = torch.from_numpy(inp["topk_weights"][0]).pin_memory()
+    cx_h = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    barrier(device)
+    torch.cuda.synchronize(device)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(x_h, non_blocking=True)
+        idx.copy_(idx_h, non_blocking=True)
+        wt.copy_(w_h, non_blocking=True)
+        step()
+        cx_h.copy_(cx, non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e2e = aggregate(bd + bc, T, a.elapsed_time(b) / e2e_steps, device)
+    h2d = x_h.numel() * 2 + idx_h.numel() * 8 + w_h.numel() * 4
+    probe = buf.notify_probe.cpu().numpy().astype(np.uint64)
+    starts = [None] * ws
+    dist.all_gather_object(starts, int(probe[2]))
+
+    line = {
+        "metric": METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": agg["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "mode": "sharded",
+        "config": {"workload": f"normal, one rank per GPU: R={R} ranks x T={T} tokens x H={H} "
+                               f"bf16, E={E} experts, top-{K} distinct uniform, fp32 softmax "
+                               "weights, identity experts",
+                   "global_batch": R * T, "seq_len": None,
+                   "parallelism": f"ep{R} (one rank per GPU, peer stores over NVLink)",
+                   "l2": "inputs larger than L2; no flush"},
+        "tokens_per_s": agg["tokens_per_s"],
+        "pct_of_8TBps": 100.0 * agg["gbs"] / (SPEC_HBM_GBS * ws),
+        "nvlink_bytes_per_step_per_gpu": link,
+        "nvlink_gbs_per_gpu": link / (agg["ms_per_step"] * 1e-3) / 1e9,
+        "notify_probe": {"launches": int(probe[1]),
+                         "mean_full_grid_us": float(probe[0]) / max(int(probe[1]), 1) / 1e3,
+                         "arrival_skew_us": (max(starts) - min(starts)) / 1e3},
+        "e2e": {"value": e2e["gbs"], "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": cx_h.numel() * 2, "ms_per_step": e2e["ms_per_step"]},
+        "gpu_launches": 6 * args.steps,   # layout, prefix, scan, pad, copy, combine per step
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    buf.close()
+    dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
 # profiling cases: one entry point of the path, looped, on a named workload
 # ---------------------------------------------------------------------------
 
@@ -793,6 +929,9 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per source rank (default 4096; smaller only for profiling)")
+    ap.add_argument("--mode", choices=["replicas", "sharded"], default="replicas",
+                    help="N > 1: independent single-GPU replicas (default), or one routing "
+                         "rank per GPU over NVLink")
     ap.add_argument("--profile", choices=sorted(PROFILE_CASES), default=None,
                     help="loop one entry point on a named small workload (for ncu captures)")
     args = ap.parse_args(argv)
@@ -802,6 +941,8 @@ def main(argv=None):
         run_profile(args)
     elif args.impl == "reference":
         run_reference(args)
+    elif args.mode == "sharded":
+        run_sharded(args)
     else:
         run_ours(args)
 

@@ -53,6 +53,16 @@ _SIGS = {
     "ep_ll_dispatch": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P,
                             _P, _P, _Z, _P, _P]),
     "ep_ll_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "ep_shard_alloc": (_I, [_Z, ctypes.POINTER(ctypes.c_void_p)]),
+    "ep_shard_free": (_I, [_P]),
+    "ep_ipc_handle": (_I, [_P, _P]),
+    "ep_ipc_open": (_I, [_P, ctypes.POINTER(ctypes.c_void_p)]),
+    "ep_ipc_close": (_I, [_P]),
+    "ep_shard_workspace_bytes": (_Z, [_I, _I]),
+    "ep_shard_notify": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                             _P, _P, _P, _P, _P, _Z, _P, _P]),
+    "ep_shard_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
+    "ep_shard_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)

@@ -2,6 +2,7 @@
 // process-wide limits of the bounded device waits, device properties.
 #include <algorithm>
 #include <atomic>
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <tuple>
@@ -132,6 +133,52 @@ EP_API int ep_set_wait_timeout_ns(long long ns) {
 EP_API int ep_set_debug_flags(unsigned flags) {
   ep::g_flags.store(flags, std::memory_order_relaxed);
   return EP_OK;
+}
+
+// ---- memory shared between the ranks of a sharded job ----------------------
+
+EP_API int ep_shard_alloc(size_t bytes, void **ptr) {
+  if (ptr == nullptr || bytes == 0) return EP_ERR_INVALID_ARG;
+  *ptr = nullptr;
+  void *p = nullptr;
+  if (cudaMalloc(&p, bytes) != cudaSuccess) return EP_ERR_CUDA;
+  if (cudaMemset(p, 0, bytes) != cudaSuccess) {
+    cudaFree(p);
+    return EP_ERR_CUDA;
+  }
+  *ptr = p;
+  return EP_OK;
+}
+
+EP_API int ep_shard_free(void *ptr) {
+  if (ptr == nullptr) return EP_OK;
+  return cudaFree(ptr) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+EP_API int ep_ipc_handle(const void *ptr, void *handle) {
+  static_assert(sizeof(cudaIpcMemHandle_t) == EP_IPC_HANDLE_BYTES, "IPC handle size");
+  if (ptr == nullptr || handle == nullptr) return EP_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, const_cast<void *>(ptr)) != cudaSuccess) return EP_ERR_CUDA;
+  memcpy(handle, &h, sizeof h);
+  return EP_OK;
+}
+
+EP_API int ep_ipc_open(const void *handle, void **ptr) {
+  if (handle == nullptr || ptr == nullptr) return EP_ERR_INVALID_ARG;
+  *ptr = nullptr;
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle, sizeof h);
+  void *p = nullptr;
+  if (cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess)
+    return EP_ERR_CUDA;
+  *ptr = p;
+  return EP_OK;
+}
+
+EP_API int ep_ipc_close(void *ptr) {
+  if (ptr == nullptr) return EP_OK;
+  return cudaIpcCloseMemHandle(ptr) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -42,17 +42,24 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float (&a)[8]) {
   return r;
 }
 
+// kTab: the destinations' buffers are given by tables of R pointers (one
+// rank of a sharded job: peers' memory, read with plain loads); else they
+// are slices d * cap of y and recv_w.
+template <bool kTab>
 __global__ void __launch_bounds__(kCombineWarps * 32)
     combine_kernel(const uint8_t *__restrict__ y, const float *__restrict__ recv_w,
+                   const uint8_t *const *y_tab, const float *const *w_tab,
                    const int32_t *__restrict__ send_pos, const uint8_t *__restrict__ bias0,
                    const uint8_t *__restrict__ bias1, int R, long num_tok, int H, int K,
-                   int cap, uint8_t *__restrict__ out, float *__restrict__ out_w,
+                   int cap, bool want_w, uint8_t *__restrict__ out, float *__restrict__ out_w,
                    int32_t *status) {
   pdl_wait();
-  extern __shared__ __align__(16) int64_t s_rows[];  // [warps][R] row indices d*cap + pos
+  // per warp: [R] row pointers of y, then [R] row pointers of recv_w
+  extern __shared__ __align__(16) const uint8_t *s_ptr[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  int64_t *rows = s_rows + static_cast<size_t>(warp) * R;
+  const uint8_t **rows = s_ptr + static_cast<size_t>(warp) * 2 * R;
+  const float **wrows = reinterpret_cast<const float **>(rows + R);
   const uint32_t lt = lanemask_lt();
   const int nvec = H >> 3;
   const long row_bytes = static_cast<long>(H) * 2;
@@ -68,7 +75,17 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
       bad |= (pos < -1 || pos >= cap);
       const bool take = pos >= 0 && pos < cap;
       const uint32_t bal = __ballot_sync(0xffffffffu, take);
-      if (take) rows[n + __popc(bal & lt)] = static_cast<int64_t>(d) * cap + pos;
+      if (take) {
+        const int i = n + __popc(bal & lt);
+        if (kTab) {
+          rows[i] = y_tab[d] + static_cast<long>(pos) * row_bytes;
+          if (want_w) wrows[i] = w_tab[d] + static_cast<long>(pos) * K;
+        } else {
+          const long row = static_cast<long>(d) * cap + pos;
+          rows[i] = y + row * row_bytes;
+          if (want_w) wrows[i] = recv_w + row * K;
+        }
+      }
       n += __popc(bal);
     }
     if (bad) report(status, EP_STATUS_BAD_POSITION);
@@ -84,7 +101,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
 #pragma unroll
         for (int b = 0; b < kCombineBatch; ++b) {
           if (i + b < n) {
-            const uint8_t *r = y + rows[i + b] * row_bytes;
+            const uint8_t *r = rows[i + b];
             v0[b] = ld_stream_v4(r + static_cast<long>(c) * 16);
             if (two) v1[b] = ld_stream_v4(r + static_cast<long>(c + 32) * 16);
           }
@@ -109,13 +126,44 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
       st_stream_v4(orow + static_cast<long>(c) * 16, pack_bf16x8(a0));
       if (two) st_stream_v4(orow + static_cast<long>(c + 32) * 16, pack_bf16x8(a1));
     }
-    if (out_w != nullptr && lane < K) {
+    if (want_w && lane < K) {
       float a = 0.f;
-      for (int i = 0; i < n; ++i) a += __ldg(recv_w + rows[i] * K + lane);
+      for (int i = 0; i < n; ++i) a += __ldg(wrows[i] + lane);
       out_w[u * K + lane] = a;
     }
     __syncwarp();
   }
+}
+
+// Launch of either form (arguments already checked).
+int combine_launch(const void *y, const float *recv_w, const uint8_t *const *y_tab,
+                   const float *const *w_tab, const int32_t *send_pos, const void *bias_0,
+                   const void *bias_1, int R, long num_tok, int H, int K, int cap,
+                   void *combined_x, float *combined_w, int32_t *status, cudaStream_t stream) {
+  const int threads = kCombineWarps * 32;
+  const size_t smem = static_cast<size_t>(kCombineWarps) * 2 * R * sizeof(void *);
+  const bool tab = y_tab != nullptr;
+  const void *fn = tab ? reinterpret_cast<const void *>(combine_kernel<true>)
+                       : reinterpret_cast<const void *>(combine_kernel<false>);
+  if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
+  const long want = (num_tok + kCombineWarps - 1) / kCombineWarps;
+  const long grid =
+      std::min<long>(want, static_cast<long>(ctas_per_sm(fn, threads, smem)) * num_sms());
+  const bool want_w = combined_w != nullptr;
+  cudaError_t launched;
+  if (tab)
+    launched = launch_pdl(combine_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(threads),
+        smem, stream, static_cast<const uint8_t *>(nullptr), static_cast<const float *>(nullptr),
+        y_tab, w_tab, send_pos, static_cast<const uint8_t *>(bias_0),
+        static_cast<const uint8_t *>(bias_1), R, num_tok, H, K, cap, want_w,
+        static_cast<uint8_t *>(combined_x), combined_w, status);
+  else
+    launched = launch_pdl(combine_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(threads),
+        smem, stream, static_cast<const uint8_t *>(y), recv_w,
+        static_cast<const uint8_t *const *>(nullptr), static_cast<const float *const *>(nullptr),
+        send_pos, static_cast<const uint8_t *>(bias_0), static_cast<const uint8_t *>(bias_1), R,
+        num_tok, H, K, cap, want_w, static_cast<uint8_t *>(combined_x), combined_w, status);
+  return launch_status(launched);
 }
 
 }  // namespace
@@ -138,17 +186,30 @@ extern "C" EP_API int ep_combine(const void *y, const float *recv_topk_weights,
       (reinterpret_cast<uintptr_t>(bias_0) & 15u) || (reinterpret_cast<uintptr_t>(bias_1) & 15u))
     return EP_ERR_INVALID_ARG;
   const long num_tok = static_cast<long>(R) * T;
-  const int threads = kCombineWarps * 32;
-  const size_t smem = static_cast<size_t>(kCombineWarps) * R * sizeof(int64_t);
-  const void *fn = reinterpret_cast<const void *>(combine_kernel);
-  if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
-  const long want = (num_tok + kCombineWarps - 1) / kCombineWarps;
-  const long grid =
-      std::min<long>(want, static_cast<long>(ctas_per_sm(fn, threads, smem)) * num_sms());
-  const cudaError_t launched = launch_pdl(combine_kernel,
-      dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream,
-      static_cast<const uint8_t *>(y), combined_topk_weights ? recv_topk_weights : nullptr,
-      send_pos, static_cast<const uint8_t *>(bias_0), static_cast<const uint8_t *>(bias_1), R,
-      num_tok, H, K, cap, static_cast<uint8_t *>(combined_x), combined_topk_weights, status);
-  return launch_status(launched);
+  return combine_launch(y, combined_topk_weights != nullptr ? recv_topk_weights : nullptr, nullptr,
+                        nullptr, send_pos, bias_0, bias_1, R, num_tok, H, K, cap, combined_x,
+                        combined_topk_weights, status, stream);
+}
+
+extern "C" EP_API int ep_shard_combine(const void *const *y_peers,
+                                       const float *const *recv_topk_weights_peers,
+                                       const int32_t *send_pos, const void *bias_0,
+                                       const void *bias_1, int num_ranks, int num_tokens,
+                                       int hidden, int num_topk, int capacity, void *combined_x,
+                                       float *combined_topk_weights, int32_t *status,
+                                       cudaStream_t stream) {
+  using namespace ep;
+  const int R = num_ranks, T = num_tokens, H = hidden, K = num_topk, cap = capacity;
+  if (R < 1 || R > kMaxRanks || T < 0 || H < 8 || H % 8 != 0 || cap < 0) return EP_ERR_INVALID_ARG;
+  if (combined_topk_weights != nullptr &&
+      (recv_topk_weights_peers == nullptr || K < 1 || K > kMaxTopk))
+    return EP_ERR_INVALID_ARG;
+  if (T == 0) return EP_OK;
+  if (y_peers == nullptr || send_pos == nullptr || combined_x == nullptr) return EP_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(combined_x) & 15u) ||
+      (reinterpret_cast<uintptr_t>(bias_0) & 15u) || (reinterpret_cast<uintptr_t>(bias_1) & 15u))
+    return EP_ERR_INVALID_ARG;
+  return combine_launch(nullptr, nullptr, reinterpret_cast<const uint8_t *const *>(y_peers),
+                        recv_topk_weights_peers, send_pos, bias_0, bias_1, R, T, H, K, cap,
+                        combined_x, combined_topk_weights, status, stream);
 }

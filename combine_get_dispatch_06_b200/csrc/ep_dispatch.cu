@@ -39,12 +39,24 @@ struct DispatchScanParams {
   int32_t *recv_src_idx;
   int64_t *recv_idx;
   float *recv_w;
-  int32_t *P;
-  int32_t *recv_count;
+  int32_t *P;            // or nullptr (one rank of a sharded job: P comes from the counts)
+  int32_t *recv_count;   // or nullptr (likewise)
   int32_t *nrte;
   int32_t *ntpr_out;     // optional layout outputs (routing from topk_idx only)
   int32_t *ntpe_out;
   uint8_t *in_rank_out;
+  // One rank of a sharded job (the call's tokens are one source rank's):
+  // row of the first of its tokens in each destination, and the destination
+  // ranks' receive buffers in peer memory.  All nullptr for the simulated
+  // ranks of one GPU (rows start at 0, buffers are slices d * cap).
+  const int32_t *dst_base;   // [R]
+  int32_t *const *rsi_tab;   // [R] -> recv_src_idx rows of rank d
+  int64_t *const *ridx_tab;  // [R] -> recv_topk_idx rows of rank d (or nullptr)
+  float *const *rw_tab;      // [R] -> recv_topk_weights rows of rank d (or nullptr)
+  // Full-grid timer of the launch (or nullptr): complemented earliest block
+  // start in the workspace; cumulative [ns, launches, last start, last end].
+  unsigned long long *probe_state;
+  unsigned long long *probe;
   ScanHeader *head;
   int32_t *expert_cnt;   // [E] all sources, then [R][E] per source
   uint64_t *desc;
@@ -58,11 +70,11 @@ struct DispatchScanParams {
 // for the others.  32-bit compares and selects; 16-byte stores when K allows
 // them (rows of K int64 / K fp32 are then 16-byte aligned).
 template <int MAXK>
-__device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, size_t row, int K,
-                                           int d, const int (&dk)[MAXK], const int (&lk)[MAXK],
+__device__ __forceinline__ void write_meta(int64_t *idx_row, float *w_row, int K, int d,
+                                           const int (&dk)[MAXK], const int (&lk)[MAXK],
                                            const float (&wk)[MAXK]) {
-  if (recv_idx != nullptr) {
-    int64_t *dst = recv_idx + row * K;
+  if (idx_row != nullptr) {
+    int64_t *dst = idx_row;
     if ((K & 1) == 0) {
 #pragma unroll
       for (int k = 0; k < MAXK; k += 2) {
@@ -79,8 +91,8 @@ __device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, siz
         if (k < K) dst[k] = dk[k] == d ? static_cast<int64_t>(lk[k]) : -1ll;
     }
   }
-  if (recv_w != nullptr) {
-    float *dst = recv_w + row * K;
+  if (w_row != nullptr) {
+    float *dst = w_row;
     if ((K & 3) == 0) {
 #pragma unroll
       for (int k = 0; k < MAXK; k += 4) {
@@ -105,6 +117,7 @@ __device__ __forceinline__ void write_meta(int64_t *recv_idx, float *recv_w, siz
 template <int MAXK>
 __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanParams p) {
   pdl_wait();
+  if (p.probe != nullptr && threadIdx.x == 0) atomicMax(p.probe_state, ~globaltimer());
   __shared__ int s_tile;
   __shared__ int s_last;
   __shared__ uint32_t s_mask[kScanTile * kMaskWords];
@@ -130,8 +143,9 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   const size_t st = static_cast<size_t>(s) * p.T + t;
 
   // ---- the token's top-k ids and weights, loaded once, all at once --------
-  const bool meta =
-      valid && p.topk_idx != nullptr && (p.recv_idx != nullptr || p.recv_w != nullptr);
+  const bool want_w = p.recv_w != nullptr || p.rw_tab != nullptr;
+  const bool meta = valid && p.topk_idx != nullptr &&
+                    (p.recv_idx != nullptr || p.ridx_tab != nullptr || want_w);
   const bool need_idx = valid && p.topk_idx != nullptr;
   int64_t ek[MAXK];
   float wk[MAXK];
@@ -141,7 +155,7 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
     wk[k] = 0.f;
     if (need_idx && k < p.K) {
       ek[k] = p.topk_idx[st * p.K + k];
-      if (meta && p.recv_w != nullptr) wk[k] = p.topk_w[st * p.K + k];
+      if (meta && want_w) wk[k] = p.topk_w[st * p.K + k];
     }
   }
 
@@ -231,8 +245,8 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
       const uint32_t excl = lookback_window<G, 4>(p.desc, tile, p.R, d, static_cast<uint32_t>(run),
                                                   publish, p.timeout_ns, p.status);
       if ((tid & (G - 1)) == 0) {
-        s_excl[d] = static_cast<int>(excl);
-        if (last_of_src) {
+        s_excl[d] = static_cast<int>(excl) + (p.dst_base != nullptr ? p.dst_base[d] : 0);
+        if (last_of_src && p.P != nullptr) {
           p.P[static_cast<size_t>(s) * p.R + d] = static_cast<int>(excl) + run;
           if (tile == p.num_tiles - 1) p.recv_count[d] = static_cast<int>(excl) + run;
         }
@@ -259,9 +273,20 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
         overflow = true;
         continue;
       }
-      const size_t row = static_cast<size_t>(d) * p.cap + pos;
-      p.recv_src_idx[row] = t;
-      if (meta) write_meta(p.recv_idx, p.recv_w, row, p.K, d, dk, lk, wk);
+      if (p.rsi_tab != nullptr) {  // the destination's buffers, in peer memory
+        p.rsi_tab[d][pos] = t;
+        if (meta)
+          write_meta(p.ridx_tab != nullptr ? p.ridx_tab[d] + static_cast<size_t>(pos) * p.K
+                                           : nullptr,
+                     p.rw_tab != nullptr ? p.rw_tab[d] + static_cast<size_t>(pos) * p.K : nullptr,
+                     p.K, d, dk, lk, wk);
+      } else {
+        const size_t row = static_cast<size_t>(d) * p.cap + pos;
+        p.recv_src_idx[row] = t;
+        if (meta)
+          write_meta(p.recv_idx != nullptr ? p.recv_idx + row * p.K : nullptr,
+                     p.recv_w != nullptr ? p.recv_w + row * p.K : nullptr, p.K, d, dk, lk, wk);
+      }
     }
   }
   if (overflow) report(p.status, EP_STATUS_CAPACITY);
@@ -315,7 +340,16 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
         const int prev = i >= p.R ? __ldcg(&p.P[i - p.R]) : 0;
         p.ntpr_out[i] = __ldcg(&p.P[i]) - prev;
       }
+    if (p.probe != nullptr && tid == 0) {  // full-grid time of this launch
+      const unsigned long long end = globaltimer();
+      const unsigned long long start = ~atomicAdd(p.probe_state, 0ull);
+      atomicAdd(&p.probe[0], end - start);
+      atomicAdd(&p.probe[1], 1ull);
+      p.probe[2] = start;
+      p.probe[3] = end;
+    }
   }
+  if (p.rsi_tab != nullptr) __threadfence_system();  // stores into peers' memory
 }
 
 // ---------------------------------------------------------------------------
@@ -340,18 +374,29 @@ constexpr int kCopyShortRow = 8192;
 constexpr int kCopyMaxCtasPerSm = 2;
 
 // bf16 rows only (the headline path): the row scatter described above.
-template <int S>
+//
+// kTab: the destinations' receive buffers are given by a table of R pointers
+// (one rank of a sharded job: peers' memory); else they are slices d * cap of
+// recv_x.
+template <int S, bool kTab>
 __global__ void __launch_bounds__(kMaxRanks)
     dispatch_copy_rows_kernel(const uint8_t *__restrict__ x, const int32_t *__restrict__ send_pos,
-                         uint8_t *__restrict__ recv_x, int R, long num_tok, int row_bytes,
-                         int chunk_bytes, int nchunks, int stage_stride, int cap,
-                         int32_t *status, unsigned long long timeout_ns) {
+                         uint8_t *__restrict__ recv_x, uint8_t *const *recv_tab, int R,
+                         long num_tok, int row_bytes, int chunk_bytes, int nchunks,
+                         int stage_stride, int cap, int32_t *status,
+                         unsigned long long timeout_ns) {
   pdl_wait();
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
   uint8_t *buf = smem + 128;
   const int tid = threadIdx.x;
   const int d = tid;
+  uint8_t *my_rows = nullptr;  // this thread's destination buffer
+  if (kTab) {
+    if (d < R) my_rows = recv_tab[d];
+  } else {
+    my_rows = recv_x + static_cast<long>(d) * cap * row_bytes;
+  }
 
   const long ntok_cta =
       static_cast<long>(blockIdx.x) < num_tok ? (num_tok - 1 - blockIdx.x) / gridDim.x + 1 : 0;
@@ -404,7 +449,7 @@ __global__ void __launch_bounds__(kMaxRanks)
         if (sp[st] < cap) {
           const int off = chunk * chunk_bytes;
           const int nb = min(chunk_bytes, row_bytes - off);
-          bulk_s2g(recv_x + (static_cast<long>(d) * cap + sp[st]) * row_bytes + off,
+          bulk_s2g(my_rows + static_cast<long>(sp[st]) * row_bytes + off,
                    buf + st * stage_stride, static_cast<uint32_t>(nb));
         } else if (chunk == 0) {
           report(status, EP_STATUS_CAPACITY);
@@ -427,6 +472,7 @@ __global__ void __launch_bounds__(kMaxRanks)
   }
   pdl_trigger();
   bulk_wait_all<0>();
+  if (kTab) __threadfence_system();  // the rows went to peers' memory
   if (!all_ok) {
     report(status, EP_STATUS_WAIT_TIMEOUT);
     if (tid == 0) {
@@ -695,6 +741,12 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   p.ntpr_out = ntpr_out;
   p.ntpe_out = ntpe_out;
   p.in_rank_out = in_rank_out;
+  p.dst_base = nullptr;
+  p.rsi_tab = nullptr;
+  p.ridx_tab = nullptr;
+  p.rw_tab = nullptr;
+  p.probe_state = nullptr;
+  p.probe = nullptr;
   p.head = reinterpret_cast<ScanHeader *>(ws);
   p.expert_cnt = reinterpret_cast<int32_t *>(ws + sizeof(ScanHeader));
   const int counters = Ectr * (1 + R);
@@ -729,7 +781,8 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
 // scales, [R][T][nblk] or, col_major, [R][nblk][T]) may be nullptr.
 int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int32_t *send_pos,
               int R, int T, int row_bytes, int cap, void *recv_x, float *recv_s,
-              int32_t *status, cudaStream_t stream) {
+              int32_t *status, cudaStream_t stream, void *const *recv_tab = nullptr,
+              int num_src = -1) {
   if (T == 0 || cap == 0) return EP_OK;
   CopyArgs a;
   a.x = static_cast<const uint8_t *>(x);
@@ -740,7 +793,7 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
   a.R = R;
   a.T = T;
   a.cap = cap;
-  a.num_tok = static_cast<long>(R) * T;
+  a.num_tok = static_cast<long>(num_src < 0 ? R : num_src) * T;  // source tokens of the call
   a.row_bytes = row_bytes;
   const bool short_rows = row_bytes <= kCopyShortRow;
   a.nchunks = short_rows ? 1 : (row_bytes + kCopyChunkMax - 1) / kCopyChunkMax;
@@ -769,9 +822,14 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
   if (xs != nullptr)
     fn = short_rows ? reinterpret_cast<const void *>(dispatch_copy_planes_kernel<kCopyStagesShort, true>)
                     : reinterpret_cast<const void *>(dispatch_copy_planes_kernel<kCopyStages, true>);
+  else if (recv_tab != nullptr)
+    fn = short_rows
+             ? reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStagesShort, true>)
+             : reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStages, true>);
   else
-    fn = short_rows ? reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStagesShort>)
-                    : reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStages>);
+    fn = short_rows
+             ? reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStagesShort, false>)
+             : reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStages, false>);
   if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
   const long grid = std::min<long>(
       a.num_tok,
@@ -787,15 +845,24 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
       launched = launch_pdl(dispatch_copy_planes_kernel<kCopyStages, true>,
           dim3(g), dim3(b), smem, stream,
         a);
-  } else if (short_rows) {
-    launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStagesShort>,
-        dim3(g), dim3(b), smem, stream,
-        a.x, a.send_pos, a.recv_x, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
-        a.stage_stride, a.cap, a.status, a.timeout_ns);
   } else {
-    launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStages>, dim3(g), dim3(b), smem, stream,
-        a.x, a.send_pos, a.recv_x, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
-        a.stage_stride, a.cap, a.status, a.timeout_ns);
+    auto *tab = reinterpret_cast<uint8_t *const *>(recv_tab);
+    if (recv_tab != nullptr && short_rows)
+      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStagesShort, true>, g, b, smem, stream,
+          a.x, a.send_pos, a.recv_x, tab, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
+          a.stage_stride, a.cap, a.status, a.timeout_ns);
+    else if (recv_tab != nullptr)
+      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStages, true>, g, b, smem, stream,
+          a.x, a.send_pos, a.recv_x, tab, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
+          a.stage_stride, a.cap, a.status, a.timeout_ns);
+    else if (short_rows)
+      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStagesShort, false>, g, b, smem,
+          stream, a.x, a.send_pos, a.recv_x, tab, a.R, a.num_tok, a.row_bytes, a.chunk_bytes,
+          a.nchunks, a.stage_stride, a.cap, a.status, a.timeout_ns);
+    else
+      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStages, false>, g, b, smem, stream,
+          a.x, a.send_pos, a.recv_x, tab, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
+          a.stage_stride, a.cap, a.status, a.timeout_ns);
   }
   return launch_status(launched);
 }
@@ -954,6 +1021,179 @@ extern "C" EP_API int ep_dispatch(const void *x, const int64_t *topk_idx,
   if (rc != EP_OK) return rc;
   return copy_impl(x, nullptr, 0, 0, send_pos, num_ranks, num_tokens, hidden * 2, capacity,
                    recv_x, nullptr, status, stream);
+}
+
+// ---------------------------------------------------------------------------
+// One rank per GPU (sharded job).  The calling process holds one source rank
+// `rank` of R; the counts every rank sends to every destination, gathered by
+// the caller's collective, give the rank prefix matrix (the notify step of
+// the pages' dispatch); the scan above then runs over this rank's tokens
+// alone, offset by the rows lower ranks take in each destination, and writes
+// the received metadata and the rows straight into the destinations' receive
+// buffers in peer memory.
+// ---------------------------------------------------------------------------
+
+namespace ep {
+namespace {
+
+// Workspace of a sharded notify: header, the probe's complemented earliest
+// start (8 bytes) and the R destination bases, then the look-back
+// descriptors of this rank's tiles.
+struct ShardWs {
+  ScanHeader *head;
+  unsigned long long *probe_state;
+  int32_t *base;
+  uint64_t *desc;
+};
+
+ShardWs shard_ws(void *workspace, int R) {
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  ShardWs w;
+  w.head = reinterpret_cast<ScanHeader *>(ws);
+  w.probe_state = reinterpret_cast<unsigned long long *>(ws + sizeof(ScanHeader));
+  w.base = reinterpret_cast<int32_t *>(ws + sizeof(ScanHeader) + 16);
+  const long counters = 4 + R;  // probe state (2 ints, padded to 4), bases
+  w.desc = reinterpret_cast<uint64_t *>(ws + sizeof(ScanHeader) +
+                                        static_cast<size_t>((counters + 3) & ~3L) * 4);
+  return w;
+}
+
+// P[s][d] = sum over s' <= s of counts[s'][d] (inclusive over source ranks),
+// base[d] = P[rank - 1][d] (0 for rank 0), recv_count = P[R - 1][rank], and
+// the received slots of each local expert, sum over s of
+// expert_counts[s][rank * E_l + j], rounded up to the alignment.
+__global__ void __launch_bounds__(256)
+    shard_prefix_kernel(const int32_t *__restrict__ counts, const int32_t *__restrict__ ecounts,
+                        int R, int E, int rank, int align, int32_t *__restrict__ P,
+                        int32_t *__restrict__ base, int32_t *__restrict__ recv_count,
+                        int32_t *__restrict__ nrte) {
+  pdl_wait();
+  pdl_trigger();
+  for (int d = threadIdx.x; d < R; d += blockDim.x) {
+    int run = 0;
+    if (rank == 0) base[d] = 0;
+    for (int s = 0; s < R; ++s) {
+      run += counts[static_cast<size_t>(s) * R + d];
+      P[static_cast<size_t>(s) * R + d] = run;
+      if (s == rank - 1) base[d] = run;
+    }
+    if (d == rank) recv_count[0] = run;
+  }
+  if (nrte != nullptr) {
+    const int El = E / R;
+    for (int j = threadIdx.x; j < El; j += blockDim.x) {
+      int n = 0;
+      for (int s = 0; s < R; ++s) n += ecounts[static_cast<size_t>(s) * E + rank * El + j];
+      if (align > 1) n = (n + align - 1) / align * align;
+      nrte[j] = n;
+    }
+  }
+}
+
+}  // namespace
+}  // namespace ep
+
+extern "C" EP_API size_t ep_shard_workspace_bytes(int num_ranks, int num_tokens) {
+  using namespace ep;
+  if (num_ranks < 1 || num_tokens < 0) return 0;
+  const long tiles = (num_tokens + kScanTile - 1) / kScanTile;
+  return scan_workspace_bytes(tiles, num_ranks, 4L + num_ranks);
+}
+
+extern "C" EP_API int ep_shard_notify(
+    const int64_t *topk_idx, const float *topk_weights, const int32_t *counts,
+    const int32_t *expert_counts, int rank, int num_ranks, int num_tokens, int num_topk,
+    int num_experts, int expert_alignment, int capacity, int32_t *const *recv_src_idx_peers,
+    int64_t *const *recv_topk_idx_peers, float *const *recv_topk_weights_peers,
+    int64_t *recv_topk_idx, int32_t *rank_prefix_matrix, int32_t *recv_count,
+    int32_t *num_recv_tokens_per_expert, int32_t *send_pos, unsigned long long *notify_probe,
+    void *workspace, size_t workspace_bytes, int32_t *status, cudaStream_t stream) {
+  using namespace ep;
+  const int R = num_ranks, T = num_tokens, K = num_topk, E = num_experts;
+  const int cap = capacity, align = expert_alignment;
+  if (R < 1 || R > kMaxRanks || rank < 0 || rank >= R || T < 0 || cap < 0 || align < 1)
+    return EP_ERR_INVALID_ARG;
+  if (K < 1 || K > kMaxTopk || E < 1 || E > kMaxExperts || E % R != 0) return EP_ERR_INVALID_ARG;
+  if (counts == nullptr || rank_prefix_matrix == nullptr || recv_count == nullptr)
+    return EP_ERR_INVALID_ARG;
+  if (num_recv_tokens_per_expert != nullptr && expert_counts == nullptr) return EP_ERR_INVALID_ARG;
+  if ((recv_topk_idx_peers != nullptr) != (recv_topk_idx != nullptr)) return EP_ERR_INVALID_ARG;
+  if (T > 0 && (topk_idx == nullptr || recv_src_idx_peers == nullptr || send_pos == nullptr))
+    return EP_ERR_INVALID_ARG;
+  if (T > 0 && recv_topk_weights_peers != nullptr && topk_weights == nullptr)
+    return EP_ERR_INVALID_ARG;
+  const size_t need = ep_shard_workspace_bytes(R, T);
+  if (workspace == nullptr || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 15u) ||
+      (reinterpret_cast<uintptr_t>(notify_probe) & 7u))
+    return EP_ERR_INVALID_ARG;
+
+  if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return EP_ERR_CUDA;
+  const ShardWs w = shard_ws(workspace, R);
+  cudaError_t launched = launch_pdl(shard_prefix_kernel, dim3(1), dim3(256), 0, stream, counts,
+                                    expert_counts, R, E, rank, align, rank_prefix_matrix,
+                                    w.base, recv_count, num_recv_tokens_per_expert);
+  if (launch_status(launched) != EP_OK) return EP_ERR_CUDA;
+  if (T > 0) {
+    const int tiles = (T + kScanTile - 1) / kScanTile;
+    DispatchScanParams p = {};
+    p.topk_idx = topk_idx;
+    p.topk_w = topk_weights;
+    p.in_rank = nullptr;
+    p.R = R;
+    p.T = T;
+    p.K = K;
+    p.E = E;
+    p.El = E / R;
+    p.el_div = make_fastdiv(p.El);
+    p.cap = cap;
+    p.align = align;
+    p.tiles_per_src = tiles;
+    p.num_tiles = tiles;  // one source rank
+    p.W = (R + 31) / 32;
+    p.send_pos = send_pos;
+    p.dst_base = w.base;
+    p.rsi_tab = recv_src_idx_peers;
+    p.ridx_tab = recv_topk_idx_peers;
+    p.rw_tab = recv_topk_weights_peers;
+    p.probe_state = notify_probe != nullptr ? w.probe_state : nullptr;
+    p.probe = notify_probe;
+    p.head = w.head;
+    p.desc = w.desc;
+    p.status = status;
+    const WaitConfig wc = wait_config();
+    p.timeout_ns = wc.timeout_ns;
+    p.flags = wc.flags;
+    if (K > 8)
+      launched = launch_pdl(dispatch_scan_kernel<16>, dim3(tiles), dim3(kScanTile), 0, stream, p);
+    else
+      launched = launch_pdl(dispatch_scan_kernel<8>, dim3(tiles), dim3(kScanTile), 0, stream, p);
+    if (launch_status(launched) != EP_OK) return EP_ERR_CUDA;
+  }
+  // this rank's own receive rows past its count read -1 (fixed capacity)
+  if (recv_topk_idx != nullptr && cap > 0) {
+    const long words = static_cast<long>(cap) * K / ((K & 1) == 0 ? 2 : 1);
+    const int bx = static_cast<int>(std::min<long>((words + 255) / 256, 64));
+    launched = launch_pdl(pad_recv_idx_kernel, dim3(bx, 1), dim3(256), 0, stream, recv_count,
+                          cap, K, recv_topk_idx);
+    return launch_status(launched);
+  }
+  return EP_OK;
+}
+
+extern "C" EP_API int ep_shard_dispatch(const void *x, const int32_t *send_pos, int num_ranks,
+                                        int num_tokens, int hidden, int capacity,
+                                        void *const *recv_x_peers, int32_t *status,
+                                        cudaStream_t stream) {
+  using namespace ep;
+  const int R = num_ranks, T = num_tokens, H = hidden, cap = capacity;
+  if (R < 1 || R > kMaxRanks || T < 0 || H < 8 || H % 8 != 0 || cap < 0)
+    return EP_ERR_INVALID_ARG;
+  if (T == 0 || cap == 0) return EP_OK;
+  if (x == nullptr || send_pos == nullptr || recv_x_peers == nullptr) return EP_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(x) & 15u) return EP_ERR_INVALID_ARG;
+  return copy_impl(x, nullptr, 0, 0, send_pos, R, T, H * 2, cap, nullptr, nullptr, status, stream,
+                   recv_x_peers, 1);
 }
 
 // ---------------------------------------------------------------------------

@@ -214,9 +214,10 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
 
 // ---------------------------------------------------------------------------
 
-constexpr int kLLThreads = 256;  // 8 warps quantise one token row together
-constexpr int kLLInStages = 2;  // >= 2: warp 0 reads the next stage's token ahead
+constexpr int kLLThreads = 256;     // 8 warps quantise one token row together
+constexpr int kLLMaxStages = 4;     // input rows in flight per CTA (fewer when H is large)
 constexpr int kLLMaxCtasPerSm = 3;
+constexpr int kLLMaxDynSmem = 227 * 1024 - 1024;  // the CTA's limit, less its static arrays
 
 __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float d) {
   // element order in memory: a, b, c, d (a in the lowest byte)
@@ -226,36 +227,36 @@ __device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float 
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-static_assert(kLLInStages >= 2, "the next token must sit in another stage");
-constexpr int kLLMaxDynSmem = 227 * 1024 - 1024;  // the CTA's limit, less its static arrays
-
-// Shared-memory plan of one CTA: 128 bytes of mbarriers, kLLInStages input
-// rows (bf16, filled by bulk copies), then (FP8 only) two e4m3 output rows
-// with their scales, used alternately by consecutive tokens.
+// Shared-memory plan of one CTA: 128 bytes of mbarriers, then `stages` input
+// rows (bf16, filled by bulk copies), as many as fit (at most kLLMaxStages,
+// at least 2).
 struct LLSmem {
-  int in_stride;   // bytes per input stage (multiple of 128)
-  int out_stride;  // bytes per output buffer (e4m3 row + scales, multiple of 128)
-  int sc_off;      // offset of the scales inside an output buffer
-  int bytes;       // total
+  int in_stride;  // bytes per input stage (multiple of 128)
+  int stages;     // input stages; 0 if not even 2 fit
+  int bytes;      // total
 };
 
-__host__ __device__ inline LLSmem ll_smem_plan(int H, bool fp8) {
+__host__ __device__ inline LLSmem ll_smem_plan(int H) {
   LLSmem m;
   m.in_stride = (2 * H + 127) & ~127;
-  m.sc_off = (H + 127) & ~127;
-  m.out_stride = fp8 ? m.sc_off + (((H / 128) * 4 + 127) & ~127) : 0;
-  m.bytes = 128 + kLLInStages * m.in_stride + 2 * m.out_stride;
+  const long fit = (static_cast<long>(kLLMaxDynSmem) - 128) / m.in_stride;
+  m.stages = fit >= 2 ? static_cast<int>(fit < kLLMaxStages ? fit : kLLMaxStages) : 0;
+  m.bytes = 128 + m.stages * m.in_stride;
   return m;
 }
 
 // One CTA per token at a time.  Tokens are claimed from a shared counter
 // (`claim`, zeroed with the workspace), so CTAs that run faster take more of
-// them and the grid finishes together.  Thread 0 keeps kLLInStages claimed
-// rows in flight as bulk loads and claims one more token ahead, to hide the
-// atomic's round trip.  All 256 threads quantise the current row (16
-// consecutive threads per 128-channel block, amax by xor-shuffles); then warp
-// 0's lanes, one per distinct expert of the token, send the e4m3 row and its
-// scales with bulk shared->global stores.
+// them and the grid finishes together.  Thread 0 keeps `stages` claimed rows
+// in flight as bulk loads and claims one more token ahead, to hide the
+// atomic's round trip.  Warp 0 turns the token's mirrored slab positions into
+// one destination row per distinct expert (in shared memory); then every
+// thread quantises its 16-channel chunks (8 threads per 128-channel block,
+// amax by xor-shuffles) in registers and stores each 16-byte chunk of e4m3
+// codes straight to every destination row, and the block's first thread
+// stores the block's scale there.  (bf16 payload: 8-channel chunks copied
+// unchanged.)  Nothing waits for the stores: a stage is refilled as soon as
+// every thread has read it.
 //
 // The kernel runs concurrently with ll_scan_kernel (see there): rows and
 // expert ids are inputs and are read at once; a token's slab rows come from
@@ -271,18 +272,17 @@ __global__ void __launch_bounds__(kLLThreads)
                        unsigned long long timeout_ns) {
   pdl_trigger();  // the next kernel may take the room this grid leaves
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ long s_tok[kLLInStages];  // token in each input stage, -1 = none
+  __shared__ long s_tok[kLLMaxStages];  // token in each input stage, -1 = none
+  __shared__ long s_dst[kMaxTopk];      // slab row (e * cap + pos) per slot, -1 = none
   const int tid = threadIdx.x;
   const int lane = tid & 31;
+  const int nst = plan.stages;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
   uint8_t *inb = smem + 128;
-  uint8_t *outb = inb + kLLInStages * plan.in_stride;
-  const int nvec = H >> 3;
-  const int nblk = H >> 7;
   const int row_in = 2 * H;
-  const int pay = kFP8 ? H : 2 * H;
-  const int sc_bytes = ue8m0 ? nblk : nblk * 4;  // fp32 scales or UE8M0 exponent bytes
-  const bool bulk_scales = (sc_bytes & 15) == 0;
+  const int pay = kFP8 ? H : 2 * H;             // bytes per slab row
+  const int nchunk = kFP8 ? (H >> 4) : (H >> 3);  // 16 (FP8) or 8 (bf16) channels per chunk
+  const int nblk = H >> 7;
   float *scales = static_cast<float *>(scales_out);
   uint8_t *scales8 = static_cast<uint8_t *>(scales_out);
 
@@ -312,11 +312,9 @@ __global__ void __launch_bounds__(kLLThreads)
 
   long ahead = -1;  // thread 0: the token claimed for the next issue
   if (tid == 0) {
-#pragma unroll
-    for (int i = 0; i < kLLInStages; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < nst; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
-#pragma unroll
-    for (int i = 0; i < kLLInStages; ++i) issue(i, i == 0 ? static_cast<long>(blockIdx.x) : take());
+    for (int i = 0; i < nst; ++i) issue(i, i == 0 ? static_cast<long>(blockIdx.x) : take());
     ahead = take();
   }
   __syncthreads();
@@ -330,88 +328,26 @@ __global__ void __launch_bounds__(kLLThreads)
   }
 
   bool all_ok = true;
-  long stop = -1;
-  for (long i = 0;; ++i) {
-    const int stg = static_cast<int>(i % kLLInStages);
+  int stop = -1;      // stage whose load was the first not waited for, on failure
+  int stg = 0;
+  uint32_t phase = 0;
+  while (true) {
     const long u = s_tok[stg];
     if (u < 0) break;  // claims are ordered: every later stage is empty too
-    uint8_t *in = inb + stg * plan.in_stride;
+    const uint8_t *in = inb + stg * plan.in_stride;
+    const int nxt = stg + 1 == nst ? 0 : stg + 1;
 
-    // warp 0: this token's experts and rows (read a token ahead); start
+    // warp 0: this token's destination rows (read a token ahead); start
     // reading the next token's
-    int e = -1;
-    int32_t m = 0;
     if (tid < 32) {
-      e = e_next;
-      m = m_next;
-      const long un = s_tok[(i + 1) % kLLInStages];
+      __syncwarp();  // lane 0's last issue() wrote s_tok[nxt]
+      const int e = e_next;
+      int32_t m = m_next;
+      const long un = s_tok[nxt];
       e_next = expert_of(un);
       m_next = mirror_of(un);
-      // FP8: the output buffer of token i - 2 must have been read by its stores
-      if (kFP8) bulk_wait_read<1>();
-    }
-    const bool ok =
-        mbar_wait_bounded(&bars[stg], static_cast<uint32_t>((i / kLLInStages) & 1), timeout_ns);
-    if (__syncthreads_and(ok) == 0) {
-      all_ok = false;
-      stop = i;
-      break;
-    }
-
-    const uint8_t *src = in;
-    float *sc = nullptr;
-    if constexpr (kFP8) {
-      uint8_t *q = outb + static_cast<int>(i & 1) * plan.out_stride;
-      sc = reinterpret_cast<float *>(q + plan.sc_off);
-#pragma unroll 2
-      for (int c0 = 0; c0 < nvec; c0 += kLLThreads) {
-        const int c = c0 + tid;
-        const bool act = c < nvec;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (act) v = reinterpret_cast<const uint4 *>(in)[c];
-        float f[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
-                      bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
-        float amax = 0.f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
-        // 16 consecutive threads hold one 128-channel block (nvec % 16 == 0)
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        amax = fmaxf(amax, 1e-4f);
-        float inv, scale;
-        uint32_t ebits = 0;
-        if (round_scale) {
-          // smallest power of two >= amax / 448, and its exact reciprocal
-          const uint32_t b = __float_as_uint(__fdiv_rn(amax, 448.0f));
-          ebits = (b >> 23) + ((b & 0x7FFFFFu) != 0u ? 1u : 0u);
-          scale = __uint_as_float(ebits << 23);
-          inv = __uint_as_float((254u - ebits) << 23);
-        } else {
-          inv = __fdiv_rn(448.0f, amax);
-          scale = __fdiv_rn(amax, 448.0f);
-        }
-        if (act) {
-          uint2 qq;
-          qq.x = cvt_e4m3x4(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv), __fmul_rn(f[2], inv),
-                            __fmul_rn(f[3], inv));
-          qq.y = cvt_e4m3x4(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv), __fmul_rn(f[6], inv),
-                            __fmul_rn(f[7], inv));
-          reinterpret_cast<uint2 *>(q)[c] = qq;
-          if ((c & 15) == 0) {
-            if (ue8m0)
-              reinterpret_cast<uint8_t *>(sc)[c >> 4] = static_cast<uint8_t>(ebits);
-            else
-              sc[c >> 4] = scale;
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      __syncthreads();
-      src = q;
-    }
-    if (tid < 32) {
-      // slab rows of this token: words still zero are read again (bounded);
-      // after a wait ran out, this and later tokens are dropped
+      // words still zero are read again (bounded); after a wait ran out,
+      // this and later tokens are dropped
       if (!failed) {
         uint64_t t0 = 0;
         while (!__all_sync(0xffffffffu, m != 0)) {
@@ -440,39 +376,104 @@ __global__ void __launch_bounds__(kLLThreads)
         else if (pos != -1)
           report(status, EP_STATUS_BAD_POSITION);
       }
-      if (dst >= 0) {
-        bulk_s2g(recv + dst * pay, src, static_cast<uint32_t>(pay));
-        if constexpr (kFP8) {
-          if (bulk_scales)
-            bulk_s2g(scales8 + dst * sc_bytes, sc, static_cast<uint32_t>(sc_bytes));
-          else if (ue8m0)
-            for (int j = 0; j < nblk; ++j)
-              scales8[dst * nblk + j] = reinterpret_cast<const uint8_t *>(sc)[j];
-          else
-            for (int j = 0; j < nblk; ++j) scales[dst * nblk + j] = sc[j];
+      if (lane < K) s_dst[lane] = dst;
+    }
+    const bool ok = mbar_wait_bounded(&bars[stg], phase, timeout_ns);
+    if (__syncthreads_and(ok) == 0) {
+      all_ok = false;
+      stop = stg;
+      break;
+    }
+
+    if constexpr (kFP8) {
+      for (int c0 = 0; c0 < nchunk; c0 += kLLThreads) {
+        const int c = c0 + tid;
+        const bool act = c < nchunk;
+        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+        if (act) {
+          v0 = reinterpret_cast<const uint4 *>(in)[2 * c];
+          v1 = reinterpret_cast<const uint4 *>(in)[2 * c + 1];
+        }
+        float f[16] = {bf16lo(v0.x), bf16hi(v0.x), bf16lo(v0.y), bf16hi(v0.y),
+                       bf16lo(v0.z), bf16hi(v0.z), bf16lo(v0.w), bf16hi(v0.w),
+                       bf16lo(v1.x), bf16hi(v1.x), bf16lo(v1.y), bf16hi(v1.y),
+                       bf16lo(v1.z), bf16hi(v1.z), bf16lo(v1.w), bf16hi(v1.w)};
+        float amax = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(f[j]));
+        // 8 consecutive threads hold one 128-channel block (nchunk % 8 == 0)
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        amax = fmaxf(amax, 1e-4f);
+        float inv, scale;
+        uint32_t ebits = 0;
+        if (round_scale) {
+          // smallest power of two >= amax / 448, and its exact reciprocal
+          const uint32_t b = __float_as_uint(__fdiv_rn(amax, 448.0f));
+          ebits = (b >> 23) + ((b & 0x7FFFFFu) != 0u ? 1u : 0u);
+          scale = __uint_as_float(ebits << 23);
+          inv = __uint_as_float((254u - ebits) << 23);
+        } else {
+          inv = __fdiv_rn(448.0f, amax);
+          scale = __fdiv_rn(amax, 448.0f);
+        }
+        if (act) {
+          uint4 q;
+          q.x = cvt_e4m3x4(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv), __fmul_rn(f[2], inv),
+                           __fmul_rn(f[3], inv));
+          q.y = cvt_e4m3x4(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv), __fmul_rn(f[6], inv),
+                           __fmul_rn(f[7], inv));
+          q.z = cvt_e4m3x4(__fmul_rn(f[8], inv), __fmul_rn(f[9], inv), __fmul_rn(f[10], inv),
+                           __fmul_rn(f[11], inv));
+          q.w = cvt_e4m3x4(__fmul_rn(f[12], inv), __fmul_rn(f[13], inv), __fmul_rn(f[14], inv),
+                           __fmul_rn(f[15], inv));
+          const bool first = (c & 7) == 0;
+          for (int k = 0; k < K; ++k) {
+            const long dst = s_dst[k];
+            if (dst < 0) continue;
+            st_stream_v4(recv + dst * pay + c * 16L, q);
+            if (first) {
+              if (ue8m0)
+                scales8[dst * nblk + (c >> 3)] = static_cast<uint8_t>(ebits);
+              else
+                scales[dst * nblk + (c >> 3)] = scale;
+            }
+          }
         }
       }
-      bulk_commit();
-      if (!kFP8) bulk_wait_read<0>();  // bf16 forwards straight from `in`
+    } else {
+      for (int c = tid; c < nchunk; c += kLLThreads) {
+        const uint4 v = reinterpret_cast<const uint4 *>(in)[c];
+        for (int k = 0; k < K; ++k) {
+          const long dst = s_dst[k];
+          if (dst >= 0) st_stream_v4(recv + dst * pay + c * 16L, v);
+        }
+      }
     }
-    if (!kFP8) __syncthreads();
-    // `in` is free: quantised (FP8) or read by the stores (bf16)
+    __syncthreads();  // every thread has read the stage and the rows
     if (tid == 0) {
       fence_proxy_async_smem();
       const long next = ahead;
       ahead = next >= 0 ? take() : -1L;
       issue(stg, next);
     }
+    stg = nxt;
+    if (stg == 0) phase ^= 1u;
   }
-  if (tid < 32) bulk_wait_all<0>();
   if (!all_ok) {
     report(status, EP_STATUS_WAIT_TIMEOUT);
     if (tid == 0) {
-      // drain the loads still in flight before the CTA's shared memory goes away
-      for (long k = stop; k < stop + kLLInStages; ++k)
-        if (s_tok[k % kLLInStages] >= 0)
-          (void)mbar_wait_bounded(&bars[k % kLLInStages],
-                                  static_cast<uint32_t>((k / kLLInStages) & 1), timeout_ns);
+      // drain the loads still in flight before the CTA's shared memory goes
+      // away: every stage from the failed one on holds one in flight
+      int sg = stop;
+      uint32_t ph = phase;
+      for (int n = 0; n < nst; ++n) {
+        if (s_tok[sg] >= 0) (void)mbar_wait_bounded(&bars[sg], ph, timeout_ns);
+        if (++sg == nst) {
+          sg = 0;
+          ph ^= 1u;
+        }
+      }
     }
   }
   // the scan grid completes before this one does
@@ -634,6 +635,8 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   const int tiles_per_src = (T + kScanTile - 1) / kScanTile;
   const long num_tiles = static_cast<long>(R) * tiles_per_src;
   if (cap > 0x7ffffffdL) return EP_ERR_UNSUPPORTED;  // mirror words hold ll_pos + 2
+  const LLSmem plan = ll_smem_plan(H);               // input rows staged whole
+  if (plan.stages < 2) return EP_ERR_UNSUPPORTED;
   // header, descriptors and the mirror words this call uses start at zero
   const size_t used = ll_mirror_offset(num_tiles, E) + static_cast<size_t>(cap) * K * sizeof(int32_t);
   if (cudaMemsetAsync(workspace, 0, used, stream) != cudaSuccess) return EP_ERR_CUDA;
@@ -678,8 +681,6 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
         p);
   if (launch_status(launched) != EP_OK) return EP_ERR_CUDA;
 
-  const LLSmem plan = ll_smem_plan(H, use_fp8 != 0);
-  if (plan.bytes > kLLMaxDynSmem) return EP_ERR_UNSUPPORTED;
   const size_t smem = spread_smem(static_cast<size_t>(plan.bytes), kLLMaxCtasPerSm);
   const long num_tok = static_cast<long>(R) * T;
   const void *fn = use_fp8 ? reinterpret_cast<const void *>(ll_dispatch_kernel<true>)

@@ -351,9 +351,9 @@ EP_API size_t ep_ll_workspace_bytes(int num_ranks, int num_tokens,
  *   cumulative_local_expert_recv_stats  int32 [R, E_l] or NULL: each call adds
  *                  its recv_count (the pages' cumulative per-expert counter)
  *   workspace      ep_ll_workspace_bytes(R, T, E) bytes, any content
- * H is limited by shared memory (two staged input rows per CTA, plus two
- * e4m3 rows for FP8): FP8 needs H <= 38016 and bf16 H <= 57792; larger
- * returns EP_ERR_UNSUPPORTED.
+ * H is limited by shared memory (at least two bf16 input rows staged per
+ * CTA): H <= 57792 (FP8: H <= 57728, a multiple of 128); larger returns
+ * EP_ERR_UNSUPPORTED.
  */
 EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
                           const int32_t *rank_mask, int num_ranks,
@@ -391,6 +391,136 @@ EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
                          int num_tokens, int hidden, int num_topk,
                          int num_experts, void *out, int32_t *status,
                          cudaStream_t stream);
+
+/* ==========================================================================
+ * One rank per GPU (sharded job).
+ *
+ * Passage: the Buffer of the DeepEP "Python 接口" page ("Distributed /
+ * ProcessGroup"): every rank allocates its communication buffer, the ranks
+ * all-gather device ids and IPC handles over a torch.distributed group, and
+ * each rank then writes into its peers' buffers directly; the dispatch notify
+ * step exchanges per-rank token counts before the data moves (DeepEP PR #720
+ * page, "Notify full-kernel duration", non-cached dispatch notify).
+ *
+ * Here each process holds ONE source rank `rank` of R, with its T tokens.
+ * The path of one dispatch + combine:
+ *   1. ep_get_dispatch_layout on the rank's own tokens (S = 1): its row of
+ *      num_tokens_per_rank [R] and num_tokens_per_expert [E];
+ *   2. the caller all-gathers those rows over its process group into
+ *      counts [R, R] and expert_counts [R, E] (the notify exchange);
+ *   3. ep_shard_notify: rank prefix matrix, this rank's send positions, and
+ *      the received metadata written into every destination's buffers;
+ *   4. ep_shard_dispatch: the token rows written into the destinations'
+ *      receive buffers;
+ *   5. a cross-rank synchronisation by the caller (a collective on the
+ *      stream, or stream sync + barrier) before receive buffers are read;
+ *   6. ep_shard_combine: each rank gathers its tokens' rows back from the
+ *      destinations' expert outputs and reduces them exactly as ep_combine
+ *      (fp32, ascending destination rank, one rounding), so the results are
+ *      bit-identical to the single-GPU path on the same inputs;
+ *   7. a synchronisation before any rank overwrites buffers peers still read.
+ * No kernel waits on another rank: all cross-rank ordering is the caller's
+ * synchronisation.  Peers' memory is written with plain and bulk (TMA)
+ * stores and read with plain loads; no multicast form is used.
+ *
+ * "Peer tables" are DEVICE arrays of R device pointers, entry d pointing at
+ * rank d's buffer as mapped in this process (this rank's own buffer at entry
+ * `rank`), built once from ep_ipc_open.
+ * ========================================================================== */
+
+#define EP_IPC_HANDLE_BYTES 64
+
+/* Allocate `bytes` of device memory on the current device for buffers that
+ * peers map (zeroed; a plain cudaMalloc allocation, so its IPC handle covers
+ * it from its first byte).  The one allocating call of the library; it
+ * synchronises the device.  Free with ep_shard_free. */
+EP_API int ep_shard_alloc(size_t bytes, void **ptr);
+EP_API int ep_shard_free(void *ptr);
+
+/* The IPC handle (EP_IPC_HANDLE_BYTES host bytes) of an allocation made by
+ * ep_shard_alloc, for the other ranks of the job. */
+EP_API int ep_ipc_handle(const void *ptr, void *handle);
+
+/* Map another process's allocation from its handle (peer access enabled
+ * lazily); *ptr is its first byte in this process.  A handle cannot be opened
+ * in the process that made it.  Unmap with ep_ipc_close. */
+EP_API int ep_ipc_open(const void *handle, void **ptr);
+EP_API int ep_ipc_close(void *ptr);
+
+/* Workspace bytes of ep_shard_notify for R ranks and T tokens on this rank. */
+EP_API size_t ep_shard_workspace_bytes(int num_ranks, int num_tokens);
+
+/*
+ * Notify + received metadata of one rank of a sharded job.
+ *
+ *   topk_idx, topk_weights  int64 / fp32 [T, K], this rank's tokens
+ *   counts            int32 [R, R]: counts[s][d] = tokens rank s sends to d
+ *                     (every rank's num_tokens_per_rank row, gathered)
+ *   expert_counts     int32 [R, E] (every rank's num_tokens_per_expert) or
+ *                     NULL (then num_recv_tokens_per_expert must be NULL)
+ *   rank              this process's rank, 0 <= rank < R
+ *   recv_src_idx_peers     peer table of int32 [cap] receive buffers
+ *   recv_topk_idx_peers    peer table of int64 [cap, K] buffers, or NULL
+ *   recv_topk_weights_peers peer table of fp32 [cap, K] buffers, or NULL
+ *   recv_topk_idx     this rank's own int64 [cap, K] buffer (entry `rank` of
+ *                     recv_topk_idx_peers; NULL iff that table is NULL): its
+ *                     rows from recv_count to cap - 1 are set to -1
+ * Outputs (this rank's device memory):
+ *   rank_prefix_matrix int32 [R, R], P[s][d] = sum over s' <= s of counts
+ *   recv_count        int32 [1]: rows this rank receives, P[R-1][rank]
+ *   num_recv_tokens_per_expert int32 [E_l] or NULL: slots this rank's
+ *                     experts receive, rounded up to expert_alignment
+ *   send_pos          int32 [T, R]: row of (rank, t) in destination d
+ *                     (P[rank-1][d] + earlier tokens of this rank to d), or -1
+ *   notify_probe      uint64 [4] or NULL: a full-grid timer of the notify
+ *                     scan kernel, from the earliest block start to the
+ *                     last block end in %globaltimer ns: [0] += duration,
+ *                     [1] += 1 launch, [2] = that launch's earliest start,
+ *                     [3] = its end (absolute ns; comparing [2] across
+ *                     ranks shows their arrival skew).  Zero it once.
+ * In the destinations' buffers (rows in rank order, then token order, as the
+ * single-GPU path numbers them): recv_src_idx = t, recv_topk_idx = local
+ * expert id or -1, recv_topk_weights = weight or 0.0.  Rows >= cap are not
+ * written and set EP_STATUS_CAPACITY.
+ */
+EP_API int ep_shard_notify(const int64_t *topk_idx, const float *topk_weights,
+                           const int32_t *counts, const int32_t *expert_counts,
+                           int rank, int num_ranks, int num_tokens, int num_topk,
+                           int num_experts, int expert_alignment, int capacity,
+                           int32_t *const *recv_src_idx_peers,
+                           int64_t *const *recv_topk_idx_peers,
+                           float *const *recv_topk_weights_peers,
+                           int64_t *recv_topk_idx, int32_t *rank_prefix_matrix,
+                           int32_t *recv_count,
+                           int32_t *num_recv_tokens_per_expert,
+                           int32_t *send_pos, unsigned long long *notify_probe,
+                           void *workspace, size_t workspace_bytes,
+                           int32_t *status, cudaStream_t stream);
+
+/*
+ * Rows of one rank of a sharded job: x bf16 [T, H] (H % 8 == 0, 16-byte
+ * aligned); row t goes to row send_pos[t][d] of rank d's bf16 [cap, H]
+ * receive buffer (peer table recv_x_peers), for every d with a position.
+ */
+EP_API int ep_shard_dispatch(const void *x, const int32_t *send_pos,
+                             int num_ranks, int num_tokens, int hidden,
+                             int capacity, void *const *recv_x_peers,
+                             int32_t *status, cudaStream_t stream);
+
+/*
+ * Combine of one rank of a sharded job: combined_x bf16 [T, H] =
+ * bf16_rne(sum over d ascending with send_pos[t][d] >= 0 of
+ * float(y_d[send_pos[t][d]]), + bias_0, + bias_1), y_d rank d's bf16
+ * [cap, H] expert outputs (peer table y_peers); combined_topk_weights fp32
+ * [T, K] (or NULL) the same sum over the peers' recv_topk_weights rows.
+ */
+EP_API int ep_shard_combine(const void *const *y_peers,
+                            const float *const *recv_topk_weights_peers,
+                            const int32_t *send_pos, const void *bias_0,
+                            const void *bias_1, int num_ranks, int num_tokens,
+                            int hidden, int num_topk, int capacity,
+                            void *combined_x, float *combined_topk_weights,
+                            int32_t *status, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

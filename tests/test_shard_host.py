@@ -1,0 +1,100 @@
+"""The sharded path's control plane on CPU ranks (gloo, world size 2 and 4).
+
+Each rank takes its own source rank's layout (the oracle's, on the CPU), and
+the rows every rank all-gathers must be the single-GPU layout's rows in rank
+order: their inclusive prefix over ranks is then the oracle's rank prefix
+matrix, its last row the oracle's receive counts, and the gathered expert
+rows give the oracle's per-expert receive counts of every destination
+(legacy-test analysis page, the inclusive recv_gbl_rank_prefix_sum that
+check_data walks; Python接口 page, num_recv_tokens_per_expert_list).  IPC
+handles come back in rank order and every rank computes the same layout of
+the shared region.
+"""
+import datetime
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _workload(world):
+    from workloads import Workload
+    return Workload("shard_host", R=world, T=300, H=0, E=8 * world, K=4, masked_frac=0.1,
+                    seed=40 + world)
+
+
+def _worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    import oracle
+    from combine_get_dispatch_06_b200.shard import (allgather_rows, exchange_handles,
+                                                    region_layout)
+    from workloads import make
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        w = _workload(world)
+        idx = make(w, with_x=False)["topk_idx"]
+        mine = oracle.layout(idx[rank:rank + 1], w.E, w.R)     # this rank's own tokens
+        counts = allgather_rows(torch.from_numpy(mine["num_tokens_per_rank"][0]))
+        ecounts = allgather_rows(torch.from_numpy(mine["num_tokens_per_expert"][0]))
+        handles = exchange_handles(bytes([rank + 1]) * 64)
+        lay = region_layout(w.R * w.T, 64, w.K, True)
+        q.put((rank, counts.numpy(), ecounts.numpy(), handles,
+               {k: (v if k == "_bytes" else (v[0], v[1], str(v[2]))) for k, v in lay.items()}))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_count_exchange_gives_the_oracle_prefix_matrix(world):
+    sys.path.insert(0, ROOT)
+    import oracle
+    from workloads import make
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict((r[0], r[1:]) for r in (q.get(timeout=240) for _ in procs))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+
+    w = _workload(world)
+    idx = make(w, with_x=False)["topk_idx"]
+    full = oracle.layout(idx, w.E, w.R)
+    pre = oracle.prefix(full["is_token_in_rank"])
+    nrte = oracle.expert_recv_counts(full["num_tokens_per_expert"], w.R)
+    El = w.E // w.R
+    layouts = set()
+    for rank in range(world):
+        counts, ecounts, handles, lay = got[rank]
+        np.testing.assert_array_equal(counts, full["num_tokens_per_rank"])
+        np.testing.assert_array_equal(np.cumsum(counts, axis=0), pre["rank_prefix_matrix"])
+        np.testing.assert_array_equal(np.cumsum(counts, axis=0)[-1], pre["recv_count"])
+        np.testing.assert_array_equal(ecounts, full["num_tokens_per_expert"])
+        for d in range(world):
+            np.testing.assert_array_equal(ecounts[:, d * El:(d + 1) * El].sum(axis=0), nrte[d])
+        assert handles == [bytes([r + 1]) * 64 for r in range(world)]
+        layouts.add(repr(sorted(lay.items())))
+    assert len(layouts) == 1

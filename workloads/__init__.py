@@ -104,30 +104,34 @@ def _draw_topk(rng: np.random.Generator, T: int, E: int, K: int, routing: str,
     raise ValueError(f"unknown routing {routing!r}")
 
 
-def make(w: Workload, *, with_x: bool = True) -> dict:
+def make(w: Workload, *, with_x: bool = True, ranks=None) -> dict:
     """Draw the inputs of workload ``w``.
 
     Returns a dict with ``topk_idx`` int64 [S,T,K], ``topk_weights`` fp32
     [S,T,K] and (if ``with_x`` and H > 0) ``x`` uint16 bf16 bits [S,T,H].
+    ``ranks``: draw only these source ranks (same values as in the full draw,
+    stacked in the order given), e.g. one process's own rank.
     """
     S, T, H, E, K = w.S, w.T, w.H, w.E, w.K
     if K > E:
         raise ValueError("K must not exceed E")
     children = np.random.SeedSequence(w.seed).spawn(S)
-    idx = np.empty((S, T, K), dtype=np.int64)
-    wts = np.empty((S, T, K), dtype=np.float32)
-    x = np.empty((S, T, H), dtype=np.uint16) if (with_x and H > 0) else None
-    for r in range(S):
+    which = list(range(S)) if ranks is None else [int(r) for r in ranks]
+    n = len(which)
+    idx = np.empty((n, T, K), dtype=np.int64)
+    wts = np.empty((n, T, K), dtype=np.float32)
+    x = np.empty((n, T, H), dtype=np.uint16) if (with_x and H > 0) else None
+    for i, r in enumerate(which):
         rng = np.random.Generator(np.random.PCG64(children[r]))
-        idx[r] = _draw_topk(rng, T, E, K, w.routing, w.zipf_s)
+        idx[i] = _draw_topk(rng, T, E, K, w.routing, w.zipf_s)
         if w.masked_frac > 0.0:
             n_mask = int(round(w.masked_frac * T * K))
             flat = rng.choice(T * K, size=n_mask, replace=False)
-            v = idx[r].reshape(-1)
+            v = idx[i].reshape(-1)
             v[flat] = -1
-        wts[r] = softmax_f32(rng.standard_normal((T, K), dtype=np.float32))
+        wts[i] = softmax_f32(rng.standard_normal((T, K), dtype=np.float32))
         if x is not None:
-            x[r] = bf16_bits_from_f32(rng.standard_normal((T, H), dtype=np.float32))
+            x[i] = bf16_bits_from_f32(rng.standard_normal((T, H), dtype=np.float32))
     out = {"topk_idx": idx, "topk_weights": wts}
     if x is not None:
         out["x"] = x
