@@ -739,22 +739,40 @@ def run_sharded(args) -> None:
     N_remote = int(((sp >= 0) & remote[None, :]).sum().item())
     bd, bc = shard_bytes(R, T, H, K, N)
 
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+
+    def timed(run) -> float:
+        barrier(device)
+        torch.cuda.synchronize(device)
+        a.record(stream)
+        for _ in range(args.steps):
+            run()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        return a.elapsed_time(b) / args.steps
+
+    eager_ms = timed(step)
+    # the whole step -- kernels and NCCL collectives -- captured once and
+    # replayed, so that host launch overhead does not pace the GPUs
+    graph, graph_note = None, None
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        torch.cuda.synchronize(device)
+        graph = g
+    except Exception as e:  # capture refused: time the eager step only
+        graph_note = f"capture failed: {type(e).__name__}: {str(e)[:200]}"
+        torch.cuda.synchronize(device)
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    barrier(device)
-    torch.cuda.synchronize(device)
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(args.steps):
-        step()
-    b.record(stream)
-    torch.cuda.synchronize(device)
-    barrier(device)
+    ms_local = timed(graph.replay) if graph is not None else eager_ms
     clocks = sampler.stop()
-    ms_local = a.elapsed_time(b) / args.steps
     agg = aggregate(bd + bc, T, ms_local, device)
+    eager = aggregate(bd + bc, T, eager_ms, device)
     if int(buf.status.item()) != 0:
         raise RuntimeError(f"device status {int(buf.status.item())} in the timed region")
     # rows crossing NVLink per step (each way): copies to other ranks, then read back
@@ -805,10 +823,14 @@ def run_sharded(args) -> None:
         "e2e": {"value": e2e["gbs"], "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": cx_h.numel() * 2, "ms_per_step": e2e["ms_per_step"]},
         "gpu_launches": 6 * args.steps,   # layout, prefix, scan, pad, copy, combine per step
+        "cuda_graph": graph is not None, "cuda_graph_note": graph_note,
+        "eager": {"ms_per_step": eager["ms_per_step"], "value": eager["gbs"]},
         "clocks": clocks,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del graph
+    torch.cuda.synchronize(device)
     buf.close()
     dist.destroy_process_group()
 

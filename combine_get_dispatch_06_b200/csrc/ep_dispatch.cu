@@ -28,6 +28,9 @@ namespace ep {
 namespace {
 
 constexpr int kMaskWords = (kMaxRanks + 31) / 32;
+// Largest tiles x R for which a tile reads every predecessor's counts at once
+// (R must divide the tile); above it, the windowed decoupled look-back.
+constexpr int kFullLookback = 8192;
 
 struct DispatchScanParams {
   const int64_t *topk_idx;
@@ -237,7 +240,57 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   // ---- look-back (a group of 16 lanes per rank column), prefix matrix ----
   const bool publish = (p.flags & EP_DEBUG_SUPPRESS_PUBLISH) == 0;
   const bool last_of_src = (tile % p.tiles_per_src) == p.tiles_per_src - 1;
-  {
+  if (kScanTile % p.R == 0 && static_cast<long>(p.num_tiles) * p.R <= kFullLookback) {
+    // Every tile publishes its counts, and each tile adds up all of its
+    // predecessors' counts at once (thread tid always reads column tid % R,
+    // since R divides the tile): no tile waits for another's inclusive
+    // prefix, only for its counts, which every running tile publishes
+    // before it waits on anything.  Tickets order the tiles, so every
+    // predecessor is running or done.
+    for (int d = tid; d < p.R; d += kScanTile) {
+      s_excl[d] = 0;
+      if (publish) publish_aggregate(p.desc, tile, p.R, d, static_cast<uint32_t>(s_agg[d]));
+    }
+    __syncthreads();
+    const int n = tile * p.R;
+    int acc = 0;
+    bool timed_out = false;
+    constexpr int B = 8;
+    for (int f0 = 0; f0 < n; f0 += kScanTile * B) {
+      uint64_t w[B];
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const int f = f0 + b * kScanTile + tid;
+        w[b] = f < n ? ld_relaxed_gpu(p.desc + f) : (1ull << 32);
+      }
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const int f = f0 + b * kScanTile + tid;
+        if ((w[b] >> 32) == 0 && f < n && !timed_out) {
+          const uint64_t ts = globaltimer();
+          do {
+            __nanosleep(64);
+            w[b] = ld_relaxed_gpu(p.desc + f);
+            if ((w[b] >> 32) != 0) break;
+            if (globaltimer() - ts > p.timeout_ns) timed_out = true;
+          } while (!timed_out);
+        }
+        if ((w[b] >> 32) != 0) acc += static_cast<int>(static_cast<uint32_t>(w[b]));
+      }
+    }
+    if (timed_out) report(p.status, EP_STATUS_WAIT_TIMEOUT);
+    if (acc != 0) atomicAdd(&s_excl[tid % p.R], acc);
+    __syncthreads();
+    for (int d = tid; d < p.R; d += kScanTile) {
+      const int excl = s_excl[d];
+      const int run = s_agg[d];
+      if (last_of_src && p.P != nullptr) {
+        p.P[static_cast<size_t>(s) * p.R + d] = excl + run;
+        if (tile == p.num_tiles - 1) p.recv_count[d] = excl + run;
+      }
+      s_excl[d] = excl + (p.dst_base != nullptr ? p.dst_base[d] : 0);
+    }
+  } else {
     constexpr int G = 16;
     const int grp = tid / G;
     for (int d = grp; d < p.R; d += kScanTile / G) {
