@@ -33,6 +33,10 @@
 namespace ep {
 namespace {
 
+// Largest tiles x E for which a tile reads every predecessor's counts at once;
+// above it, the windowed decoupled look-back.
+constexpr int kLLFullLookback = 16384;
+
 struct LLScanParams {
   const int64_t *topk_idx;
   const int32_t *mask;   // [R], non-zero = failed rank; nullptr = none
@@ -72,12 +76,26 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
   const int lane = tid & 31;
   const int warp = tid >> 5;
   if (tid == 0) s_tile = static_cast<int>(atomicAdd(&p.head->ticket, 1u));
+  // Tiles are usually handed out in block order: the ids of tile blockIdx.x
+  // are loaded while the ticket is on its way, and loaded again in the rare
+  // case the ticket names another tile.
+  auto load_ids = [&](int tl, int64_t (&ids)[MAXK]) {
+    const int s_ = tl / p.tiles_per_src;
+    const int t_ = (tl % p.tiles_per_src) * kScanTile + tid;
+    const size_t st_ = static_cast<size_t>(s_) * p.T + t_;
+#pragma unroll
+    for (int k = 0; k < MAXK; ++k)
+      ids[k] = (t_ < p.T && k < p.K) ? p.topk_idx[st_ * p.K + k] : -1;
+  };
+  int64_t ids[MAXK];
+  load_ids(static_cast<int>(blockIdx.x), ids);
   for (int i = tid; i < kScanWarps * kMaxExperts; i += kScanTile) (&s_lanes[0][0])[i] = 0u;
   if (p.mask != nullptr)
     for (int i = tid; i < p.R; i += kScanTile) s_mask[i] = p.mask[i];
   __syncthreads();
 
   const int tile = s_tile;
+  if (tile != static_cast<int>(blockIdx.x)) load_ids(tile, ids);
   const int s = tile / p.tiles_per_src;
   const int t = (tile % p.tiles_per_src) * kScanTile + tid;
   const bool valid = t < p.T;
@@ -96,7 +114,7 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
     col[k] = -1;
     rnk[k] = 0;
     if (valid && k < p.K) {
-      const int64_t e = p.topk_idx[st * p.K + k];
+      const int64_t e = ids[k];
       if (e >= 0 && e < p.E) {
         if (!src_ok || (p.mask != nullptr && s_mask[static_cast<int>(e) / p.El] != 0)) continue;
         ev[k] = static_cast<int>(e);
@@ -157,13 +175,60 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
       if (publish) publish_aggregate(p.desc, tile, p.E, c, static_cast<uint32_t>(run));
     }
   }
+  uint32_t excls[kCols];
+  if (static_cast<long>(p.num_tiles) * p.E <= kLLFullLookback) {
+    // every predecessor's count of every column this thread owns, all loads
+    // issued before any is waited for (no tile waits for another's
+    // inclusive prefix, only for its counts, published above before any wait)
+#pragma unroll
+    for (int i = 0; i < kCols; ++i) excls[i] = 0u;
+    bool timed_out = false;
+    constexpr int B = 8;
+    for (int j0 = 0; j0 < tile; j0 += B) {
+      uint64_t w[B][kCols];
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+#pragma unroll
+        for (int i = 0; i < kCols; ++i) {
+          const int c = tid + i * kScanTile;
+          w[b][i] = (j0 + b < tile && c < p.E)
+                        ? ld_relaxed_gpu(p.desc + static_cast<size_t>(j0 + b) * p.E + c)
+                        : (1ull << 32);
+        }
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+#pragma unroll
+        for (int i = 0; i < kCols; ++i) {
+          const int c = tid + i * kScanTile;
+          if ((w[b][i] >> 32) == 0 && !timed_out) {  // not published yet: read again (bounded)
+            const uint64_t ts = globaltimer();
+            do {
+              __nanosleep(64);
+              w[b][i] = ld_relaxed_gpu(p.desc + static_cast<size_t>(j0 + b) * p.E + c);
+              if ((w[b][i] >> 32) != 0) break;
+              if (globaltimer() - ts > p.timeout_ns) timed_out = true;
+            } while (!timed_out);
+          }
+          if ((w[b][i] >> 32) != 0) excls[i] += static_cast<uint32_t>(w[b][i]);
+        }
+    }
+    if (timed_out) report(p.status, EP_STATUS_WAIT_TIMEOUT);
+  } else {
+#pragma unroll
+    for (int i = 0; i < kCols; ++i) {
+      const int c = tid + i * kScanTile;
+      excls[i] = c < p.E ? lookback_window<1, 32>(p.desc, tile, p.E, c,
+                                                  static_cast<uint32_t>(runs[i]), publish,
+                                                  p.timeout_ns, p.status, true)
+                         : 0u;
+    }
+  }
 #pragma unroll
   for (int i = 0; i < kCols; ++i) {
     const int c = tid + i * kScanTile;
     if (c >= p.E) break;
     const int run = runs[i];
-    const uint32_t excl = lookback_window<1, 32>(p.desc, tile, p.E, c, static_cast<uint32_t>(run),
-                                                 publish, p.timeout_ns, p.status, true);
+    const uint32_t excl = excls[i];
     s_excl[c] = static_cast<int>(excl);
     const size_t o = (static_cast<size_t>(c) * p.R + s) * 2;
     if (first_of_src) p.layout_range[o] = static_cast<int>(excl);
