@@ -264,6 +264,24 @@ __device__ __forceinline__ void st_stream_v4(void *p, uint4 v) {
                : "memory");
 }
 
+// 32-byte stores (one whole L2 sector per thread; address 32-byte aligned).
+__device__ __forceinline__ void st_v4_b64(void *p, int64_t a, int64_t b, int64_t c, int64_t d) {
+  asm volatile("st.global.v4.b64 [%0], {%1, %2, %3, %4};" ::"l"(p), "l"(a), "l"(b), "l"(c),
+               "l"(d)
+               : "memory");
+}
+
+template <typename T>
+__device__ __forceinline__ void st_v8_b32(void *p, const T (&v)[8]) {
+  static_assert(sizeof(T) == 4, "32-bit elements");
+  uint32_t u[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) u[j] = __builtin_bit_cast(uint32_t, v[j]);
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(u[0]),
+               "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7])
+               : "memory");
+}
+
 // bf16 pair (packed in a u32, element 0 in the low half) -> two floats.
 __device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }

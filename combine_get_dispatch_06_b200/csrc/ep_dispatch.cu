@@ -60,6 +60,7 @@ struct DispatchScanParams {
   // start in the workspace; cumulative [ns, launches, last start, last end].
   unsigned long long *probe_state;
   unsigned long long *probe;
+  int idx32, w32, sp32;  // 32-byte stores of received ids / weights / send_pos rows
   ScanHeader *head;
   int32_t *expert_cnt;   // [E] all sources, then [R][E] per source
   uint64_t *desc;
@@ -75,10 +76,19 @@ struct DispatchScanParams {
 template <int MAXK>
 __device__ __forceinline__ void write_meta(int64_t *idx_row, float *w_row, int K, int d,
                                            const int (&dk)[MAXK], const int (&lk)[MAXK],
-                                           const float (&wk)[MAXK]) {
+                                           const float (&wk)[MAXK], bool idx32, bool w32) {
   if (idx_row != nullptr) {
     int64_t *dst = idx_row;
-    if ((K & 1) == 0) {
+    if (idx32) {  // K % 4 == 0, rows 32-byte aligned: one whole sector per store
+#pragma unroll
+      for (int k = 0; k < MAXK; k += 4) {
+        if (k < K)
+          st_v4_b64(dst + k, dk[k] == d ? static_cast<int64_t>(lk[k]) : -1ll,
+                    dk[k + 1] == d ? static_cast<int64_t>(lk[k + 1]) : -1ll,
+                    dk[k + 2] == d ? static_cast<int64_t>(lk[k + 2]) : -1ll,
+                    dk[k + 3] == d ? static_cast<int64_t>(lk[k + 3]) : -1ll);
+      }
+    } else if ((K & 1) == 0) {
 #pragma unroll
       for (int k = 0; k < MAXK; k += 2) {
         if (k < K) {
@@ -96,7 +106,17 @@ __device__ __forceinline__ void write_meta(int64_t *idx_row, float *w_row, int K
   }
   if (w_row != nullptr) {
     float *dst = w_row;
-    if ((K & 3) == 0) {
+    if (w32) {  // K % 8 == 0, rows 32-byte aligned
+#pragma unroll
+      for (int k = 0; k < MAXK; k += 8) {
+        if (k < K) {
+          float v[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = dk[k + j] == d ? wk[k + j] : 0.f;
+          st_v8_b32(dst + k, v);
+        }
+      }
+    } else if ((K & 3) == 0) {
 #pragma unroll
       for (int k = 0; k < MAXK; k += 4) {
         if (k < K) {
@@ -311,6 +331,9 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   // ---- pass 2: positions, handle and received metadata -------------------
   const uint32_t lt = lanemask_lt();
   bool overflow = false;
+  int32_t spq[8];  // send positions of the current group of 8 destinations
+#pragma unroll
+  for (int j = 0; j < 8; ++j) spq[j] = -1;
   for (int d0 = 0; d0 < p.R; d0 += 32) {
     const uint32_t word = my_mask[d0 >> 5];
     const int nb = min(32, p.R - d0);
@@ -320,7 +343,13 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
       const uint32_t bal = __ballot_sync(0xffffffffu, has);
       if (!valid) continue;
       const int pos = has ? s_excl[d] + s_woff[warp][d] + __popc(bal & lt) : -1;
-      p.send_pos[st * p.R + d] = pos;
+      if (p.sp32) {  // R % 8 == 0, rows 32-byte aligned: a whole sector per 8 ranks
+#pragma unroll
+        for (int j = 0; j < 8; ++j) spq[j] = (b & 7) == j ? pos : spq[j];
+        if ((b & 7) == 7) st_v8_b32(p.send_pos + st * p.R + d - 7, spq);
+      } else {
+        p.send_pos[st * p.R + d] = pos;
+      }
       if (!has) continue;
       if (pos < 0 || pos >= p.cap) {  // pos < 0 only after a timed-out look-back
         overflow = true;
@@ -332,13 +361,14 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
           write_meta(p.ridx_tab != nullptr ? p.ridx_tab[d] + static_cast<size_t>(pos) * p.K
                                            : nullptr,
                      p.rw_tab != nullptr ? p.rw_tab[d] + static_cast<size_t>(pos) * p.K : nullptr,
-                     p.K, d, dk, lk, wk);
+                     p.K, d, dk, lk, wk, p.idx32 != 0, p.w32 != 0);
       } else {
         const size_t row = static_cast<size_t>(d) * p.cap + pos;
         p.recv_src_idx[row] = t;
         if (meta)
           write_meta(p.recv_idx != nullptr ? p.recv_idx + row * p.K : nullptr,
-                     p.recv_w != nullptr ? p.recv_w + row * p.K : nullptr, p.K, d, dk, lk, wk);
+                     p.recv_w != nullptr ? p.recv_w + row * p.K : nullptr, p.K, d, dk, lk, wk,
+                     p.idx32 != 0, p.w32 != 0);
       }
     }
   }
@@ -734,6 +764,15 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// 32-byte stores need rows that are whole multiples of 32 bytes and a
+// 32-byte-aligned base (peer buffers are allocation-aligned).
+void set_store_widths(DispatchScanParams &p) {
+  auto al32 = [](const void *q) { return (reinterpret_cast<uintptr_t>(q) & 31u) == 0; };
+  p.idx32 = (p.K % 4 == 0) && (p.ridx_tab != nullptr || (p.recv_idx != nullptr && al32(p.recv_idx)));
+  p.w32 = (p.K % 8 == 0) && (p.rw_tab != nullptr || (p.recv_w != nullptr && al32(p.recv_w)));
+  p.sp32 = (p.R % 8 == 0) && al32(p.send_pos);
+}
+
 // A2 (+ received metadata): the scan kernel.  Arguments already checked.
 int notify_impl(const int64_t *topk_idx, const float *topk_weights,
                 const uint8_t *is_token_in_rank, int R, int T, int K, int E, int align, int cap,
@@ -809,6 +848,7 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   const WaitConfig wc = wait_config();
   p.timeout_ns = wc.timeout_ns;
   p.flags = wc.flags;
+  set_store_widths(p);
   cudaError_t launched;
   if (topk_idx != nullptr && K > 8)
     launched = launch_pdl(dispatch_scan_kernel<16>,
@@ -1217,6 +1257,7 @@ extern "C" EP_API int ep_shard_notify(
     const WaitConfig wc = wait_config();
     p.timeout_ns = wc.timeout_ns;
     p.flags = wc.flags;
+    set_store_widths(p);
     if (K > 8)
       launched = launch_pdl(dispatch_scan_kernel<16>, dim3(tiles), dim3(kScanTile), 0, stream, p);
     else
