@@ -98,3 +98,44 @@ def test_count_exchange_gives_the_oracle_prefix_matrix(world):
         assert handles == [bytes([r + 1]) * 64 for r in range(world)]
         layouts.add(repr(sorted(lay.items())))
     assert len(layouts) == 1
+
+
+def _dying_worker(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import time
+
+    import torch.distributed as dist
+
+    from combine_get_dispatch_06_b200.shard import allgather_rows
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        os._exit(3)  # this rank fails between steps, before the notify exchange
+    t0 = time.monotonic()
+    try:
+        allgather_rows(torch.zeros(world, dtype=torch.int32))
+        q.put((rank, "completed", time.monotonic() - t0))
+    except Exception as e:  # the survivor learns of it from its collective
+        q.put((rank, type(e).__name__, time.monotonic() - t0))
+    os._exit(0)
+
+
+def test_a_rank_that_dies_before_the_notify_exchange_is_detected():
+    """Failure detection on the host: a rank exits between steps; the other
+    rank's count exchange ends with an error within the process group's
+    timeout instead of waiting for ever (no GPU is involved)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dying_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    rank, outcome, seconds = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+    assert rank == 0
+    assert outcome != "completed"
+    assert seconds < 60
+    assert procs[1].exitcode == 3
