@@ -132,6 +132,23 @@ __device__ __forceinline__ int32_t ld_relaxed_gpu(const int32_t *p) {
   return v;
 }
 
+// four consecutive 32-bit words (16-byte aligned) with one relaxed store
+__device__ __forceinline__ void st_relaxed_gpu_v4(int32_t *p, int a, int b, int c, int d) {
+  asm volatile("st.relaxed.gpu.global.v4.s32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b),
+               "r"(c), "r"(d)
+               : "memory");
+}
+
+// four consecutive 32-bit words (16-byte aligned) with one relaxed load
+__device__ __forceinline__ uint4 ld_relaxed_gpu_v4(const uint32_t *p) {
+  uint4 v;
+  asm volatile("ld.relaxed.gpu.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));

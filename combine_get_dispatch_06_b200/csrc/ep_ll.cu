@@ -56,23 +56,40 @@ struct LLScanParams {
 
 // MAXK: compile-time bound on the top-k slots (8 or 16), chosen per call.
 //
+// Threads 0..kScanTile-1 hold one token each; the other kScanTile threads
+// run the look-back.  As soon as its ids are read, every token thread sets
+// its lane's bit in the word of each of its experts (one word per warp and
+// expert, shared atomicOr): the popcounts of those words are the tile's rows
+// per expert, which the look-back warps publish at once, and a token's rank
+// among the warp's tokens with the same expert is the number of lower lanes
+// in the word -- token order, whatever slot the expert is in.  Up to
+// kLLFullLookback tiles x experts, a tile reads every predecessor's count of
+// every expert in one pass (32-bit words, count + 1, 0 = not yet published;
+// four experts per 16-byte load where E % 4 == 0; a batch of loads that
+// found words not yet published is read again as a whole); above it, the
+// windowed decoupled look-back on 64-bit descriptors.
+//
 // The dispatch kernel that follows runs concurrently with this one: it is
 // scheduled once every tile has passed pdl_trigger(), which comes after
 // pdl_wait(), so everything before this kernel in the stream is complete by
 // then.  It takes each token's slab rows from a mirror of ll_pos in the
 // workspace, zeroed before this kernel and written here as ll_pos + 2, so
 // that a non-zero word is its own proof of being written.
+constexpr int kLLScanThreads = 2 * kScanTile;
+
 template <int MAXK>
-__global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
+__global__ void __launch_bounds__(kLLScanThreads, 2) ll_scan_kernel(LLScanParams p) {
   pdl_wait();
   pdl_trigger();  // after the wait: see above
   __shared__ int s_tile;
   __shared__ uint32_t s_lanes[kScanWarps][kMaxExperts];  // lanes of the warp holding expert c
-  __shared__ int s_whist[kScanWarps][kMaxExperts];
-  __shared__ int s_excl[kMaxExperts];
+  __shared__ int s_whist[kScanWarps][kMaxExperts];       // rows of expert c in earlier warps
+  __shared__ int s_cnt[kMaxExperts];                     // the tile's rows of expert c
+  __shared__ int s_excl[kMaxExperts];                    // rows of expert c in earlier tiles
   __shared__ int s_mask[kMaxRanks];  // failed ranks (non-zero), if a mask is given
 
   const int tid = threadIdx.x;
+  const bool tok = tid < kScanTile;  // a token thread (warps 0..kScanWarps-1)
   const int lane = tid & 31;
   const int warp = tid >> 5;
   if (tid == 0) s_tile = static_cast<int>(atomicAdd(&p.head->ticket, 1u));
@@ -88,17 +105,21 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
       ids[k] = (t_ < p.T && k < p.K) ? p.topk_idx[st_ * p.K + k] : -1;
   };
   int64_t ids[MAXK];
-  load_ids(static_cast<int>(blockIdx.x), ids);
-  for (int i = tid; i < kScanWarps * kMaxExperts; i += kScanTile) (&s_lanes[0][0])[i] = 0u;
+  if (tok) load_ids(static_cast<int>(blockIdx.x), ids);
+  for (int i = tid; i < kScanWarps * kMaxExperts; i += kLLScanThreads) (&s_lanes[0][0])[i] = 0u;
+  for (int i = tid; i < p.E; i += kLLScanThreads) {
+    s_cnt[i] = 0;
+    s_excl[i] = 0;
+  }
   if (p.mask != nullptr)
-    for (int i = tid; i < p.R; i += kScanTile) s_mask[i] = p.mask[i];
+    for (int i = tid; i < p.R; i += kLLScanThreads) s_mask[i] = p.mask[i];
   __syncthreads();
 
   const int tile = s_tile;
-  if (tile != static_cast<int>(blockIdx.x)) load_ids(tile, ids);
+  if (tok && tile != static_cast<int>(blockIdx.x)) load_ids(tile, ids);
   const int s = tile / p.tiles_per_src;
   const int t = (tile % p.tiles_per_src) * kScanTile + tid;
-  const bool valid = t < p.T;
+  const bool valid = tok && t < p.T;
   const size_t st = static_cast<size_t>(s) * p.T + t;
   // a failed (masked) source rank sends nothing
   const bool src_ok = p.mask == nullptr || s_mask[s] == 0;
@@ -121,127 +142,131 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
         bool dup = false;
 #pragma unroll
         for (int k2 = 0; k2 < k; ++k2) dup |= (col[k2] == ev[k]);
-        if (!dup) col[k] = ev[k];
+        if (!dup) {
+          col[k] = ev[k];
+          atomicOr(&s_lanes[warp][ev[k]], 1u << lane);
+        }
       } else if (e != -1) {
         bad = true;
       }
     }
   }
   if (bad) report(p.status, EP_STATUS_BAD_EXPERT);
-
-  // For every expert, the set of the warp's lanes (tokens) that hold it:
-  // slot by slot, lanes with the same expert find each other with match.any
-  // and their lowest lane ORs the group into the expert's word.  A token's
-  // rank among the warp's tokens with that expert is then the number of
-  // lower lanes in the word -- token order, whatever slot the expert is in.
-#pragma unroll
-  for (int k = 0; k < MAXK; ++k) {
-    if (k < p.K) {
-      const uint32_t peers = __match_any_sync(0xffffffffu, col[k]);
-      if (col[k] >= 0 && lane == __ffs(peers) - 1) s_lanes[warp][col[k]] |= peers;
-      __syncwarp();
-    }
-  }
-  const uint32_t lt = lanemask_lt();
-#pragma unroll
-  for (int k = 0; k < MAXK; ++k)
-    if (col[k] >= 0) rnk[k] = __popc(s_lanes[warp][col[k]] & lt);
-  __syncthreads();  // every warp's lane masks are complete before they are counted
-  for (int c = tid; c < p.E; c += kScanTile)
-#pragma unroll
-    for (int w = 0; w < kScanWarps; ++w) s_whist[w][c] = __popc(s_lanes[w][c]);
-  __syncthreads();
+  __syncthreads();  // every warp's lane words are complete
 
   const bool publish = (p.flags & EP_DEBUG_SUPPRESS_PUBLISH) == 0;
-  const bool first_of_src = (tile % p.tiles_per_src) == 0;
-  // The tile's count of every column is published before any column looks
-  // back, so no tile waits for a predecessor that is still busy with its
-  // other columns.
-  constexpr int kCols = kMaxExperts / kScanTile;
-  int runs[kCols];
+  const bool full = static_cast<long>(p.num_tiles) * p.E <= kLLFullLookback;
+  if (!tok) {
+    // ---- look-back warps: publish the tile's counts, then sum the earlier tiles'
+    const int lt = tid - kScanTile;
+    uint32_t *cnt32 = reinterpret_cast<uint32_t *>(p.desc);  // [num_tiles][E]: rows + 1
+    for (int c = lt; c < p.E; c += kScanTile) {
+      int n = 0;
 #pragma unroll
-  for (int i = 0; i < kCols; ++i) {
-    const int c = tid + i * kScanTile;
-    runs[i] = 0;
-    if (c < p.E) {
+      for (int w = 0; w < kScanWarps; ++w) n += __popc(s_lanes[w][c]);
+      s_cnt[c] = n;
+      if (!publish) continue;
+      if (full)
+        st_relaxed_gpu(reinterpret_cast<int32_t *>(cnt32) + static_cast<size_t>(tile) * p.E + c,
+                       n + 1);
+      else
+        publish_aggregate(p.desc, tile, p.E, c, static_cast<uint32_t>(n));
+    }
+    if (full) {
+      // item i = (predecessor j, group g of cw experts), i = j * G + g; this
+      // thread takes i = lt, lt + kScanTile, ... with kB loads in flight,
+      // and keeps the sums of one group in registers until the group changes
+      const int cw = (p.E & 3) == 0 ? 4 : 1;
+      const int G = p.E / cw;
+      const int items = tile * G;
+      constexpr int kB = 16;
+      uint32_t acc[4] = {0u, 0u, 0u, 0u};
+      int cur = -1;
+      bool timed_out = false;
+      auto flush = [&]() {
+        if (cur < 0) return;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (q < cw && acc[q] != 0u) atomicAdd(&s_excl[cur * cw + q], static_cast<int>(acc[q]));
+      };
+      auto load_item = [&](int i) -> uint4 {
+        const int j = i / G, g = i - j * G;
+        const uint32_t *a = cnt32 + static_cast<size_t>(j) * p.E + g * cw;
+        if (cw == 4) return ld_relaxed_gpu_v4(a);
+        return make_uint4(static_cast<uint32_t>(ld_relaxed_gpu(reinterpret_cast<const int32_t *>(a))),
+                          1u, 1u, 1u);
+      };
+      auto unpublished = [](const uint4 &w) {
+        return w.x == 0u || w.y == 0u || w.z == 0u || w.w == 0u;
+      };
+      for (int i0 = lt; i0 < items; i0 += kScanTile * kB) {
+        uint4 v[kB];
+        uint32_t pend = 0u;  // loads of this batch that found a word not yet published
+#pragma unroll
+        for (int b = 0; b < kB; ++b) {
+          const int i = i0 + b * kScanTile;
+          v[b] = i < items ? load_item(i) : make_uint4(1u, 1u, 1u, 1u);
+        }
+#pragma unroll
+        for (int b = 0; b < kB; ++b)
+          if (unpublished(v[b])) pend |= 1u << b;
+        if (pend != 0u && !timed_out) {
+          // read them again, all at once, until every word is there (bounded)
+          const uint64_t ts = globaltimer();
+          do {
+            __nanosleep(64);
+#pragma unroll
+            for (int b = 0; b < kB; ++b)
+              if ((pend >> b) & 1u) v[b] = load_item(i0 + b * kScanTile);
+#pragma unroll
+            for (int b = 0; b < kB; ++b)
+              if (((pend >> b) & 1u) && !unpublished(v[b])) pend &= ~(1u << b);
+            if (pend != 0u && globaltimer() - ts > p.timeout_ns) timed_out = true;
+          } while (pend != 0u && !timed_out);
+        }
+#pragma unroll
+        for (int b = 0; b < kB; ++b) {
+          const int i = i0 + b * kScanTile;
+          if (i >= items) break;
+          const int g = i % G;
+          if (g != cur) {
+            flush();
+            cur = g;
+            acc[0] = acc[1] = acc[2] = acc[3] = 0u;
+          }
+          acc[0] += v[b].x != 0u ? v[b].x - 1u : 0u;
+          acc[1] += v[b].y != 0u ? v[b].y - 1u : 0u;
+          acc[2] += v[b].z != 0u ? v[b].z - 1u : 0u;
+          acc[3] += v[b].w != 0u ? v[b].w - 1u : 0u;
+        }
+      }
+      flush();
+      if (timed_out) report(p.status, EP_STATUS_WAIT_TIMEOUT);
+    } else {
+      for (int c = lt; c < p.E; c += kScanTile)
+        s_excl[c] = static_cast<int>(lookback_window<1, 32>(p.desc, tile, p.E, c,
+                                                             static_cast<uint32_t>(s_cnt[c]),
+                                                             publish, p.timeout_ns, p.status,
+                                                             true));
+    }
+  } else {
+    // ---- token warps: each token's rank among the warp's tokens with its
+    // expert, and every expert's rows in the tile's earlier warps
+    const uint32_t lt = lanemask_lt();
+#pragma unroll
+    for (int k = 0; k < MAXK; ++k)
+      if (col[k] >= 0) rnk[k] = __popc(s_lanes[warp][col[k]] & lt);
+    for (int c = tid; c < p.E; c += kScanTile) {
       int run = 0;
 #pragma unroll
       for (int w = 0; w < kScanWarps; ++w) {
-        const int n = s_whist[w][c];
+        const int n = __popc(s_lanes[w][c]);
         s_whist[w][c] = run;
         run += n;
       }
-      runs[i] = run;
-      if (publish) publish_aggregate(p.desc, tile, p.E, c, static_cast<uint32_t>(run));
     }
   }
-  uint32_t excls[kCols];
-  if (static_cast<long>(p.num_tiles) * p.E <= kLLFullLookback) {
-    // every predecessor's count of every column this thread owns, all loads
-    // issued before any is waited for (no tile waits for another's
-    // inclusive prefix, only for its counts, published above before any wait)
-#pragma unroll
-    for (int i = 0; i < kCols; ++i) excls[i] = 0u;
-    bool timed_out = false;
-    constexpr int B = 8;
-    for (int j0 = 0; j0 < tile; j0 += B) {
-      uint64_t w[B][kCols];
-#pragma unroll
-      for (int b = 0; b < B; ++b)
-#pragma unroll
-        for (int i = 0; i < kCols; ++i) {
-          const int c = tid + i * kScanTile;
-          w[b][i] = (j0 + b < tile && c < p.E)
-                        ? ld_relaxed_gpu(p.desc + static_cast<size_t>(j0 + b) * p.E + c)
-                        : (1ull << 32);
-        }
-#pragma unroll
-      for (int b = 0; b < B; ++b)
-#pragma unroll
-        for (int i = 0; i < kCols; ++i) {
-          const int c = tid + i * kScanTile;
-          if ((w[b][i] >> 32) == 0 && !timed_out) {  // not published yet: read again (bounded)
-            const uint64_t ts = globaltimer();
-            do {
-              __nanosleep(64);
-              w[b][i] = ld_relaxed_gpu(p.desc + static_cast<size_t>(j0 + b) * p.E + c);
-              if ((w[b][i] >> 32) != 0) break;
-              if (globaltimer() - ts > p.timeout_ns) timed_out = true;
-            } while (!timed_out);
-          }
-          if ((w[b][i] >> 32) != 0) excls[i] += static_cast<uint32_t>(w[b][i]);
-        }
-    }
-    if (timed_out) report(p.status, EP_STATUS_WAIT_TIMEOUT);
-  } else {
-#pragma unroll
-    for (int i = 0; i < kCols; ++i) {
-      const int c = tid + i * kScanTile;
-      excls[i] = c < p.E ? lookback_window<1, 32>(p.desc, tile, p.E, c,
-                                                  static_cast<uint32_t>(runs[i]), publish,
-                                                  p.timeout_ns, p.status, true)
-                         : 0u;
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < kCols; ++i) {
-    const int c = tid + i * kScanTile;
-    if (c >= p.E) break;
-    const int run = runs[i];
-    const uint32_t excl = excls[i];
-    s_excl[c] = static_cast<int>(excl);
-    const size_t o = (static_cast<size_t>(c) * p.R + s) * 2;
-    if (first_of_src) p.layout_range[o] = static_cast<int>(excl);
-    // rows source s owns: its only tile stores the count; several tiles add
-    // theirs (zeroed on the host)
-    if (p.tiles_per_src == 1)
-      p.layout_range[o + 1] = run;
-    else if (run != 0)
-      atomicAdd(&p.layout_range[o + 1], run);
-    if (run != 0 && p.stats != nullptr) atomicAdd(&p.stats[c], run);
-    if (tile == p.num_tiles - 1) p.recv_count[c] = static_cast<int>(excl) + run;
-  }
-  __syncthreads();
+  __syncthreads();  // s_excl and s_whist are complete
 
   if (valid) {
     int pos[MAXK];
@@ -250,31 +275,73 @@ __global__ void __launch_bounds__(kScanTile) ll_scan_kernel(LLScanParams p) {
     for (int k = 0; k < MAXK; ++k) {
       pos[k] = -1;
       if (col[k] >= 0) {
-        const int c = col[k];
-        const int r = s_excl[c] + s_whist[warp][c] + rnk[k];
-        if (r >= 0 && r < p.cap) {
+        const int r = s_excl[col[k]] + s_whist[warp][col[k]] + rnk[k];
+        if (r >= 0 && r < p.cap)
           pos[k] = r;
-          p.recv_src_info[static_cast<size_t>(c) * p.cap + r] = t;
-        } else {
+        else
           oob = true;  // only reachable after a timed-out look-back
-        }
       }
     }
+    // a repeated expert's slot takes the row of its first slot
+    int v[MAXK];
 #pragma unroll
     for (int k = 0; k < MAXK; ++k) {
-      if (k >= p.K) break;
-      int v = pos[k];
+      v[k] = pos[k];
       if (col[k] < 0 && ev[k] >= 0) {
 #pragma unroll
         for (int k2 = 0; k2 < MAXK; ++k2)
-          if (k2 < k && col[k2] == ev[k]) v = pos[k2];
+          if (k2 < k && col[k2] == ev[k]) v[k] = pos[k2];
       }
-      p.ll_pos[st * p.K + k] = v;
-      st_relaxed_gpu(p.pos_mirror + st * p.K + k, v + 2);
     }
+    // the mirror first (the dispatch kernel waits on it), then ll_pos and
+    // recv_src_info; 16 bytes per store where K % 4 == 0 and the row allows
+    int32_t *mrow = p.pos_mirror + st * p.K;
+    int32_t *prow = p.ll_pos + st * p.K;
+    const bool v4m = (p.K & 3) == 0 && (reinterpret_cast<uintptr_t>(mrow) & 15u) == 0;
+    const bool v4p = (p.K & 3) == 0 && (reinterpret_cast<uintptr_t>(prow) & 15u) == 0;
+#pragma unroll
+    for (int k = 0; k < MAXK; k += 4) {
+      if (k >= p.K) break;
+      if (v4m) {
+        st_relaxed_gpu_v4(mrow + k, v[k] + 2, v[k + 1] + 2, v[k + 2] + 2, v[k + 3] + 2);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (k + q < p.K) st_relaxed_gpu(mrow + k + q, v[k + q] + 2);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < MAXK; k += 4) {
+      if (k >= p.K) break;
+      if (v4p) {
+        *reinterpret_cast<int4 *>(prow + k) = make_int4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (k + q < p.K) prow[k + q] = v[k + q];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < MAXK; ++k)
+      if (pos[k] >= 0) p.recv_src_info[static_cast<size_t>(col[k]) * p.cap + pos[k]] = t;
     if (oob) report(p.status, EP_STATUS_BAD_POSITION);
   }
 
+  const bool first_of_src = (tile % p.tiles_per_src) == 0;
+  for (int c = tid; c < p.E; c += kLLScanThreads) {
+    const int run = s_cnt[c];
+    const int excl = s_excl[c];
+    const size_t o = (static_cast<size_t>(c) * p.R + s) * 2;
+    if (first_of_src) p.layout_range[o] = excl;
+    // rows source s owns: its only tile stores the count; several tiles add
+    // theirs (zeroed on the host)
+    if (p.tiles_per_src == 1)
+      p.layout_range[o + 1] = run;
+    else if (run != 0)
+      atomicAdd(&p.layout_range[o + 1], run);
+    if (run != 0 && p.stats != nullptr) atomicAdd(&p.stats[c], run);
+    if (tile == p.num_tiles - 1) p.recv_count[c] = excl + run;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -641,8 +708,9 @@ namespace ep {
 namespace {
 // LL workspace: scan header, descriptors [tiles][E] (64-bit), then the
 // position mirror [R*T][K] int32 (room for K up to kMaxTopk).
-size_t ll_mirror_offset(long tiles, int E) {
-  return sizeof(ScanHeader) + static_cast<size_t>(tiles) * E * sizeof(uint64_t);
+size_t ll_mirror_offset(long tiles, int E) {  // 16-byte aligned
+  return (sizeof(ScanHeader) + static_cast<size_t>(tiles) * E * sizeof(uint64_t) + 15) &
+         ~static_cast<size_t>(15);
 }
 }  // namespace
 }  // namespace ep
@@ -738,11 +806,11 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   cudaError_t launched;
   if (K > 8)
     launched = launch_pdl(ll_scan_kernel<16>,
-        dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
+        dim3(static_cast<unsigned>(num_tiles)), dim3(kLLScanThreads), 0, stream,
         p);
   else
     launched = launch_pdl(ll_scan_kernel<8>,
-        dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
+        dim3(static_cast<unsigned>(num_tiles)), dim3(kLLScanThreads), 0, stream,
         p);
   if (launch_status(launched) != EP_OK) return EP_ERR_CUDA;
 
