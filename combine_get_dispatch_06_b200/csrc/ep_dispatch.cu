@@ -262,44 +262,78 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   const bool last_of_src = (tile % p.tiles_per_src) == p.tiles_per_src - 1;
   if (kScanTile % p.R == 0 && static_cast<long>(p.num_tiles) * p.R <= kFullLookback) {
     // Every tile publishes its counts, and each tile adds up all of its
-    // predecessors' counts at once (thread tid always reads column tid % R,
-    // since R divides the tile): no tile waits for another's inclusive
+    // predecessors' counts at once: no tile waits for another's inclusive
     // prefix, only for its counts, which every running tile publishes
     // before it waits on anything.  Tickets order the tiles, so every
-    // predecessor is running or done.
+    // predecessor is running or done.  Counts are 32-bit words (count + 1,
+    // 0 = not yet published), [tile][R] flat; thread tid reads the groups
+    // of four words 4 * tid + 512 * m, so (R dividing the tile and hence
+    // 512) its word q always belongs to column (4 * tid + q) % R.  A batch
+    // that found words not yet published is read again as a whole.
+    uint32_t *cnt32 = reinterpret_cast<uint32_t *>(p.desc);
     for (int d = tid; d < p.R; d += kScanTile) {
       s_excl[d] = 0;
-      if (publish) publish_aggregate(p.desc, tile, p.R, d, static_cast<uint32_t>(s_agg[d]));
+      if (publish)
+        st_relaxed_gpu(reinterpret_cast<int32_t *>(cnt32) + static_cast<size_t>(tile) * p.R + d,
+                       s_agg[d] + 1);
     }
     __syncthreads();
     const int n = tile * p.R;
-    int acc = 0;
+    const int ngroups = (n + 3) >> 2;
+    const bool vec = (reinterpret_cast<uintptr_t>(cnt32) & 15u) == 0;
+    auto load_group = [&](int gi) -> uint4 {
+      const int f = gi * 4;
+      if (vec && f + 3 < n) return ld_relaxed_gpu_v4(cnt32 + f);
+      uint4 v = make_uint4(1u, 1u, 1u, 1u);  // words past n count as published zeros
+      const int32_t *w32 = reinterpret_cast<const int32_t *>(cnt32) + f;
+      v.x = static_cast<uint32_t>(ld_relaxed_gpu(w32));
+      if (f + 1 < n) v.y = static_cast<uint32_t>(ld_relaxed_gpu(w32 + 1));
+      if (f + 2 < n) v.z = static_cast<uint32_t>(ld_relaxed_gpu(w32 + 2));
+      if (f + 3 < n) v.w = static_cast<uint32_t>(ld_relaxed_gpu(w32 + 3));
+      return v;
+    };
+    auto unpublished = [](const uint4 &w) {
+      return w.x == 0u || w.y == 0u || w.z == 0u || w.w == 0u;
+    };
+    uint32_t acc[4] = {0u, 0u, 0u, 0u};
     bool timed_out = false;
-    constexpr int B = 8;
-    for (int f0 = 0; f0 < n; f0 += kScanTile * B) {
-      uint64_t w[B];
+    constexpr int kB = 8;
+    for (int g0 = tid; g0 < ngroups; g0 += kScanTile * kB) {
+      uint4 v[kB];
+      uint32_t pend = 0u;
 #pragma unroll
-      for (int b = 0; b < B; ++b) {
-        const int f = f0 + b * kScanTile + tid;
-        w[b] = f < n ? ld_relaxed_gpu(p.desc + f) : (1ull << 32);
+      for (int b = 0; b < kB; ++b) {
+        const int gi = g0 + b * kScanTile;
+        v[b] = gi < ngroups ? load_group(gi) : make_uint4(1u, 1u, 1u, 1u);
       }
 #pragma unroll
-      for (int b = 0; b < B; ++b) {
-        const int f = f0 + b * kScanTile + tid;
-        if ((w[b] >> 32) == 0 && f < n && !timed_out) {
-          const uint64_t ts = globaltimer();
-          do {
-            __nanosleep(64);
-            w[b] = ld_relaxed_gpu(p.desc + f);
-            if ((w[b] >> 32) != 0) break;
-            if (globaltimer() - ts > p.timeout_ns) timed_out = true;
-          } while (!timed_out);
-        }
-        if ((w[b] >> 32) != 0) acc += static_cast<int>(static_cast<uint32_t>(w[b]));
+      for (int b = 0; b < kB; ++b)
+        if (unpublished(v[b])) pend |= 1u << b;
+      if (pend != 0u && !timed_out) {
+        const uint64_t ts = globaltimer();
+        do {
+          __nanosleep(64);
+#pragma unroll
+          for (int b = 0; b < kB; ++b)
+            if ((pend >> b) & 1u) v[b] = load_group(g0 + b * kScanTile);
+#pragma unroll
+          for (int b = 0; b < kB; ++b)
+            if (((pend >> b) & 1u) && !unpublished(v[b])) pend &= ~(1u << b);
+          if (pend != 0u && globaltimer() - ts > p.timeout_ns) timed_out = true;
+        } while (pend != 0u && !timed_out);
+      }
+#pragma unroll
+      for (int b = 0; b < kB; ++b) {
+        acc[0] += v[b].x != 0u ? v[b].x - 1u : 0u;
+        acc[1] += v[b].y != 0u ? v[b].y - 1u : 0u;
+        acc[2] += v[b].z != 0u ? v[b].z - 1u : 0u;
+        acc[3] += v[b].w != 0u ? v[b].w - 1u : 0u;
       }
     }
     if (timed_out) report(p.status, EP_STATUS_WAIT_TIMEOUT);
-    if (acc != 0) atomicAdd(&s_excl[tid % p.R], acc);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (acc[q] != 0u) atomicAdd(&s_excl[(4 * tid + q) % p.R], static_cast<int>(acc[q]));
     __syncthreads();
     for (int d = tid; d < p.R; d += kScanTile) {
       const int excl = s_excl[d];
