@@ -20,7 +20,6 @@ namespace ep {
 namespace {
 
 constexpr int kCombineWarps = 8;
-constexpr int kCombineBatch = 8;
 
 __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 &v) {
   acc[0] += bf16lo(v.x);
@@ -44,9 +43,13 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float (&a)[8]) {
 
 // kTab: the destinations' buffers are given by tables of R pointers (one
 // rank of a sharded job: peers' memory, read with plain loads); else they
-// are slices d * cap of y and recv_w.
-template <bool kTab>
-__global__ void __launch_bounds__(kCombineWarps * 32)
+// are slices d * cap of y and recv_w.  kBatch: rows whose chunks are loaded
+// at once; kMinCtas: CTAs per SM the registers are sized for.  Two shapes:
+// 8 rows at 2 CTAs per SM, and -- when no token can have more than 6
+// copies -- 6 rows at 3 CTAs per SM, where the extra warps put more loads in
+// flight than the rows of one token can.
+template <bool kTab, int kBatch, int kMinCtas>
+__global__ void __launch_bounds__(kCombineWarps * 32, kMinCtas)
     combine_kernel(const uint8_t *__restrict__ y, const float *__restrict__ recv_w,
                    const uint8_t *const *y_tab, const float *const *w_tab,
                    const int32_t *__restrict__ send_pos, const uint8_t *__restrict__ bias0,
@@ -96,10 +99,10 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
       const bool two = c + 32 < nvec;
       float a0[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       float a1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int i = 0; i < n; i += kCombineBatch) {
-        uint4 v0[kCombineBatch], v1[kCombineBatch];
+      for (int i = 0; i < n; i += kBatch) {
+        uint4 v0[kBatch], v1[kBatch];
 #pragma unroll
-        for (int b = 0; b < kCombineBatch; ++b) {
+        for (int b = 0; b < kBatch; ++b) {
           if (i + b < n) {
             const uint8_t *r = rows[i + b];
             v0[b] = ld_stream_v4(r + static_cast<long>(c) * 16);
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
           }
         }
 #pragma unroll
-        for (int b = 0; b < kCombineBatch; ++b) {
+        for (int b = 0; b < kBatch; ++b) {
           if (i + b < n) {
             add_bf16x8(a0, v0[b]);
             if (two) add_bf16x8(a1, v1[b]);
@@ -135,35 +138,51 @@ __global__ void __launch_bounds__(kCombineWarps * 32)
   }
 }
 
-// Launch of either form (arguments already checked).
-int combine_launch(const void *y, const float *recv_w, const uint8_t *const *y_tab,
-                   const float *const *w_tab, const int32_t *send_pos, const void *bias_0,
-                   const void *bias_1, int R, long num_tok, int H, int K, int cap,
-                   void *combined_x, float *combined_w, int32_t *status, cudaStream_t stream) {
+// Launch of one instantiation (arguments already checked).
+template <bool kTab, int kBatch, int kMinCtas>
+int combine_launch_as(const void *y, const float *recv_w, const uint8_t *const *y_tab,
+                      const float *const *w_tab, const int32_t *send_pos, const void *bias_0,
+                      const void *bias_1, int R, long num_tok, int H, int K, int cap,
+                      void *combined_x, float *combined_w, int32_t *status,
+                      cudaStream_t stream) {
   const int threads = kCombineWarps * 32;
   const size_t smem = static_cast<size_t>(kCombineWarps) * 2 * R * sizeof(void *);
-  const bool tab = y_tab != nullptr;
-  const void *fn = tab ? reinterpret_cast<const void *>(combine_kernel<true>)
-                       : reinterpret_cast<const void *>(combine_kernel<false>);
+  auto *kernel = combine_kernel<kTab, kBatch, kMinCtas>;
+  const void *fn = reinterpret_cast<const void *>(kernel);
   if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
   const long want = (num_tok + kCombineWarps - 1) / kCombineWarps;
   const long grid =
       std::min<long>(want, static_cast<long>(ctas_per_sm(fn, threads, smem)) * num_sms());
-  const bool want_w = combined_w != nullptr;
-  cudaError_t launched;
-  if (tab)
-    launched = launch_pdl(combine_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(threads),
-        smem, stream, static_cast<const uint8_t *>(nullptr), static_cast<const float *>(nullptr),
-        y_tab, w_tab, send_pos, static_cast<const uint8_t *>(bias_0),
-        static_cast<const uint8_t *>(bias_1), R, num_tok, H, K, cap, want_w,
-        static_cast<uint8_t *>(combined_x), combined_w, status);
-  else
-    launched = launch_pdl(combine_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(threads),
-        smem, stream, static_cast<const uint8_t *>(y), recv_w,
-        static_cast<const uint8_t *const *>(nullptr), static_cast<const float *const *>(nullptr),
-        send_pos, static_cast<const uint8_t *>(bias_0), static_cast<const uint8_t *>(bias_1), R,
-        num_tok, H, K, cap, want_w, static_cast<uint8_t *>(combined_x), combined_w, status);
+  const cudaError_t launched = launch_pdl(
+      kernel, dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream,
+      static_cast<const uint8_t *>(y), recv_w, y_tab, w_tab, send_pos,
+      static_cast<const uint8_t *>(bias_0), static_cast<const uint8_t *>(bias_1), R, num_tok, H,
+      K, cap, combined_w != nullptr, static_cast<uint8_t *>(combined_x), combined_w, status);
   return launch_status(launched);
+}
+
+// Launch of either form.  A token has at most min(K, R) copies (one per
+// destination rank of its experts); when that is at most 6, the 6-row,
+// 3-CTA shape reads every token's copies in one batch.  (K only bounds the
+// copies when it is the routing's top-k; any K gives the same results.)
+int combine_launch(const void *y, const float *recv_w, const uint8_t *const *y_tab,
+                   const float *const *w_tab, const int32_t *send_pos, const void *bias_0,
+                   const void *bias_1, int R, long num_tok, int H, int K, int cap,
+                   void *combined_x, float *combined_w, int32_t *status, cudaStream_t stream) {
+  const bool narrow = R <= 6 || (K >= 1 && K <= 6);
+  if (y_tab != nullptr)
+    return narrow ? combine_launch_as<true, 6, 3>(y, recv_w, y_tab, w_tab, send_pos, bias_0,
+                                                  bias_1, R, num_tok, H, K, cap, combined_x,
+                                                  combined_w, status, stream)
+                  : combine_launch_as<true, 8, 2>(y, recv_w, y_tab, w_tab, send_pos, bias_0,
+                                                  bias_1, R, num_tok, H, K, cap, combined_x,
+                                                  combined_w, status, stream);
+  return narrow ? combine_launch_as<false, 6, 3>(y, recv_w, y_tab, w_tab, send_pos, bias_0, bias_1,
+                                                 R, num_tok, H, K, cap, combined_x, combined_w,
+                                                 status, stream)
+                : combine_launch_as<false, 8, 2>(y, recv_w, y_tab, w_tab, send_pos, bias_0, bias_1,
+                                                 R, num_tok, H, K, cap, combined_x, combined_w,
+                                                 status, stream);
 }
 
 }  // namespace
