@@ -145,6 +145,7 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   __shared__ int s_last;
   __shared__ uint32_t s_mask[kScanTile * kMaskWords];
   __shared__ int s_woff[kScanWarps][kMaxRanks];
+  __shared__ uint32_t s_bal[kScanWarps][kMaxRanks];  // lanes of the warp whose token goes to d
   __shared__ int s_excl[kMaxRanks];
   __shared__ int s_agg[kMaxRanks];
   __shared__ int s_ehist[kMaxExperts];
@@ -239,7 +240,10 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
     const int nb = min(32, p.R - d0);
     for (int b = 0; b < nb; ++b) {
       const uint32_t bal = __ballot_sync(0xffffffffu, (word >> b) & 1u);
-      if (lane == 0) s_woff[warp][d0 + b] = __popc(bal);
+      if (lane == 0) {
+        s_woff[warp][d0 + b] = __popc(bal);
+        s_bal[warp][d0 + b] = bal;
+      }
     }
   }
   __syncthreads();
@@ -363,46 +367,52 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
   __syncthreads();
 
   // ---- pass 2: positions, handle and received metadata -------------------
+  // The token's row in destination d (where it goes): rows of earlier tiles,
+  // of earlier warps of this tile, then of lower lanes of this warp.  Each
+  // thread writes its own send_pos row, then one row of handle and metadata
+  // per destination it goes to (its set routing bits), so the work follows
+  // the token's copies, not R.
   const uint32_t lt = lanemask_lt();
   bool overflow = false;
-  int32_t spq[8];  // send positions of the current group of 8 destinations
+  auto goes = [&](int d) { return ((my_mask[d >> 5] >> (d & 31)) & 1u) != 0u; };
+  auto pos_of = [&](int d) { return s_excl[d] + s_woff[warp][d] + __popc(s_bal[warp][d] & lt); };
+  if (valid) {
+    if (p.sp32) {  // R % 8 == 0, rows 32-byte aligned: a whole sector per 8 ranks
+      for (int d0 = 0; d0 < p.R; d0 += 8) {
+        int32_t q[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) spq[j] = -1;
-  for (int d0 = 0; d0 < p.R; d0 += 32) {
-    const uint32_t word = my_mask[d0 >> 5];
-    const int nb = min(32, p.R - d0);
-    for (int b = 0; b < nb; ++b) {
-      const int d = d0 + b;
-      const bool has = (word >> b) & 1u;
-      const uint32_t bal = __ballot_sync(0xffffffffu, has);
-      if (!valid) continue;
-      const int pos = has ? s_excl[d] + s_woff[warp][d] + __popc(bal & lt) : -1;
-      if (p.sp32) {  // R % 8 == 0, rows 32-byte aligned: a whole sector per 8 ranks
-#pragma unroll
-        for (int j = 0; j < 8; ++j) spq[j] = (b & 7) == j ? pos : spq[j];
-        if ((b & 7) == 7) st_v8_b32(p.send_pos + st * p.R + d - 7, spq);
-      } else {
-        p.send_pos[st * p.R + d] = pos;
+        for (int j = 0; j < 8; ++j) q[j] = goes(d0 + j) ? pos_of(d0 + j) : -1;
+        st_v8_b32(p.send_pos + st * p.R + d0, q);
       }
-      if (!has) continue;
-      if (pos < 0 || pos >= p.cap) {  // pos < 0 only after a timed-out look-back
-        overflow = true;
-        continue;
-      }
-      if (p.rsi_tab != nullptr) {  // the destination's buffers, in peer memory
-        p.rsi_tab[d][pos] = t;
-        if (meta)
-          write_meta(p.ridx_tab != nullptr ? p.ridx_tab[d] + static_cast<size_t>(pos) * p.K
+    } else {
+      for (int d = 0; d < p.R; ++d) p.send_pos[st * p.R + d] = goes(d) ? pos_of(d) : -1;
+    }
+    for (int w = 0; w < p.W; ++w) {
+      uint32_t word = my_mask[w];
+      while (word != 0u) {
+        const int d = w * 32 + __ffs(word) - 1;
+        word &= word - 1u;
+        const int pos = pos_of(d);
+        if (pos < 0 || pos >= p.cap) {  // pos < 0 only after a timed-out look-back
+          overflow = true;
+          continue;
+        }
+        if (p.rsi_tab != nullptr) {  // the destination's buffers, in peer memory
+          p.rsi_tab[d][pos] = t;
+          if (meta)
+            write_meta(p.ridx_tab != nullptr ? p.ridx_tab[d] + static_cast<size_t>(pos) * p.K
+                                             : nullptr,
+                       p.rw_tab != nullptr ? p.rw_tab[d] + static_cast<size_t>(pos) * p.K
                                            : nullptr,
-                     p.rw_tab != nullptr ? p.rw_tab[d] + static_cast<size_t>(pos) * p.K : nullptr,
-                     p.K, d, dk, lk, wk, p.idx32 != 0, p.w32 != 0);
-      } else {
-        const size_t row = static_cast<size_t>(d) * p.cap + pos;
-        p.recv_src_idx[row] = t;
-        if (meta)
-          write_meta(p.recv_idx != nullptr ? p.recv_idx + row * p.K : nullptr,
-                     p.recv_w != nullptr ? p.recv_w + row * p.K : nullptr, p.K, d, dk, lk, wk,
-                     p.idx32 != 0, p.w32 != 0);
+                       p.K, d, dk, lk, wk, p.idx32 != 0, p.w32 != 0);
+        } else {
+          const size_t row = static_cast<size_t>(d) * p.cap + pos;
+          p.recv_src_idx[row] = t;
+          if (meta)
+            write_meta(p.recv_idx != nullptr ? p.recv_idx + row * p.K : nullptr,
+                       p.recv_w != nullptr ? p.recv_w + row * p.K : nullptr, p.K, d, dk, lk, wk,
+                       p.idx32 != 0, p.w32 != 0);
+        }
       }
     }
   }
