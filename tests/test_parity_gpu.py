@@ -136,6 +136,12 @@ PARITY_CASES = [
     ("el3_align4", Workload("e3", R=5, T=150, H=64, E=15, K=4, masked_frac=0.05, seed=14), 4),
     # the largest rank count (12 warps per copy CTA, 384-bit routing masks)
     ("r384_max", Workload("r384", R=384, T=3, H=64, E=384, K=4, seed=16), 1),
+    # one and two ranks: a tile's predecessors hold a number of counts that is
+    # not a multiple of four (the look-back's last group is partly past the end)
+    ("r1_tiles", Workload("r1", R=1, T=700, H=64, E=8, K=3, seed=19), 1),
+    ("r2_tiles", Workload("r2", R=2, T=650, H=64, E=10, K=4, masked_frac=0.05, seed=20), 1),
+    # seven slots on eight ranks: just past the bound for combine's 6-row shape
+    ("k7_r8", Workload("k7", R=8, T=300, H=136, E=32, K=7, masked_frac=0.05, seed=23), 1),
 ]
 
 
@@ -559,6 +565,36 @@ def test_dispatch_combine_k16_e512():
     check_dispatch(out, ref, w.R, w.K)
     np.testing.assert_array_equal(to_host(cx), ref["combined_x"])
     np.testing.assert_array_equal(to_host(cw), ref["combined_topk_weights"])
+
+
+def test_ll_windowed_lookback():
+    """40 scan tiles x 512 experts is past the size at which a tile reads every
+    predecessor's counts at once: the windowed decoupled look-back on 64-bit
+    descriptors, five tiles per source (row counts added by atomics)."""
+    w = Workload("llw", R=8, T=600, H=128, E=512, K=8, masked_frac=0.05, seed=76)
+    inp = make(w)
+    x = inp["x"]
+    idx = _dup_slots(inp["topk_idx"], 0.1, w.seed)
+    R, E = w.R, w.E
+    El = E // R
+    ref = oracle.ll_layout(idx, E)
+    rq, rs = oracle.ll_dispatch_rows(x, idx, ref["ll_pos"], E, use_fp8=True)
+    st = ep.new_status()
+    out = ep.ep_ll_dispatch(to_dev(x), to_dev(idx), E, use_fp8=True, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(to_host(out["recv_count"]), ref["recv_count"])
+    np.testing.assert_array_equal(to_host(out["layout_range"]), ref["layout_range"])
+    np.testing.assert_array_equal(to_host(out["ll_pos"]), ref["ll_pos"])
+    q = to_host(out["recv_x"])
+    rsi = to_host(out["recv_src_info"])
+    sc = to_host(out["recv_scales"])
+    for d in range(R):
+        for j in range(El):
+            n = ref["recv_count"][d, j]
+            np.testing.assert_array_equal(rsi[d, j, :n], ref["recv_src_info"][d, j, :n])
+            np.testing.assert_array_equal(q[d, j, :n], rq[d, j, :n])
+            np.testing.assert_array_equal(sc[d, j, :n], rs[d, j, :n])
 
 
 def test_ll_k16_e512():
