@@ -119,6 +119,8 @@ def _dying_worker(rank, world, port, q):
         q.put((rank, "completed", time.monotonic() - t0))
     except Exception as e:  # the survivor learns of it from its collective
         q.put((rank, type(e).__name__, time.monotonic() - t0))
+    q.close()
+    q.join_thread()  # the message is written out before the process ends
     os._exit(0)
 
 
