@@ -345,33 +345,40 @@ def to_dev_bf16(a: np.ndarray, device):
     return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
 
 
+def graph_time_ms(fn, device, iters=20, warm=3) -> float:
+    """Mean device time of fn() in ms: `iters` calls captured in one CUDA
+    graph and replayed, so host launch overhead does not enter the number.
+    fn launches on the current stream (the capture stream while capturing)."""
+    import torch
+
+    stream = torch.cuda.current_stream(device)
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(iters):
+            fn()
+    g.replay()
+    torch.cuda.synchronize(device)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    g.replay()
+    b.record(stream)
+    b.synchronize()
+    del g
+    return a.elapsed_time(b) / iters
+
+
 def extra_configs(device, ep) -> dict:
     """Secondary workloads (timed only; parity is the tests' job)."""
     import torch
 
     out = {}
-    stream = torch.cuda.current_stream(device)
 
     def timeit(fn, iters=20, warm=3):
-        """Mean device time of fn(): `iters` calls captured in one CUDA graph
-        and replayed, so host launch overhead does not enter the number."""
-        for _ in range(warm):
-            fn()
-        torch.cuda.synchronize(device)
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for _ in range(iters):
-                fn()
-        g.replay()
-        torch.cuda.synchronize(device)
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        g.replay()
-        b.record(stream)
-        b.synchronize()
-        del g
-        return a.elapsed_time(b) / iters
+        return graph_time_ms(fn, device, iters=iters, warm=warm)
 
     # layout only: [4096, 8] of 256 experts, 8 ranks
     w = CONFIGS["layout"]
@@ -587,6 +594,25 @@ def run_ours(args) -> None:
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the timed region")
 
+    # Each phase alone, replayed from a CUDA graph on the same buffers (outside
+    # the timed region): no event sits between the kernels of a phase, so the
+    # launch chaining inside it stays, as in the steps of the timed region.
+    phases_graph = {
+        "dispatch_notify_with_layout": graph_time_ms(
+            lambda: ep.ep_notify_dispatch(idx, wt, T, R, E, with_layout=True, out=out,
+                                          workspace=wsp, status=status), device, iters=50),
+        "dispatch_copy": graph_time_ms(
+            lambda: ep.ep_dispatch_cached(x, out["send_pos"], recv_x=out["recv_x"],
+                                          status=status), device, iters=10),
+        "combine": graph_time_ms(
+            lambda: ep.ep_combine(out["recv_x"], out["send_pos"], out["recv_topk_weights"],
+                                  combined_x=cx, combined_topk_weights=cw, status=status),
+            device, iters=10),
+    }
+    torch.cuda.synchronize(device)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the phase replays")
+
     # ---- end to end: host inputs in, host result out, every step -----------
     # Batches stream the way a serving loop feeds them: while step i computes,
     # the inputs of step i+1 go up on one copy stream and the result of step
@@ -666,6 +692,7 @@ def run_ours(args) -> None:
         "phases_ms": {"dispatch": disp_ms, "dispatch_notify_with_layout": notify_ms,
                       "dispatch_copy": copy_ms, "combine": comb_ms,
                       "step_with_phase_events": ms_phased},
+        "phases_graph_replay_ms": phases_graph,
         "bytes_per_step": {"dispatch": bytes_d, "combine": bytes_c, "copies": N},
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
