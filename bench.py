@@ -701,7 +701,7 @@ def run_ours(args) -> None:
                      if peak_kind == "measured" else "fallback 6.65 TB/s"},
         "e2e": {"value": e2e["gbs"], "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e["ms_per_step"]},
-        "gpu_launches": 4 * args.steps,   # scan (+layout), pad, copy, combine per step
+        "gpu_launches": 5 * args.steps,   # zeroing, scan (+layout), pad, copy, combine per step
         "clocks": clocks,
     }
     if ws == 1 and rank == 0 and not args.no_extra and T == CONFIGS["normal"].T:
@@ -859,7 +859,7 @@ def run_sharded(args) -> None:
                          "arrival_skew_us": (max(starts) - min(starts)) / 1e3},
         "e2e": {"value": e2e["gbs"], "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": cx_h.numel() * 2, "ms_per_step": e2e["ms_per_step"]},
-        "gpu_launches": 6 * args.steps,   # layout, prefix, scan, pad, copy, combine per step
+        "gpu_launches": 7 * args.steps,   # layout, zeroing, prefix, scan, pad, copy, combine per step
         "cuda_graph": graph is not None, "cuda_graph_note": graph_note,
         "eager": {"ms_per_step": eager["ms_per_step"], "value": eager["gbs"]},
         "clocks": clocks,

@@ -108,6 +108,42 @@ int ctas_per_sm(const void *func, int threads, size_t smem) {
   return n;
 }
 
+namespace {
+
+__global__ void __launch_bounds__(256) zero_prefetch_kernel(uint4 *a, long a16, int32_t *b,
+                                                            long b_words, const char *pf,
+                                                            long pf_bytes) {
+  const long nthr = static_cast<long>(gridDim.x) * blockDim.x;
+  const long me = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (long off = me * 128; off < pf_bytes; off += nthr * 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(pf + off));
+  pdl_wait();
+  pdl_trigger();  // the next kernel's CTAs may start; they wait for this grid to complete
+  for (long i = me; i < a16; i += nthr) a[i] = make_uint4(0u, 0u, 0u, 0u);
+  for (long i = me; i < b_words; i += nthr) b[i] = 0;
+}
+
+}  // namespace
+
+int zero_prefetch(void *a, size_t a_bytes, int32_t *b, long b_words, const void *pf,
+                  long pf_bytes, cudaStream_t stream) {
+  if ((reinterpret_cast<uintptr_t>(a) & 15u) != 0 || (a_bytes & 15u) != 0) {
+    if (a_bytes > 0 && cudaMemsetAsync(a, 0, a_bytes, stream) != cudaSuccess) return EP_ERR_CUDA;
+    if (b_words > 0 &&
+        cudaMemsetAsync(b, 0, sizeof(int32_t) * static_cast<size_t>(b_words), stream) !=
+            cudaSuccess)
+      return EP_ERR_CUDA;
+    return EP_OK;
+  }
+  const long a16 = static_cast<long>(a_bytes / 16);
+  if (pf == nullptr) pf_bytes = 0;
+  const long want = (std::max({a16, b_words, (pf_bytes + 127) / 128}) + 255) / 256;
+  const long grid = std::max(1L, std::min<long>(want, num_sms()));
+  return launch_status(launch_pdl(zero_prefetch_kernel, dim3(static_cast<unsigned>(grid)),
+                                  dim3(256), 0, stream, static_cast<uint4 *>(a), a16, b, b_words,
+                                  static_cast<const char *>(pf), pf_bytes));
+}
+
 }  // namespace ep
 
 extern "C" {

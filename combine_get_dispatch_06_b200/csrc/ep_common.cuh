@@ -74,6 +74,15 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
 }
 
+// Zeroes a[0, a_bytes) and b[0, b_words) on `stream` with a kernel chained
+// to its neighbours by programmatic launch (a memset node would break that
+// chain): it waits for the previous kernel in the stream before it stores,
+// and lets the next one start.  Before that wait it asks L2 for
+// pf[0, pf_bytes) (a hint only; pf may be nullptr).  Falls back to memsets
+// where `a` is not 16-byte aligned or a_bytes not a multiple of 16.
+int zero_prefetch(void *a, size_t a_bytes, int32_t *b, long b_words, const void *pf,
+                  long pf_bytes, cudaStream_t stream);
+
 __device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }

@@ -847,7 +847,10 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   }
   const int Ectr = topk_idx != nullptr ? E : 0;
   const size_t need = ep_dispatch_workspace_bytes(R, T, Ectr);
-  if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return EP_ERR_CUDA;
+  // zeroed by a kernel chained to the scan, which first asks L2 for the ids
+  if (zero_prefetch(workspace, need, nullptr, 0, topk_idx,
+                    topk_idx != nullptr ? static_cast<long>(R) * T * K * 8 : 0L, stream) != EP_OK)
+    return EP_ERR_CUDA;
 
   const int tiles_per_src = (T + kScanTile - 1) / kScanTile;
   const long num_tiles = static_cast<long>(R) * tiles_per_src;
@@ -1265,7 +1268,7 @@ extern "C" EP_API int ep_shard_notify(
       (reinterpret_cast<uintptr_t>(notify_probe) & 7u))
     return EP_ERR_INVALID_ARG;
 
-  if (cudaMemsetAsync(workspace, 0, need, stream) != cudaSuccess) return EP_ERR_CUDA;
+  if (zero_prefetch(workspace, need, nullptr, 0, nullptr, 0, stream) != EP_OK) return EP_ERR_CUDA;
   const ShardWs w = shard_ws(workspace, R);
   cudaError_t launched = launch_pdl(shard_prefix_kernel, dim3(1), dim3(256), 0, stream, counts,
                                     expert_counts, R, E, rank, align, rank_prefix_matrix,

@@ -15,9 +15,7 @@
 //   - combine: acc = fmaf(y, w_k, acc) over slots k ascending, one bf16
 //     rounding at the end.
 //
-// Kernels:
-//   ll_prepare_kernel   zeroes the workspace words the call uses (after the
-//                       previous kernel), prefetching the ids into L2 first
+// Kernels (after zero_prefetch clears the workspace words the call uses):
 //   ll_scan_kernel      positions, recv_src_info, layout_range, counts, and
 //                       a mirror of the positions for the dispatch kernel
 //   ll_dispatch_kernel  runs concurrently with the scan; one CTA per token at
@@ -56,26 +54,6 @@ struct LLScanParams {
   unsigned long long timeout_ns;
   unsigned flags;
 };
-
-// The call's first kernel: zeroes the workspace words the call uses (and
-// layout_range where several tiles add up a source's counts), once the
-// previous kernel in the stream is complete.  Before that wait it asks L2 for
-// the routing ids the scan reads first: a hint only, since the scan reads
-// them after its own wait.  It stands in for a memset so that the chain of
-// programmatically serialized launches is not broken before the scan.
-__global__ void __launch_bounds__(256) ll_prepare_kernel(uint4 *ws, long words16, int32_t *lr,
-                                                         long lr_words, const int64_t *ids,
-                                                         long id_bytes) {
-  const long nthr = static_cast<long>(gridDim.x) * blockDim.x;
-  const long me = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const char *base = reinterpret_cast<const char *>(ids);
-  for (long off = me * 128; off < id_bytes; off += nthr * 128)
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(base + off));
-  pdl_wait();
-  pdl_trigger();  // the scan's CTAs may start; they wait for this grid to complete
-  for (long i = me; i < words16; i += nthr) ws[i] = make_uint4(0u, 0u, 0u, 0u);
-  for (long i = me; i < lr_words; i += nthr) lr[i] = 0;
-}
 
 // MAXK: compile-time bound on the top-k slots (8 or 16), chosen per call.
 //
@@ -795,20 +773,13 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   if (plan.stages < 2) return EP_ERR_UNSUPPORTED;
   // header, descriptors and the mirror words this call uses start at zero
   const size_t used = ll_mirror_offset(num_tiles, E) + static_cast<size_t>(cap) * K * sizeof(int32_t);
-  {
-    // (the workspace is at least ep_ll_workspace_bytes, a multiple of 256 bytes
-    // past `used`, so whole 16-byte words stay inside it)
-    const long words16 = static_cast<long>((used + 15) / 16);
-    // several tiles per source add up their counts; a single tile stores them
-    const long lr_words = tiles_per_src > 1 ? 2L * E * R : 0L;
-    const long id_bytes = static_cast<long>(R) * T * K * 8;
-    const long want = (std::max({words16, lr_words, (id_bytes + 127) / 128}) + 255) / 256;
-    const long grid = std::max(1L, std::min<long>(want, num_sms()));
-    if (launch_status(launch_pdl(ll_prepare_kernel, dim3(static_cast<unsigned>(grid)), dim3(256),
-                                 0, stream, static_cast<uint4 *>(workspace), words16,
-                                 layout_range, lr_words, topk_idx, id_bytes)) != EP_OK)
-      return EP_ERR_CUDA;
-  }
+  // the call's first kernel zeroes them (the workspace is at least
+  // ep_ll_workspace_bytes, a multiple of 256 bytes past `used`, so whole
+  // 16-byte words stay inside it), prefetching the ids the scan reads first
+  if (zero_prefetch(workspace, (used + 15) & ~static_cast<size_t>(15), layout_range,
+                    tiles_per_src > 1 ? 2L * E * R : 0L, topk_idx,
+                    static_cast<long>(R) * T * K * 8, stream) != EP_OK)
+    return EP_ERR_CUDA;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   LLScanParams p;
