@@ -60,6 +60,7 @@ struct DispatchScanParams {
   // start in the workspace; cumulative [ns, launches, last start, last end].
   unsigned long long *probe_state;
   unsigned long long *probe;
+  int finalise;  // the last CTA writes nrte / ntpe_out / ntpr_out (else notify_finish_kernel)
   int idx32, w32, sp32;  // 32-byte stores of received ids / weights / send_pos rows
   ScanHeader *head;
   int32_t *expert_cnt;   // [E] all sources, then [R][E] per source
@@ -428,11 +429,12 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
       }
     }
   pdl_trigger();
-  if (elect_last_cta(&p.head->done, static_cast<uint32_t>(p.num_tiles), &s_last)) {
+  if ((p.finalise != 0 || p.probe != nullptr) &&
+      elect_last_cta(&p.head->done, static_cast<uint32_t>(p.num_tiles), &s_last)) {
     // one CTA finalises: loads are issued in batches of 8 so that the loop
     // does not wait one L2 round trip per element
     constexpr int B = 8;
-    if (p.nrte != nullptr)
+    if (p.finalise != 0 && p.nrte != nullptr)
       for (int e0 = 0; e0 < p.E; e0 += kScanTile * B) {
         int v[B];
 #pragma unroll
@@ -448,7 +450,7 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
           if (e < p.E) p.nrte[e] = n;
         }
       }
-    if (p.ntpe_out != nullptr)
+    if (p.finalise != 0 && p.ntpe_out != nullptr)
       for (int i0 = 0; i0 < p.R * p.E; i0 += kScanTile * B) {
         int v[B];
 #pragma unroll
@@ -462,7 +464,7 @@ __global__ void __launch_bounds__(kScanTile) dispatch_scan_kernel(DispatchScanPa
           if (i < p.R * p.E) p.ntpe_out[i] = v[b];
         }
       }
-    if (p.ntpr_out != nullptr)  // tokens of s to d = P[s][d] - P[s-1][d]
+    if (p.finalise != 0 && p.ntpr_out != nullptr)  // tokens of s to d = P[s][d] - P[s-1][d]
       for (int i = tid; i < p.R * p.R; i += kScanTile) {
         const int prev = i >= p.R ? __ldcg(&p.P[i - p.R]) : 0;
         p.ntpr_out[i] = __ldcg(&p.P[i]) - prev;
@@ -784,28 +786,58 @@ extern "C" EP_API size_t ep_dispatch_workspace_bytes(int num_ranks, int num_toke
 namespace ep {
 namespace {
 
-// recv_topk_idx rows from recv_count[d] to cap - 1 := -1 (grid: x over the
-// rows, y over the destination ranks).  16-byte stores when a row of K int64
-// is a multiple of 16 bytes.
-__global__ void __launch_bounds__(256)
-    pad_recv_idx_kernel(const int32_t *__restrict__ recv_count, int cap, int K,
-                        int64_t *__restrict__ recv_idx) {
+// After the scan.  recv_topk_idx rows from recv_count[d] to cap - 1 := -1
+// (grid: x over the rows, y over the destination ranks; 16-byte stores when
+// a row of K int64 is a multiple of 16 bytes), and the counts the scan
+// gathered become the call's outputs, spread over the whole grid: aligned
+// per-expert receive counts (nrte) and, for the fused layout, every source's
+// tokens per expert (ntpe_out) and per rank (ntpr_out = P[s] - P[s-1]).
+// Any of recv_idx, nrte, ntpe_out, ntpr_out may be nullptr.
+struct NotifyFinishParams {
+  const int32_t *recv_count;
+  int cap, K;
+  int64_t *recv_idx;
+  const int32_t *expert_cnt;  // [E] all sources, then [R][E] per source
+  const int32_t *P;
+  int R, E, align;
+  int32_t *nrte, *ntpe_out, *ntpr_out;
+};
+
+__global__ void __launch_bounds__(256) notify_finish_kernel(NotifyFinishParams f) {
   pdl_wait();
   pdl_trigger();
-  const int d = blockIdx.y;
-  const long first = min(max(recv_count[d], 0), cap);
-  int64_t *base = recv_idx + static_cast<long>(d) * cap * K;
-  const long lo = first * K, hi = static_cast<long>(cap) * K;  // in int64 elements
-  const long step = static_cast<long>(gridDim.x) * blockDim.x;
-  if ((K & 1) == 0) {
-    const longlong2 v = make_longlong2(-1, -1);
-    for (long i = lo / 2 + static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; i < hi / 2;
-         i += step)
-      reinterpret_cast<longlong2 *>(base)[i] = v;
-  } else {
-    for (long i = lo + static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; i < hi; i += step)
-      base[i] = -1;
+  if (f.recv_idx != nullptr) {
+    const int d = blockIdx.y;
+    const long first = min(max(f.recv_count[d], 0), f.cap);
+    int64_t *base = f.recv_idx + static_cast<long>(d) * f.cap * f.K;
+    const long lo = first * f.K, hi = static_cast<long>(f.cap) * f.K;  // in int64 elements
+    const long step = static_cast<long>(gridDim.x) * blockDim.x;
+    if ((f.K & 1) == 0) {
+      const longlong2 v = make_longlong2(-1, -1);
+      for (long i = lo / 2 + static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+           i < hi / 2; i += step)
+        reinterpret_cast<longlong2 *>(base)[i] = v;
+    } else {
+      for (long i = lo + static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; i < hi;
+           i += step)
+        base[i] = -1;
+    }
   }
+  const long nthr = static_cast<long>(gridDim.x) * gridDim.y * blockDim.x;
+  const long me = (static_cast<long>(blockIdx.y) * gridDim.x + blockIdx.x) * blockDim.x +
+                  threadIdx.x;
+  if (f.nrte != nullptr)
+    for (long e = me; e < f.E; e += nthr) {
+      int n = __ldcg(&f.expert_cnt[e]);
+      if (f.align > 1) n = (n + f.align - 1) / f.align * f.align;
+      f.nrte[e] = n;
+    }
+  if (f.ntpe_out != nullptr)
+    for (long i = me; i < static_cast<long>(f.R) * f.E; i += nthr)
+      f.ntpe_out[i] = __ldcg(&f.expert_cnt[f.E + i]);
+  if (f.ntpr_out != nullptr)
+    for (long i = me; i < static_cast<long>(f.R) * f.R; i += nthr)
+      f.ntpr_out[i] = __ldcg(&f.P[i]) - (i >= f.R ? __ldcg(&f.P[i - f.R]) : 0);
 }
 
 // 32-byte stores need rows that are whole multiples of 32 bytes and a
@@ -886,6 +918,7 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   p.rw_tab = nullptr;
   p.probe_state = nullptr;
   p.probe = nullptr;
+  p.finalise = 0;  // notify_finish_kernel writes the counts after the scan
   p.head = reinterpret_cast<ScanHeader *>(ws);
   p.expert_cnt = reinterpret_cast<int32_t *>(ws + sizeof(ScanHeader));
   const int counters = Ectr * (1 + R);
@@ -906,15 +939,26 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
         dim3(static_cast<unsigned>(num_tiles)), dim3(kScanTile), 0, stream,
         p);
   if (launch_status(launched) != EP_OK) return EP_ERR_CUDA;
-  // rows past the receive count read -1 (fixed worst-case capacity)
-  if (recv_topk_idx != nullptr && cap > 0) {
-    const long words = static_cast<long>(cap) * K / ((K & 1) == 0 ? 2 : 1);
-    const int bx = static_cast<int>(std::min<long>((words + 255) / 256, 64));
-    launched = launch_pdl(pad_recv_idx_kernel, dim3(bx, R), dim3(256), 0, stream,
-        recv_count, cap, K, recv_topk_idx);
-    return launch_status(launched);
-  }
-  return EP_OK;
+  // rows past the receive count read -1 (fixed worst-case capacity), and the
+  // gathered counts become the outputs
+  NotifyFinishParams f;
+  f.recv_count = recv_count;
+  f.cap = cap;
+  f.K = K;
+  f.recv_idx = cap > 0 ? recv_topk_idx : nullptr;
+  f.expert_cnt = p.expert_cnt;
+  f.P = rank_prefix_matrix;
+  f.R = R;
+  f.E = E;
+  f.align = align;
+  f.nrte = num_recv_tokens_per_expert;
+  f.ntpe_out = ntpe_out;
+  f.ntpr_out = ntpr_out;
+  const long words = f.recv_idx != nullptr ? static_cast<long>(cap) * K / ((K & 1) == 0 ? 2 : 1)
+                                           : 0L;
+  const int bx = static_cast<int>(std::max<long>(1L, std::min<long>((words + 255) / 256, 64)));
+  launched = launch_pdl(notify_finish_kernel, dim3(bx, R), dim3(256), 0, stream, f);
+  return launch_status(launched);
 }
 
 // A3 rows: the bulk-copy kernel.  Arguments already checked.  `xs` (FP8
@@ -1313,10 +1357,14 @@ extern "C" EP_API int ep_shard_notify(
   }
   // this rank's own receive rows past its count read -1 (fixed capacity)
   if (recv_topk_idx != nullptr && cap > 0) {
+    NotifyFinishParams f = {};
+    f.recv_count = recv_count;
+    f.cap = cap;
+    f.K = K;
+    f.recv_idx = recv_topk_idx;
     const long words = static_cast<long>(cap) * K / ((K & 1) == 0 ? 2 : 1);
     const int bx = static_cast<int>(std::min<long>((words + 255) / 256, 64));
-    launched = launch_pdl(pad_recv_idx_kernel, dim3(bx, 1), dim3(256), 0, stream, recv_count,
-                          cap, K, recv_topk_idx);
+    launched = launch_pdl(notify_finish_kernel, dim3(bx, 1), dim3(256), 0, stream, f);
     return launch_status(launched);
   }
   return EP_OK;
