@@ -699,6 +699,10 @@ FUSED_CASES = [
     ("normal_like", Workload("fu1", R=8, T=300, H=64, E=256, K=8, seed=81)),
     ("ragged_masked", Workload("fu2", R=5, T=129, H=64, E=40, K=3, masked_frac=0.2, seed=82)),
     ("r40_unaligned", Workload("fu3", R=40, T=33, H=64, E=80, K=4, seed=83)),
+    # sixteen slots (the scan's 16-slot form) on 16 ranks with 512 experts: the
+    # per-source expert counts the kernel after the scan writes are 16 x 512
+    ("k16_e512", Workload("fu4", R=16, T=140, H=64, E=512, K=16, masked_frac=0.05, seed=84)),
+    ("r2_tiles", Workload("fu5", R=2, T=333, H=64, E=6, K=2, seed=85)),
 ]
 
 
