@@ -63,6 +63,11 @@ _SIGS = {
                              _P, _P, _P, _P, _P, _Z, _P, _P]),
     "ep_shard_dispatch": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "ep_shard_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "ep_shard_ll_counts": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "ep_shard_ll_workspace_bytes": (_Z, [_I, _I, _I]),
+    "ep_shard_ll_dispatch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P,
+                                  _P, _P, _P, _P, _Z, _P, _P]),
+    "ep_shard_ll_combine": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)

@@ -50,6 +50,13 @@ struct LLScanParams {
   ScanHeader *head;
   uint64_t *desc;
   int32_t *pos_mirror;  // [R*T][K] ll_pos + 2 (0 = not written yet), for the dispatch kernel
+  // One source rank of a sharded job (the call's tokens are rank s0's): rows
+  // of each expert that earlier ranks send (base[E]) and the destination
+  // ranks' recv_src_info ([R] -> [El][cap]); nullptr and s0 = 0 otherwise.
+  // layout_range, recv_count and stats then come from the gathered counts.
+  int s0;
+  const int32_t *base;
+  int32_t *const *rsi_tab;
   int32_t *status;
   unsigned long long timeout_ns;
   unsigned flags;
@@ -78,7 +85,8 @@ struct LLScanParams {
 // that a non-zero word is its own proof of being written.
 constexpr int kLLScanThreads = 2 * kScanTile;
 
-template <int MAXK>
+// kShard: one rank of a sharded job (p.s0, p.base and p.rsi_tab set).
+template <int MAXK, bool kShard>
 __global__ void __launch_bounds__(kLLScanThreads, 2) ll_scan_kernel(LLScanParams p) {
   pdl_wait();
   pdl_trigger();  // after the wait: see above
@@ -118,12 +126,12 @@ __global__ void __launch_bounds__(kLLScanThreads, 2) ll_scan_kernel(LLScanParams
 
   const int tile = s_tile;
   if (tok && tile != static_cast<int>(blockIdx.x)) load_ids(tile, ids);
-  const int s = tile / p.tiles_per_src;
+  const int s = tile / p.tiles_per_src;  // the call's source index (rank p.s0 + s)
   const int t = (tile % p.tiles_per_src) * kScanTile + tid;
   const bool valid = tok && t < p.T;
   const size_t st = static_cast<size_t>(s) * p.T + t;
   // a failed (masked) source rank sends nothing
-  const bool src_ok = p.mask == nullptr || s_mask[s] == 0;
+  const bool src_ok = p.mask == nullptr || s_mask[(kShard ? p.s0 : 0) + s] == 0;
 
   // Distinct valid experts of this token (a repeated expert keeps only its
   // first slot in `col`; `ev` keeps every valid id).  Experts on a failed
@@ -276,7 +284,8 @@ __global__ void __launch_bounds__(kLLScanThreads, 2) ll_scan_kernel(LLScanParams
     for (int k = 0; k < MAXK; ++k) {
       pos[k] = -1;
       if (col[k] >= 0) {
-        const int r = s_excl[col[k]] + s_whist[warp][col[k]] + rnk[k];
+        const int r = s_excl[col[k]] + s_whist[warp][col[k]] + rnk[k] +
+                      (kShard ? p.base[col[k]] : 0);
         if (r >= 0 && r < p.cap)
           pos[k] = r;
         else
@@ -323,11 +332,22 @@ __global__ void __launch_bounds__(kLLScanThreads, 2) ll_scan_kernel(LLScanParams
       }
     }
 #pragma unroll
-    for (int k = 0; k < MAXK; ++k)
-      if (pos[k] >= 0) p.recv_src_info[static_cast<size_t>(col[k]) * p.cap + pos[k]] = t;
+    for (int k = 0; k < MAXK; ++k) {
+      if (pos[k] < 0) continue;
+      if constexpr (kShard) {  // the destination's slab handle, in peer memory
+        const int d = col[k] / p.El;
+        p.rsi_tab[d][static_cast<size_t>(col[k] - d * p.El) * p.cap + pos[k]] = t;
+      } else {
+        p.recv_src_info[static_cast<size_t>(col[k]) * p.cap + pos[k]] = t;
+      }
+    }
     if (oob) report(p.status, EP_STATUS_BAD_POSITION);
   }
 
+  if constexpr (kShard) {  // the counts' outputs come from the gathered counts
+    __threadfence_system();  // handle entries stored into peers' memory
+    return;
+  }
   const bool first_of_src = (tile % p.tiles_per_src) == 0;
   for (int c = tid; c < p.E; c += kLLScanThreads) {
     const int run = s_cnt[c];
@@ -396,17 +416,24 @@ __host__ __device__ inline LLSmem ll_smem_plan(int H) {
 // the scan's mirror of ll_pos, read a token ahead and read again while a
 // word is still zero (not written yet).  The kernel waits for the scan grid
 // to complete before it exits, so later work in the stream sees both.
-template <bool kFP8>
+//
+// kTab: one rank of a sharded job; the slabs of destination d are recv_tab[d]
+// ([El][cap] rows) and scales_tab[d] in peer memory, and warp 0 turns each
+// slot's row into the two row pointers.
+template <bool kFP8, bool kTab>
 __global__ void __launch_bounds__(kLLThreads)
     ll_dispatch_kernel(const uint8_t *__restrict__ x, const int64_t *__restrict__ topk_idx,
                        const int32_t *pos_mirror, long num_tok, int H, int K, int E, int cap,
                        int round_scale, int ue8m0, LLSmem plan, uint8_t *__restrict__ recv,
                        void *__restrict__ scales_out, uint32_t *claim, int32_t *status,
-                       unsigned long long timeout_ns) {
+                       unsigned long long timeout_ns, uint8_t *const *recv_tab,
+                       uint8_t *const *scales_tab, int El) {
   pdl_trigger();  // the next kernel may take the room this grid leaves
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ long s_tok[kLLMaxStages];  // token in each input stage, -1 = none
   __shared__ long s_dst[kMaxTopk];      // slab row (e * cap + pos) per slot, -1 = none
+  __shared__ uint8_t *s_qp[kTab ? kMaxTopk : 1];  // kTab: payload row per slot, or nullptr
+  __shared__ uint8_t *s_sp[kTab ? kMaxTopk : 1];  // kTab: scale row per slot
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int nst = plan.stages;
@@ -510,6 +537,19 @@ __global__ void __launch_bounds__(kLLThreads)
           report(status, EP_STATUS_BAD_POSITION);
       }
       if (lane < K) s_dst[lane] = dst;
+      if constexpr (kTab) {
+        if (lane < K) {
+          uint8_t *qp = nullptr, *sp = nullptr;
+          if (dst >= 0) {
+            const int d = e / El;
+            const long row = static_cast<long>(e - d * El) * cap + pos;
+            qp = recv_tab[d] + row * pay;
+            if (kFP8) sp = scales_tab[d] + row * nblk * (ue8m0 ? 1 : 4);
+          }
+          s_qp[lane] = qp;
+          s_sp[lane] = sp;
+        }
+      }
     }
     const bool ok = mbar_wait_bounded(&bars[stg], phase, timeout_ns);
     if (__syncthreads_and(ok) == 0) {
@@ -562,14 +602,26 @@ __global__ void __launch_bounds__(kLLThreads)
                            __fmul_rn(f[15], inv));
           const bool first = (c & 7) == 0;
           for (int k = 0; k < K; ++k) {
-            const long dst = s_dst[k];
-            if (dst < 0) continue;
-            st_stream_v4(recv + dst * pay + c * 16L, q);
-            if (first) {
-              if (ue8m0)
-                scales8[dst * nblk + (c >> 3)] = static_cast<uint8_t>(ebits);
-              else
-                scales[dst * nblk + (c >> 3)] = scale;
+            if constexpr (kTab) {
+              uint8_t *qr = s_qp[k];
+              if (qr == nullptr) continue;
+              st_stream_v4(qr + c * 16L, q);
+              if (first) {
+                if (ue8m0)
+                  s_sp[k][c >> 3] = static_cast<uint8_t>(ebits);
+                else
+                  reinterpret_cast<float *>(s_sp[k])[c >> 3] = scale;
+              }
+            } else {
+              const long dst = s_dst[k];
+              if (dst < 0) continue;
+              st_stream_v4(recv + dst * pay + c * 16L, q);
+              if (first) {
+                if (ue8m0)
+                  scales8[dst * nblk + (c >> 3)] = static_cast<uint8_t>(ebits);
+                else
+                  scales[dst * nblk + (c >> 3)] = scale;
+              }
             }
           }
         }
@@ -578,8 +630,12 @@ __global__ void __launch_bounds__(kLLThreads)
       for (int c = tid; c < nchunk; c += kLLThreads) {
         const uint4 v = reinterpret_cast<const uint4 *>(in)[c];
         for (int k = 0; k < K; ++k) {
-          const long dst = s_dst[k];
-          if (dst >= 0) st_stream_v4(recv + dst * pay + c * 16L, v);
+          if constexpr (kTab) {
+            if (s_qp[k] != nullptr) st_stream_v4(s_qp[k] + c * 16L, v);
+          } else {
+            const long dst = s_dst[k];
+            if (dst >= 0) st_stream_v4(recv + dst * pay + c * 16L, v);
+          }
         }
       }
     }
@@ -609,25 +665,93 @@ __global__ void __launch_bounds__(kLLThreads)
       }
     }
   }
+  if constexpr (kTab) __threadfence_system();  // rows stored into peers' memory
   // the scan grid completes before this one does
   pdl_wait();
 }
 
 // ---------------------------------------------------------------------------
 
+// One rank of a sharded LL dispatch: the rows it sends to each expert (its
+// tokens whose distinct valid slots hold the expert; nothing from a failed
+// source rank, nothing to a failed rank's experts), the same count the
+// single-GPU scan takes per source rank.  A thread per token; counts zeroed
+// before.
+__global__ void __launch_bounds__(256)
+    ll_count_kernel(const int64_t *__restrict__ topk_idx, const int32_t *__restrict__ mask,
+                    int rank, int T, int K, int E, int El, int32_t *counts, int32_t *status) {
+  pdl_wait();
+  pdl_trigger();
+  const long t = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= T || (mask != nullptr && mask[rank] != 0)) return;
+  int seen[kMaxTopk];
+  int n = 0;
+  bool bad = false;
+  for (int k = 0; k < K; ++k) {
+    const int64_t e = topk_idx[t * K + k];
+    if (e == -1) continue;
+    if (e < -1 || e >= E) {
+      bad = true;
+      continue;
+    }
+    if (mask != nullptr && mask[static_cast<int>(e) / El] != 0) continue;
+    bool dup = false;
+    for (int i = 0; i < n; ++i) dup |= seen[i] == static_cast<int>(e);
+    if (dup) continue;
+    seen[n++] = static_cast<int>(e);
+    atomicAdd(&counts[e], 1);
+  }
+  if (bad) report(status, EP_STATUS_BAD_EXPERT);
+}
+
+// One rank of a sharded LL dispatch, from every rank's counts (gathered,
+// [R][E]): base[e] = rows of expert e that the ranks before `rank` send (its
+// own rows follow them, as source ranks are in order in a slab); this rank's
+// (first row, rows) entry of every destination's layout_range ([El][R][2],
+// in peer memory); and for its own experts the rows received from all ranks
+// and the cumulative counter.
+__global__ void __launch_bounds__(256)
+    shard_ll_prefix_kernel(const int32_t *__restrict__ counts, int rank, int R, int E, int El,
+                           int32_t *base, int32_t *const *lr_tab, int32_t *recv_count,
+                           int32_t *stats) {
+  pdl_wait();
+  pdl_trigger();  // the scan's CTAs may start; they wait for this grid to complete
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < E; e += gridDim.x * blockDim.x) {
+    int b = 0;
+    for (int s = 0; s < rank; ++s) b += counts[static_cast<size_t>(s) * E + e];
+    const int mine = counts[static_cast<size_t>(rank) * E + e];
+    base[e] = b;
+    const int d = e / El, j = e - d * El;
+    int32_t *lr = lr_tab[d] + (static_cast<size_t>(j) * R + rank) * 2;
+    lr[0] = b;
+    lr[1] = mine;
+    if (d == rank) {
+      int tot = b + mine;
+      for (int s = rank + 1; s < R; ++s) tot += counts[static_cast<size_t>(s) * E + e];
+      recv_count[j] = tot;
+      if (stats != nullptr) stats[j] += tot;
+    }
+  }
+  __threadfence_system();  // layout_range entries stored into peers' memory
+}
+
 constexpr int kLLCombineWarps = 8;
 
 // One warp per (token, channel segment): the token's up-to-K slab rows are
 // listed in slot order, then each lane accumulates 16-byte chunks of the
 // segment with fmaf in that order.  Splitting rows into `nseg` segments gives
-// enough work items to keep every warp busy to the end.
+// enough work items to keep every warp busy to the end.  y_tab: one rank of
+// a sharded job (its tokens are source rank s0's); expert e's rows are in
+// destination e / El's slab y_tab[e / El] in peer memory, read with plain
+// loads.  Otherwise y holds every destination's slabs and s0 = 0.
 __global__ void __launch_bounds__(kLLCombineWarps * 32)
-    ll_combine_kernel(const uint8_t *__restrict__ y, const int64_t *__restrict__ topk_idx,
+    ll_combine_kernel(const uint8_t *__restrict__ y, const uint8_t *const *y_tab, int s0,
+                      const int64_t *__restrict__ topk_idx,
                       const float *__restrict__ topk_w, const int32_t *__restrict__ ll_pos,
                       const int32_t *__restrict__ mask, long num_tok, int T, int H, int K, int E,
                       int cap, int nseg, uint8_t *__restrict__ out, int32_t *status) {
   pdl_wait();
-  __shared__ int64_t s_row[kLLCombineWarps][kMaxTopk];
+  __shared__ const uint8_t *s_row[kLLCombineWarps][kMaxTopk];
   __shared__ float s_w[kLLCombineWarps][kMaxTopk];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -642,16 +766,22 @@ __global__ void __launch_bounds__(kLLCombineWarps * 32)
     const long u = it / nseg;
     const int sg = static_cast<int>(it % nseg);
     bool take = false;
-    long row = 0;
+    const uint8_t *row = nullptr;
     float w = 0.f;
-    const bool src_ok = mask == nullptr || mask[u / T] == 0;
+    const bool src_ok = mask == nullptr || mask[s0 + u / T] == 0;
     if (lane < K && src_ok) {
       const int64_t e = topk_idx[u * K + lane];
       if (e >= 0 && e < E && (mask == nullptr || mask[e / El] == 0)) {
         const int pos = ll_pos[u * K + lane];
         if (pos >= 0 && pos < cap) {
           take = true;
-          row = e * cap + pos;
+          if (y_tab != nullptr) {
+            const int d = static_cast<int>(e) / El;
+            row = y_tab[d] + (static_cast<long>(static_cast<int>(e) - d * El) * cap + pos) *
+                                 row_bytes;
+          } else {
+            row = y + (e * cap + pos) * row_bytes;
+          }
           w = topk_w[u * K + lane];
         } else if (sg == 0 && pos != -1) {  // -1: dropped at dispatch
           report(status, EP_STATUS_BAD_POSITION);
@@ -675,7 +805,7 @@ __global__ void __launch_bounds__(kLLCombineWarps * 32)
         uint4 v[8];
 #pragma unroll
         for (int b = 0; b < 8; ++b)
-          if (i + b < n) v[b] = ld_stream_v4(y + s_row[warp][i + b] * row_bytes + c * 16L);
+          if (i + b < n) v[b] = ld_stream_v4(s_row[warp][i + b] + c * 16L);
 #pragma unroll
         for (int b = 0; b < 8; ++b) {
           if (i + b < n) {
@@ -712,6 +842,88 @@ namespace {
 size_t ll_mirror_offset(long tiles, int E) {  // 16-byte aligned
   return (sizeof(ScanHeader) + static_cast<size_t>(tiles) * E * sizeof(uint64_t) + 15) &
          ~static_cast<size_t>(15);
+}
+
+// LL combine of num_tok tokens (arguments already checked): from y, or from
+// the destinations' slabs y_tab (one rank's tokens, source rank s0).
+int ll_combine_launch(const uint8_t *y, const uint8_t *const *y_tab, int s0,
+                      const int64_t *topk_idx, const float *topk_weights, const int32_t *ll_pos,
+                      const int32_t *rank_mask, long num_tok, int T, int H, int K, int E,
+                      long cap, void *out, int32_t *status, cudaStream_t stream) {
+  const int threads = kLLCombineWarps * 32;
+  const void *fn = reinterpret_cast<const void *>(ll_combine_kernel);
+  const long resident = static_cast<long>(ctas_per_sm(fn, threads, 0)) * num_sms();
+  // split rows into segments until there are >= 4 work items per resident warp
+  const int nvec = H / 8;
+  int nseg = static_cast<int>((4 * resident * kLLCombineWarps + num_tok - 1) / num_tok);
+  nseg = std::max(1, std::min(nseg, std::max(1, nvec / 32)));
+  const long items = num_tok * nseg;
+  const long grid = std::min<long>((items + kLLCombineWarps - 1) / kLLCombineWarps, resident);
+  const cudaError_t launched = launch_pdl(ll_combine_kernel,
+      dim3(static_cast<unsigned>(grid)), dim3(threads), 0, stream, y, y_tab, s0, topk_idx,
+      topk_weights, ll_pos, rank_mask, num_tok, T, H, K, E, static_cast<int>(cap), nseg,
+      static_cast<uint8_t *>(out), status);
+  return launch_status(launched);
+}
+
+// The scan, then the dispatch kernel that runs alongside it (arguments
+// already checked, the workspace words zeroed).  recv_tab / scales_tab: the
+// destinations' slabs in peer memory (one rank of a sharded job), else
+// recv_x / recv_scales hold every destination's slabs.
+int ll_scan_and_dispatch(const LLScanParams &p, const void *x, int H, int use_fp8,
+                         int round_scale, int ue8m0, const LLSmem &plan, void *recv_x,
+                         void *recv_scales, uint8_t *const *recv_tab, uint8_t *const *scales_tab,
+                         long num_tok, cudaStream_t stream) {
+  cudaError_t launched;
+  const dim3 sg(static_cast<unsigned>(p.num_tiles)), sb(kLLScanThreads);
+  const bool shard = p.rsi_tab != nullptr;
+  if (p.K > 8)
+    launched = shard ? launch_pdl(ll_scan_kernel<16, true>, sg, sb, 0, stream, p)
+                     : launch_pdl(ll_scan_kernel<16, false>, sg, sb, 0, stream, p);
+  else
+    launched = shard ? launch_pdl(ll_scan_kernel<8, true>, sg, sb, 0, stream, p)
+                     : launch_pdl(ll_scan_kernel<8, false>, sg, sb, 0, stream, p);
+  if (launch_status(launched) != EP_OK) return EP_ERR_CUDA;
+
+  const bool tab = recv_tab != nullptr;
+  const size_t smem = spread_smem(static_cast<size_t>(plan.bytes), kLLMaxCtasPerSm);
+  const void *fn =
+      use_fp8 ? (tab ? reinterpret_cast<const void *>(ll_dispatch_kernel<true, true>)
+                     : reinterpret_cast<const void *>(ll_dispatch_kernel<true, false>))
+              : (tab ? reinterpret_cast<const void *>(ll_dispatch_kernel<false, true>)
+                     : reinterpret_cast<const void *>(ll_dispatch_kernel<false, false>));
+  if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
+  const long grid = std::min<long>(
+      num_tok,
+      static_cast<long>(std::min(kLLMaxCtasPerSm, ctas_per_sm(fn, kLLThreads, smem))) *
+          num_sms());
+  const dim3 g(static_cast<unsigned>(grid)), b(kLLThreads);
+  const uint8_t *xb = static_cast<const uint8_t *>(x);
+  uint8_t *rx = static_cast<uint8_t *>(recv_x);
+  uint32_t *claim = &p.head->claim;
+  const unsigned long long to = p.timeout_ns;
+  if (use_fp8 && tab)
+    launched = launch_pdl(ll_dispatch_kernel<true, true>, g, b, smem, stream, xb, p.topk_idx,
+                          p.pos_mirror, num_tok, H, p.K, p.E, p.cap, round_scale, ue8m0, plan,
+                          rx, recv_scales, claim, p.status, to, recv_tab, scales_tab, p.El);
+  else if (use_fp8)
+    launched = launch_pdl(ll_dispatch_kernel<true, false>, g, b, smem, stream, xb, p.topk_idx,
+                          p.pos_mirror, num_tok, H, p.K, p.E, p.cap, round_scale, ue8m0, plan,
+                          rx, recv_scales, claim, p.status, to,
+                          static_cast<uint8_t *const *>(nullptr),
+                          static_cast<uint8_t *const *>(nullptr), p.El);
+  else if (tab)
+    launched = launch_pdl(ll_dispatch_kernel<false, true>, g, b, smem, stream, xb, p.topk_idx,
+                          p.pos_mirror, num_tok, H, p.K, p.E, p.cap, 0, 0, plan, rx,
+                          static_cast<void *>(nullptr), claim, p.status, to, recv_tab,
+                          static_cast<uint8_t *const *>(nullptr), p.El);
+  else
+    launched = launch_pdl(ll_dispatch_kernel<false, false>, g, b, smem, stream, xb, p.topk_idx,
+                          p.pos_mirror, num_tok, H, p.K, p.E, p.cap, 0, 0, plan, rx,
+                          static_cast<void *>(nullptr), claim, p.status, to,
+                          static_cast<uint8_t *const *>(nullptr),
+                          static_cast<uint8_t *const *>(nullptr), p.El);
+  return launch_status(launched);
 }
 }  // namespace
 }  // namespace ep
@@ -783,6 +995,9 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   LLScanParams p;
+  p.s0 = 0;
+  p.base = nullptr;
+  p.rsi_tab = nullptr;
   p.topk_idx = topk_idx;
   p.mask = rank_mask;
   p.stats = cumulative_local_expert_recv_stats;
@@ -805,39 +1020,8 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   const WaitConfig wc = wait_config();
   p.timeout_ns = wc.timeout_ns;
   p.flags = wc.flags;
-  cudaError_t launched;
-  if (K > 8)
-    launched = launch_pdl(ll_scan_kernel<16>,
-        dim3(static_cast<unsigned>(num_tiles)), dim3(kLLScanThreads), 0, stream,
-        p);
-  else
-    launched = launch_pdl(ll_scan_kernel<8>,
-        dim3(static_cast<unsigned>(num_tiles)), dim3(kLLScanThreads), 0, stream,
-        p);
-  if (launch_status(launched) != EP_OK) return EP_ERR_CUDA;
-
-  const size_t smem = spread_smem(static_cast<size_t>(plan.bytes), kLLMaxCtasPerSm);
-  const long num_tok = static_cast<long>(R) * T;
-  const void *fn = use_fp8 ? reinterpret_cast<const void *>(ll_dispatch_kernel<true>)
-                           : reinterpret_cast<const void *>(ll_dispatch_kernel<false>);
-  if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
-  const long grid = std::min<long>(
-      num_tok,
-      static_cast<long>(std::min(kLLMaxCtasPerSm, ctas_per_sm(fn, kLLThreads, smem))) *
-          num_sms());
-  if (use_fp8)
-    launched = launch_pdl(ll_dispatch_kernel<true>,
-        dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
-        static_cast<const uint8_t *>(x), topk_idx, p.pos_mirror, num_tok, H, K, E,
-        static_cast<int>(cap), round_scale, ue8m0, plan, static_cast<uint8_t *>(recv_x),
-        recv_scales, &p.head->claim, status, wc.timeout_ns);
-  else
-    launched = launch_pdl(ll_dispatch_kernel<false>,
-        dim3(static_cast<unsigned>(grid)), dim3(kLLThreads), smem, stream,
-        static_cast<const uint8_t *>(x), topk_idx, p.pos_mirror, num_tok, H, K, E,
-        static_cast<int>(cap), 0, 0, plan, static_cast<uint8_t *>(recv_x), nullptr,
-        &p.head->claim, status, wc.timeout_ns);
-  return launch_status(launched);
+  return ll_scan_and_dispatch(p, x, H, use_fp8, round_scale, ue8m0, plan, recv_x, recv_scales,
+                              nullptr, nullptr, static_cast<long>(R) * T, stream);
 }
 
 extern "C" EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
@@ -858,19 +1042,145 @@ extern "C" EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
     return EP_ERR_INVALID_ARG;
   const long cap = static_cast<long>(R) * T;
   if (cap > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
-  const long num_tok = static_cast<long>(R) * T;
-  const int threads = kLLCombineWarps * 32;
-  const void *fn = reinterpret_cast<const void *>(ll_combine_kernel);
-  const long resident = static_cast<long>(ctas_per_sm(fn, threads, 0)) * num_sms();
-  // split rows into segments until there are >= 4 work items per resident warp
-  const int nvec = H / 8;
-  int nseg = static_cast<int>((4 * resident * kLLCombineWarps + num_tok - 1) / num_tok);
-  nseg = std::max(1, std::min(nseg, std::max(1, nvec / 32)));
-  const long items = num_tok * nseg;
-  const long grid = std::min<long>((items + kLLCombineWarps - 1) / kLLCombineWarps, resident);
-  const cudaError_t launched = launch_pdl(ll_combine_kernel,
-      dim3(static_cast<unsigned>(grid)), dim3(threads), 0, stream,
-      static_cast<const uint8_t *>(y), topk_idx, topk_weights, ll_pos, rank_mask, num_tok, T, H,
-      K, E, static_cast<int>(cap), nseg, static_cast<uint8_t *>(out), status);
-  return launch_status(launched);
+  return ll_combine_launch(static_cast<const uint8_t *>(y), nullptr, 0, topk_idx, topk_weights,
+                           ll_pos, rank_mask, static_cast<long>(R) * T, T, H, K, E, cap, out,
+                           status, stream);
+}
+
+// ---------------------------------------------------------------------------
+// One rank per GPU: the low-latency pair with each rank's tokens on its own
+// GPU and every destination's slabs in that destination's memory.
+
+extern "C" EP_API size_t ep_shard_ll_workspace_bytes(int num_ranks, int num_tokens,
+                                                     int num_experts) {
+  using namespace ep;
+  if (num_ranks < 1 || num_tokens < 0 || num_experts < 1) return 0;
+  // the scan's words for one source rank's tokens, then base[E]
+  return ep_ll_workspace_bytes(1, num_tokens, num_experts) +
+         ((static_cast<size_t>(num_experts) * sizeof(int32_t) + 255) & ~static_cast<size_t>(255));
+}
+
+extern "C" EP_API int ep_shard_ll_counts(const int64_t *topk_idx, const int32_t *rank_mask,
+                                         int rank, int num_ranks, int num_tokens, int num_topk,
+                                         int num_experts, int32_t *counts, int32_t *status,
+                                         cudaStream_t stream) {
+  using namespace ep;
+  const int R = num_ranks, T = num_tokens, K = num_topk, E = num_experts;
+  if (R < 1 || R > kMaxRanks || rank < 0 || rank >= R || T < 0 || K < 1 || K > kMaxTopk ||
+      E < 1 || E > kMaxExperts || E % R != 0 || counts == nullptr ||
+      (T > 0 && topk_idx == nullptr))
+    return EP_ERR_INVALID_ARG;
+  if (zero_prefetch(nullptr, 0, counts, E, topk_idx, static_cast<long>(T) * K * 8, stream) !=
+      EP_OK)
+    return EP_ERR_CUDA;
+  if (T == 0) return EP_OK;
+  return launch_status(launch_pdl(ll_count_kernel, dim3(static_cast<unsigned>((T + 255) / 256)),
+                                  dim3(256), 0, stream, topk_idx, rank_mask, rank, T, K, E, E / R,
+                                  counts, status));
+}
+
+extern "C" EP_API int ep_shard_ll_dispatch(
+    const void *x, const int64_t *topk_idx, const int32_t *rank_mask, const int32_t *counts,
+    int rank, int num_ranks, int num_tokens, int hidden, int num_topk, int num_experts,
+    int fp8_flags, void *const *recv_x_peers, void *const *recv_scales_peers,
+    int32_t *const *recv_src_info_peers, int32_t *const *layout_range_peers, int32_t *recv_count,
+    int32_t *ll_pos, int32_t *cumulative_local_expert_recv_stats, void *workspace,
+    size_t workspace_bytes, int32_t *status, cudaStream_t stream) {
+  using namespace ep;
+  const int R = num_ranks, T = num_tokens, H = hidden, K = num_topk, E = num_experts;
+  const int use_fp8 = (fp8_flags & EP_LL_FP8) != 0;
+  const int round_scale = (fp8_flags & EP_LL_ROUND_SCALE) != 0;
+  const int ue8m0 = (fp8_flags & EP_LL_UE8M0) != 0;
+  if ((fp8_flags & ~(EP_LL_FP8 | EP_LL_ROUND_SCALE | EP_LL_UE8M0)) != 0 ||
+      (round_scale && !use_fp8) || (ue8m0 && !round_scale))
+    return EP_ERR_INVALID_ARG;
+  if (R < 1 || R > kMaxRanks || rank < 0 || rank >= R || T < 0 || K < 1 || K > kMaxTopk ||
+      E < 1 || E > kMaxExperts || E % R != 0 || H < 8 ||
+      (use_fp8 ? (H % 128 != 0) : (H % 8 != 0)))
+    return EP_ERR_INVALID_ARG;
+  if (counts == nullptr || layout_range_peers == nullptr || recv_count == nullptr)
+    return EP_ERR_INVALID_ARG;
+  if (T > 0 && (x == nullptr || topk_idx == nullptr || recv_x_peers == nullptr ||
+                recv_src_info_peers == nullptr || ll_pos == nullptr ||
+                (use_fp8 && recv_scales_peers == nullptr)))
+    return EP_ERR_INVALID_ARG;
+  if (x != nullptr && (reinterpret_cast<uintptr_t>(x) & 15u)) return EP_ERR_INVALID_ARG;
+  if (cumulative_local_expert_recv_stats != nullptr &&
+      (reinterpret_cast<uintptr_t>(cumulative_local_expert_recv_stats) & 3u))
+    return EP_ERR_INVALID_ARG;
+  const size_t need = ep_shard_ll_workspace_bytes(R, T, E);
+  if (workspace == nullptr || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 15u))
+    return EP_ERR_INVALID_ARG;
+  const long cap = static_cast<long>(R) * T;
+  if (cap > 0x7ffffffdL) return EP_ERR_UNSUPPORTED;  // mirror words hold ll_pos + 2
+  const LLSmem plan = ll_smem_plan(H);
+  if (plan.stages < 2) return EP_ERR_UNSUPPORTED;
+  const int tiles = (T + kScanTile - 1) / kScanTile;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int32_t *base = reinterpret_cast<int32_t *>(ws + ep_ll_workspace_bytes(1, T, E));
+  // header, descriptors and this call's mirror words start at zero
+  const size_t used = ll_mirror_offset(tiles, E) + static_cast<size_t>(T) * K * sizeof(int32_t);
+  if (zero_prefetch(workspace, (used + 15) & ~static_cast<size_t>(15), nullptr, 0, topk_idx,
+                    static_cast<long>(T) * K * 8, stream) != EP_OK)
+    return EP_ERR_CUDA;
+  if (launch_status(launch_pdl(shard_ll_prefix_kernel, dim3(static_cast<unsigned>((E + 255) / 256)),
+                               dim3(256), 0, stream, counts, rank, R, E, E / R, base,
+                               layout_range_peers, recv_count,
+                               cumulative_local_expert_recv_stats)) != EP_OK)
+    return EP_ERR_CUDA;
+  if (T == 0) return EP_OK;
+
+  LLScanParams p;
+  p.s0 = rank;
+  p.base = base;
+  p.rsi_tab = recv_src_info_peers;
+  p.topk_idx = topk_idx;
+  p.mask = rank_mask;
+  p.stats = nullptr;
+  p.El = E / R;
+  p.R = R;
+  p.T = T;
+  p.K = K;
+  p.E = E;
+  p.cap = static_cast<int>(cap);
+  p.tiles_per_src = tiles;
+  p.num_tiles = tiles;  // one source rank
+  p.ll_pos = ll_pos;
+  p.recv_src_info = nullptr;
+  p.layout_range = nullptr;
+  p.recv_count = nullptr;
+  p.head = reinterpret_cast<ScanHeader *>(ws);
+  p.desc = reinterpret_cast<uint64_t *>(ws + sizeof(ScanHeader));
+  p.pos_mirror = reinterpret_cast<int32_t *>(ws + ll_mirror_offset(tiles, E));
+  p.status = status;
+  const WaitConfig wc = wait_config();
+  p.timeout_ns = wc.timeout_ns;
+  p.flags = wc.flags;
+  return ll_scan_and_dispatch(p, x, H, use_fp8, round_scale, ue8m0, plan, nullptr, nullptr,
+                              reinterpret_cast<uint8_t *const *>(recv_x_peers),
+                              reinterpret_cast<uint8_t *const *>(recv_scales_peers), T, stream);
+}
+
+extern "C" EP_API int ep_shard_ll_combine(const void *const *y_peers, const int64_t *topk_idx,
+                                          const float *topk_weights, const int32_t *ll_pos,
+                                          const int32_t *rank_mask, int rank, int num_ranks,
+                                          int num_tokens, int hidden, int num_topk,
+                                          int num_experts, void *out, int32_t *status,
+                                          cudaStream_t stream) {
+  using namespace ep;
+  const int R = num_ranks, T = num_tokens, H = hidden, K = num_topk, E = num_experts;
+  if (R < 1 || R > kMaxRanks || rank < 0 || rank >= R || T < 0 || K < 1 || K > kMaxTopk ||
+      E < 1 || E > kMaxExperts || E % R != 0 || H < 8 || H % 8 != 0)
+    return EP_ERR_INVALID_ARG;
+  if (T == 0) return EP_OK;
+  if (y_peers == nullptr || topk_idx == nullptr || topk_weights == nullptr ||
+      ll_pos == nullptr || out == nullptr)
+    return EP_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(out) & 15u) return EP_ERR_INVALID_ARG;
+  const long cap = static_cast<long>(R) * T;
+  if (cap > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
+  return ll_combine_launch(nullptr, reinterpret_cast<const uint8_t *const *>(y_peers), rank,
+                           topk_idx, topk_weights, ll_pos, rank_mask, T, T, H, K, E, cap, out,
+                           status, stream);
 }

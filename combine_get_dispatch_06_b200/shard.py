@@ -12,7 +12,9 @@ counts into the same rank prefix matrix.
 This module is argument marshalling and the control plane only -- the layout,
 prefix matrix, positions, row moves and reduction run in the library's
 kernels (``ep_get_dispatch_layout``, ``ep_shard_notify``,
-``ep_shard_dispatch``, ``ep_shard_combine``).  The process group carries the
+``ep_shard_dispatch``, ``ep_shard_combine``; for the low-latency pair
+``ep_shard_ll_counts``, ``ep_shard_ll_dispatch``, ``ep_shard_ll_combine``,
+whose per-expert counts are all-gathered the same way).  The process group carries the
 IPC handles, the count rows and the synchronisation between phases: with an
 NCCL group the counts are gathered on the device and the synchronisation is
 a one-element all-reduce on the current stream (no host round trip); with a
@@ -33,7 +35,8 @@ from typing import Optional
 import torch
 import torch.distributed as dist
 
-from . import (EPError, _check, _lib, _need, _ptr, ep_get_dispatch_layout, new_status)
+from . import (EP_LL_FP8, EP_LL_ROUND_SCALE, EP_LL_UE8M0, EPError, _check, _lib, _need, _ptr,
+               ep_get_dispatch_layout, new_status)
 
 IPC_HANDLE_BYTES = 64
 _ALIGN = 256
@@ -53,6 +56,31 @@ def region_layout(capacity: int, hidden: int, num_topk: int, expert_outputs: boo
              ("recv_src_idx", (cap,), torch.int32, 4)]
     if expert_outputs:
         parts.append(("y", (cap, H), torch.bfloat16, 2))
+    return _pack(parts)
+
+
+def ll_region_layout(num_ranks: int, num_tokens: int, hidden: int, local_experts: int,
+                     use_fp8: bool = True, ue8m0: bool = False) -> dict:
+    """The low-latency region of one rank (destination of its E_l experts):
+    slabs [E_l, R*T, H] (e4m3 bytes or bf16), FP8 scales [E_l, R*T, H/128]
+    (fp32, or UE8M0 bytes), recv_src_info [E_l, R*T], layout_range
+    [E_l, R, 2] and the experts' output slabs ``ll_y`` [E_l, R*T, H] bf16
+    that combine reads (legacy-test page, low_latency_dispatch outputs and
+    low_latency_combine input)."""
+    cap, H, El = num_ranks * num_tokens, hidden, local_experts
+    parts = [("ll_recv_x", (El, cap, H), torch.uint8 if use_fp8 else torch.bfloat16,
+              1 if use_fp8 else 2)]
+    if use_fp8:
+        parts.append(("ll_recv_scales", (El, cap, H // 128),
+                      torch.uint8 if ue8m0 else torch.float32, 1 if ue8m0 else 4))
+    parts += [("ll_recv_src_info", (El, cap), torch.int32, 4),
+              ("ll_layout_range", (El, num_ranks, 2), torch.int32, 4),
+              ("ll_y", (El, cap, H), torch.bfloat16, 2)]
+    return _pack(parts)
+
+
+def _pack(parts) -> dict:
+    """Consecutive 256-byte-aligned parts: name -> (offset, shape, dtype)."""
     out, off = {}, 0
     for name, shape, dtype, size in parts:
         n = size
@@ -128,33 +156,12 @@ class ShardedBuffer:
             else torch.device(device)
         self.nccl = dist.get_backend(group) == "nccl"
         self.layout = region_layout(self.cap, self.H, self.K, expert_outputs)
-        self._base = None
-        self._peers = []
+        self._bases = []   # this rank's regions (freed at close)
+        self._peers = []   # peers' regions mapped here (unmapped at close)
+        self.tables, self.buffers = {}, {}
+        self._ll = None
         with torch.cuda.device(self.device):
-            p = ctypes.c_void_p()
-            _check(_lib.ep_shard_alloc(self.layout["_bytes"], ctypes.byref(p)), "ep_shard_alloc")
-            self._base = p.value
-            h = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
-            _check(_lib.ep_ipc_handle(self._base, h), "ep_ipc_handle")
-            handles = exchange_handles(h.raw, group)
-            bases = []
-            for r, hr in enumerate(handles):
-                if r == self.rank:
-                    bases.append(self._base)
-                    continue
-                q = ctypes.c_void_p()
-                _check(_lib.ep_ipc_open(ctypes.create_string_buffer(hr, IPC_HANDLE_BYTES),
-                                        ctypes.byref(q)), "ep_ipc_open")
-                self._peers.append(q.value)
-                bases.append(q.value)
-            # peer tables: entry d = rank d's buffer of each kind, in this process
-            parts = {k: v for k, v in self.layout.items() if not k.startswith("_")}
-            self.tables = {name: torch.tensor([b + off for b in bases], dtype=torch.int64,
-                                              device=self.device)
-                           for name, (off, _, _) in parts.items()}
-            # this rank's buffers, as tensors
-            self.buffers = {name: _view(self._base + off, shape, dtype, self.device)
-                            for name, (off, shape, dtype) in parts.items()}
+            self._share(self.layout)
             R, T, E = self.R, self.T, self.E
             dev = self.device
             self.send_pos = torch.empty((T, R), dtype=torch.int32, device=dev)
@@ -171,6 +178,36 @@ class ShardedBuffer:
             self.status = new_status(dev)
             self._one = torch.ones((1,), dtype=torch.int32, device=dev)
         self.sync()
+
+    def _share(self, layout: dict) -> None:
+        """Allocate this rank's region of `layout`, exchange IPC handles over
+        the group (collective) and map every peer's region; adds one peer
+        table and one local tensor per part."""
+        p = ctypes.c_void_p()
+        _check(_lib.ep_shard_alloc(layout["_bytes"], ctypes.byref(p)), "ep_shard_alloc")
+        base = p.value
+        self._bases.append(base)
+        h = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+        _check(_lib.ep_ipc_handle(base, h), "ep_ipc_handle")
+        handles = exchange_handles(h.raw, self.group)
+        bases = []
+        for r, hr in enumerate(handles):
+            if r == self.rank:
+                bases.append(base)
+                continue
+            q = ctypes.c_void_p()
+            _check(_lib.ep_ipc_open(ctypes.create_string_buffer(hr, IPC_HANDLE_BYTES),
+                                    ctypes.byref(q)), "ep_ipc_open")
+            self._peers.append(q.value)
+            bases.append(q.value)
+        parts = {k: v for k, v in layout.items() if not k.startswith("_")}
+        # peer tables: entry d = rank d's buffer of each kind, in this process
+        self.tables.update({name: torch.tensor([b + off for b in bases], dtype=torch.int64,
+                                               device=self.device)
+                            for name, (off, _, _) in parts.items()})
+        # this rank's buffers, as tensors
+        self.buffers.update({name: _view(base + off, shape, dtype, self.device)
+                             for name, (off, shape, dtype) in parts.items()})
 
     # ---- cross-rank ordering -------------------------------------------------
 
@@ -258,10 +295,109 @@ class ShardedBuffer:
         self.sync()
         return combined_x, (combined_topk_weights if with_weights else None)
 
+    # ---- the low-latency pair ------------------------------------------------
+
+    def enable_low_latency(self, use_fp8: bool = True, use_ue8m0: bool = False) -> None:
+        """Allocate and map this rank's low-latency region (collective: every
+        rank calls it): the slabs of its E_l experts for every source rank's
+        T tokens, their scales and handle, and the experts' output slabs."""
+        if self._ll is not None:
+            return
+        if use_ue8m0 and not use_fp8:
+            raise EPError("UE8M0 scales need the FP8 payload")
+        R, T, E, El = self.R, self.T, self.E, self.El
+        dev = self.device
+        with torch.cuda.device(dev):
+            self._share(ll_region_layout(R, T, self.H, El, use_fp8, use_ue8m0))
+            self._ll = {
+                "use_fp8": use_fp8, "ue8m0": use_ue8m0,
+                "counts": torch.empty((E,), dtype=torch.int32, device=dev),
+                "recv_count": torch.empty((El,), dtype=torch.int32, device=dev),
+                "ll_pos": torch.empty((T, self.K), dtype=torch.int32, device=dev),
+                "workspace": torch.empty(
+                    max(int(_lib.ep_shard_ll_workspace_bytes(R, T, E)), 16), dtype=torch.uint8,
+                    device=dev),
+            }
+        self.sync()
+
+    def ll_dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, round_scale: bool = False,
+                    rank_mask: Optional[torch.Tensor] = None,
+                    cumulative_local_expert_recv_stats: Optional[torch.Tensor] = None) -> dict:
+        """x bf16 [T, H], topk_idx int64 [T, K] -> this rank's slabs (as the
+        destination of its E_l experts: rows below recv_count[j] are valid once
+        every rank has dispatched; this call synchronises the ranks at its end)
+        and ll_pos of its own tokens.  The per-expert counts travel by an
+        all-gather (the notify exchange of the low-latency pair)."""
+        if self._ll is None:
+            raise EPError("call enable_low_latency() first")
+        L = self._ll
+        R, T, H, K, E, El = self.R, self.T, self.H, self.K, self.E, self.El
+        _need(x, torch.bfloat16, (T, H), "x")
+        _need(topk_idx, torch.int64, (T, K), "topk_idx")
+        if rank_mask is not None:
+            _need(rank_mask, torch.int32, (R,), "rank_mask")
+        if cumulative_local_expert_recv_stats is not None:
+            _need(cumulative_local_expert_recv_stats, torch.int32, (El,),
+                  "cumulative_local_expert_recv_stats")
+        if round_scale and not L["use_fp8"]:
+            raise EPError("round_scale needs the FP8 payload")
+        flags = (EP_LL_FP8 if L["use_fp8"] else 0) | \
+            (EP_LL_ROUND_SCALE if round_scale or L["ue8m0"] else 0) | \
+            (EP_LL_UE8M0 if L["ue8m0"] else 0)
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        t = self.tables
+        with torch.cuda.device(self.device):
+            rc = _lib.ep_shard_ll_counts(_ptr(topk_idx), _ptr(rank_mask), self.rank, R, T, K, E,
+                                         _ptr(L["counts"]), _ptr(self.status), stream)
+            _check(rc, "ep_shard_ll_counts")
+            counts = allgather_rows(L["counts"], self.group)     # [R, E]
+            rc = _lib.ep_shard_ll_dispatch(
+                _ptr(x), _ptr(topk_idx), _ptr(rank_mask), _ptr(counts), self.rank, R, T, H, K, E,
+                flags, _ptr(t["ll_recv_x"]),
+                _ptr(t["ll_recv_scales"]) if L["use_fp8"] else None,
+                _ptr(t["ll_recv_src_info"]), _ptr(t["ll_layout_range"]), _ptr(L["recv_count"]),
+                _ptr(L["ll_pos"]), _ptr(cumulative_local_expert_recv_stats),
+                _ptr(L["workspace"]), L["workspace"].numel(), _ptr(self.status), stream)
+            _check(rc, "ep_shard_ll_dispatch")
+        self.sync()
+        b = self.buffers
+        return {"recv_x": b["ll_recv_x"], "recv_scales": b.get("ll_recv_scales"),
+                "recv_src_info": b["ll_recv_src_info"], "layout_range": b["ll_layout_range"],
+                "recv_count": L["recv_count"], "ll_pos": L["ll_pos"],
+                "expert_outputs": b["ll_y"]}
+
+    def ll_combine(self, topk_idx: torch.Tensor, topk_weights: torch.Tensor,
+                   rank_mask: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """Gather this rank's tokens' rows back from the destinations' expert
+        output slabs (``ll_y``, written by the experts after ll_dispatch) and
+        take their top-k weighted sum.  Synchronises the ranks before and
+        after."""
+        if self._ll is None:
+            raise EPError("call enable_low_latency() first")
+        R, T, H, K, E = self.R, self.T, self.H, self.K, self.E
+        _need(topk_idx, torch.int64, (T, K), "topk_idx")
+        _need(topk_weights, torch.float32, (T, K), "topk_weights")
+        if rank_mask is not None:
+            _need(rank_mask, torch.int32, (R,), "rank_mask")
+        if out is None:
+            out = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
+        _need(out, torch.bfloat16, (T, H), "out")
+        stream = torch.cuda.current_stream(self.device).cuda_stream
+        self.sync()
+        with torch.cuda.device(self.device):
+            rc = _lib.ep_shard_ll_combine(_ptr(self.tables["ll_y"]), _ptr(topk_idx),
+                                          _ptr(topk_weights), _ptr(self._ll["ll_pos"]),
+                                          _ptr(rank_mask), self.rank, R, T, H, K, E, _ptr(out),
+                                          _ptr(self.status), stream)
+            _check(rc, "ep_shard_ll_combine")
+        self.sync()
+        return out
+
     def close(self) -> None:
         """Unmap the peers' buffers and free this rank's (after a final
         synchronisation, so no peer still reads or writes it)."""
-        if self._base is None:
+        if not self._bases:
             return
         self.sync()
         torch.cuda.synchronize(self.device)
@@ -271,7 +407,8 @@ class ShardedBuffer:
             self._peers = []
             self.buffers = {}
             self.tables = {}
-        dist.barrier(group=self.group)   # every rank has unmapped this rank's buffer
+        dist.barrier(group=self.group)   # every rank has unmapped this rank's buffers
         with torch.cuda.device(self.device):
-            _check(_lib.ep_shard_free(self._base), "ep_shard_free")
-        self._base = None
+            for b in self._bases:
+                _check(_lib.ep_shard_free(b), "ep_shard_free")
+        self._bases = []

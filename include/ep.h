@@ -522,6 +522,78 @@ EP_API int ep_shard_combine(const void *const *y_peers,
                             void *combined_x, float *combined_topk_weights,
                             int32_t *status, cudaStream_t stream);
 
+/* --------------------------------------------------------------------------
+ * The low-latency pair, one rank per GPU.
+ *
+ * Passage: the legacy-test page's low_latency_dispatch / low_latency_combine
+ * (per-expert slabs [E_l, R * T, H], the handle (recv_src_info,
+ * recv_layout_range), per-expert counts) and, for the exchange, the sharding
+ * of the Buffer as above.  Each process holds source rank `rank`'s T tokens
+ * and, as destination `rank`, the slabs of its E_l = E / R experts:
+ *   1. ep_shard_ll_counts: counts[E] = rows this rank sends to each expert;
+ *   2. the caller all-gathers them into counts [R, E];
+ *   3. ep_shard_ll_dispatch: positions, quantised rows and handle entries
+ *      written into every destination's slabs (through the peer tables);
+ *   4. a cross-rank synchronisation by the caller; experts run on their slabs;
+ *   5. ep_shard_ll_combine: each rank reads its tokens' rows back from the
+ *      destinations' expert-output slabs and takes the weighted sum.
+ * Every output equals the single-GPU ep_ll_dispatch / ep_ll_combine on the
+ * stacked inputs, restricted to the rank: ll_pos rows of source `rank`, the
+ * slab rows, recv_src_info and layout_range of destination d in d's memory,
+ * recv_count of the rank's own experts.  Slab rows are ordered by source rank,
+ * then token, so rank r's rows of expert e follow those of ranks 0..r-1.
+ *
+ * Peer tables are device arrays of R device pointers, entry d = rank d's
+ * buffer mapped in this process: recv_x_peers [R] -> e4m3 or bf16 [E_l, R*T, H];
+ * recv_scales_peers [R] -> fp32 or UE8M0 bytes [E_l, R*T, H/128] (FP8 only);
+ * recv_src_info_peers [R] -> int32 [E_l, R*T]; layout_range_peers [R] ->
+ * int32 [E_l, R, 2]; y_peers [R] -> bf16 [E_l, R*T, H].  Nothing here waits
+ * for another rank's kernels.  rank_mask: as in ep_ll_dispatch (nullable).
+ * ========================================================================== */
+
+/* counts [E] int32, written (zeroed first) with this rank's rows per expert:
+ * its tokens whose distinct valid slots hold the expert, none if `rank`
+ * fails, none to a failed rank's experts.  topk_idx [T, K] int64. */
+EP_API int ep_shard_ll_counts(const int64_t *topk_idx, const int32_t *rank_mask,
+                              int rank, int num_ranks, int num_tokens,
+                              int num_topk, int num_experts, int32_t *counts,
+                              int32_t *status, cudaStream_t stream);
+
+/* Workspace bytes of ep_shard_ll_dispatch (any content). */
+EP_API size_t ep_shard_ll_workspace_bytes(int num_ranks, int num_tokens,
+                                          int num_experts);
+
+/* x bf16 [T, H] (16-byte aligned), topk_idx int64 [T, K], counts int32
+ * [R, E] (every rank's ep_shard_ll_counts, in rank order).  fp8_flags as in
+ * ep_ll_dispatch.  Writes through the peer tables (see above); locally
+ * recv_count int32 [E_l] (rows received by this rank's experts), ll_pos int32
+ * [T, K] (slab row of each slot, -1 when dropped) and, if non-null,
+ * cumulative_local_expert_recv_stats int32 [E_l] += recv_count.  Returns
+ * before anything is launched on a bad argument. */
+EP_API int ep_shard_ll_dispatch(const void *x, const int64_t *topk_idx,
+                                const int32_t *rank_mask, const int32_t *counts,
+                                int rank, int num_ranks, int num_tokens,
+                                int hidden, int num_topk, int num_experts,
+                                int fp8_flags, void *const *recv_x_peers,
+                                void *const *recv_scales_peers,
+                                int32_t *const *recv_src_info_peers,
+                                int32_t *const *layout_range_peers,
+                                int32_t *recv_count, int32_t *ll_pos,
+                                int32_t *cumulative_local_expert_recv_stats,
+                                void *workspace, size_t workspace_bytes,
+                                int32_t *status, cudaStream_t stream);
+
+/* out bf16 [T, H] (16-byte aligned): for each token, sum over its slots k in
+ * ascending order of fmaf(y[row of slot k], topk_weights[k], acc), one bf16
+ * rounding, where the rows are read from y_peers (the destinations'
+ * expert-output slabs) at ll_pos.  topk_weights fp32 [T, K]. */
+EP_API int ep_shard_ll_combine(const void *const *y_peers, const int64_t *topk_idx,
+                               const float *topk_weights, const int32_t *ll_pos,
+                               const int32_t *rank_mask, int rank, int num_ranks,
+                               int num_tokens, int hidden, int num_topk,
+                               int num_experts, void *out, int32_t *status,
+                               cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
