@@ -30,6 +30,7 @@ import subprocess
 import sys
 import tempfile
 import time
+from typing import Optional
 
 import numpy as np
 
@@ -728,6 +729,65 @@ def shard_bytes(R, T, H, K, N):
     return disp, comb
 
 
+def sharded_ll(args, device, rank: int, ws: int, timed) -> Optional[dict]:
+    """The low-latency pair with one rank per GPU, at the LL workload's shape
+    per rank (T = 128 tokens, H = 7168, top-8 of 256 experts, FP8): counts
+    exchange, dispatch into the destinations' slabs, identity experts (the
+    output slabs are left as they are), combine.  Timed like the normal step
+    (CUDA-graph replay when the capture works); None when the experts do not
+    divide over the ranks."""
+    import torch
+    import torch.distributed as dist
+
+    from combine_get_dispatch_06_b200.shard import ShardedBuffer
+
+    w0 = CONFIGS["ll"]
+    if w0.E % ws != 0:
+        return None
+    w = Workload("ll_sharded", R=ws, T=w0.T, H=w0.H, E=w0.E, K=w0.K, seed=w0.seed)
+    inp = make(w, ranks=[rank])
+    x = to_dev_bf16(inp["x"][0], device)
+    idx = torch.from_numpy(inp["topk_idx"][0]).to(device)
+    wt = torch.from_numpy(inp["topk_weights"][0]).to(device)
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device=device)
+    buf = ShardedBuffer(dist.group.WORLD, w.T, w.H, w.K, w.E, device=device)
+    buf.enable_low_latency(use_fp8=True)
+
+    def step():
+        buf.ll_dispatch(x, idx)
+        buf.ll_combine(idx, wt, out=out)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    if int(buf.status.item()) != 0:
+        raise RuntimeError(f"device status {int(buf.status.item())} in the LL warm-up")
+    C = int(buf._ll["counts"].sum().item())          # rows this rank sends
+    nbytes = ll_dispatch_bytes(1, w.T, w.H, w.K, C) + ll_combine_bytes(1, w.T, w.H, w.K, C)
+    graph, note = None, None
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        torch.cuda.synchronize(device)
+        graph = g
+    except Exception as e:  # capture refused: time the eager pair only
+        note = f"capture failed: {type(e).__name__}: {str(e)[:200]}"
+        torch.cuda.synchronize(device)
+    ms = timed(graph.replay) if graph is not None else timed(step)
+    agg = aggregate(nbytes, w.T, ms, device)
+    if int(buf.status.item()) != 0:
+        raise RuntimeError(f"device status {int(buf.status.item())} in the LL timed region")
+    del graph
+    torch.cuda.synchronize(device)
+    buf.close()
+    return {"workload": f"low latency, one rank per GPU: R={ws} x T={w.T} tokens x H={w.H}, "
+                        f"E={w.E}, top-{w.K}, FP8 dispatch, weighted combine",
+            "us_per_step": agg["ms_per_step"] * 1e3, "gbs": agg["gbs"],
+            "tokens_per_s": agg["tokens_per_s"], "cuda_graph": note is None,
+            "cuda_graph_note": note}
+
+
 def run_sharded(args) -> None:
     """The normal workload with one rank per GPU: rank r holds its own T
     tokens, writes their rows into the destination GPUs' receive buffers
@@ -838,6 +898,7 @@ def run_sharded(args) -> None:
     probe = buf.notify_probe.cpu().numpy().astype(np.uint64)
     starts = [None] * ws
     dist.all_gather_object(starts, int(probe[2]))
+    low_latency = sharded_ll(args, device, rank, ws, timed)
 
     line = {
         "metric": METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
@@ -863,6 +924,7 @@ def run_sharded(args) -> None:
         "cuda_graph": graph is not None, "cuda_graph_note": graph_note,
         "eager": {"ms_per_step": eager["ms_per_step"], "value": eager["gbs"]},
         "clocks": clocks,
+        "low_latency": low_latency,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
