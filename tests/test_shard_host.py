@@ -1,4 +1,4 @@
-"""The sharded path's control plane on CPU ranks (gloo, world size 2 and 4).
+"""The sharded paths' control plane on CPU ranks (gloo, world size 2 and 4).
 
 Each rank takes its own source rank's layout (the oracle's, on the CPU), and
 the rows every rank all-gathers must be the single-GPU layout's rows in rank
@@ -8,7 +8,10 @@ rows give the oracle's per-expert receive counts of every destination
 (legacy-test analysis page, the inclusive recv_gbl_rank_prefix_sum that
 check_data walks; Python接口 page, num_recv_tokens_per_expert_list).  IPC
 handles come back in rank order and every rank computes the same layout of
-the shared region.
+the shared region.  For the low-latency pair, the gathered per-expert rows
+of every rank add up to the oracle's receive counts, and their prefix over
+earlier ranks is the first row of each rank's block in the oracle's
+layout_range (legacy-test page, the low_latency_dispatch handle).
 """
 import datetime
 import os
@@ -55,10 +58,14 @@ def _worker(rank, world, port, q):
         mine = oracle.layout(idx[rank:rank + 1], w.E, w.R)     # this rank's own tokens
         counts = allgather_rows(torch.from_numpy(mine["num_tokens_per_rank"][0]))
         ecounts = allgather_rows(torch.from_numpy(mine["num_tokens_per_expert"][0]))
+        # the low-latency pair's exchange: rows this rank sends to each expert
+        ll_mine = oracle.ll_layout(idx[rank:rank + 1], w.E)["recv_count"].reshape(w.E)
+        llcounts = allgather_rows(torch.from_numpy(ll_mine))
         handles = exchange_handles(bytes([rank + 1]) * 64)
         lay = region_layout(w.R * w.T, 64, w.K, True)
         q.put((rank, counts.numpy(), ecounts.numpy(), handles,
-               {k: (v if k == "_bytes" else (v[0], v[1], str(v[2]))) for k, v in lay.items()}))
+               {k: (v if k == "_bytes" else (v[0], v[1], str(v[2]))) for k, v in lay.items()},
+               llcounts.numpy()))
     finally:
         dist.destroy_process_group()
 
@@ -87,8 +94,18 @@ def test_count_exchange_gives_the_oracle_prefix_matrix(world):
     nrte = oracle.expert_recv_counts(full["num_tokens_per_expert"], w.R)
     El = w.E // w.R
     layouts = set()
+    llref = oracle.ll_layout(idx, w.E)
     for rank in range(world):
-        counts, ecounts, handles, lay = got[rank]
+        counts, ecounts, handles, lay, llcounts = got[rank]
+        # the sharded LL prefix: rows of each expert from earlier ranks are the
+        # first row of that rank's block in the destination's layout_range
+        # (legacy-test page, low_latency_dispatch handle), and every rank's
+        # rows add up to the expert's receive count
+        np.testing.assert_array_equal(llcounts.sum(axis=0), llref["recv_count"].reshape(w.E))
+        before = np.cumsum(llcounts, axis=0) - llcounts                      # [R, E]
+        lr = llref["layout_range"].reshape(w.E, w.R, 2)
+        np.testing.assert_array_equal(before.T, lr[:, :, 0])
+        np.testing.assert_array_equal(llcounts.T, lr[:, :, 1])
         np.testing.assert_array_equal(counts, full["num_tokens_per_rank"])
         np.testing.assert_array_equal(np.cumsum(counts, axis=0), pre["rank_prefix_matrix"])
         np.testing.assert_array_equal(np.cumsum(counts, axis=0)[-1], pre["recv_count"])
