@@ -12,7 +12,9 @@ and its per-expert count check).  The experts then write the dequantised
 rows into the shared output slabs and each rank's weighted combine is
 compared with the oracle's (legacy-test page, low_latency_combine).  A second
 step on new inputs, with rank 1 marked failed, reuses the buffers and adds to
-the cumulative per-expert counter.
+the cumulative per-expert counter.  A second test covers the other payloads:
+bf16 rows with sixteen slots (and their combine), and e4m3 rows with UE8M0
+scales (round_scale), each slab row against the oracle's quantiser.
 """
 import datetime
 import os
@@ -151,3 +153,117 @@ def test_two_ranks_low_latency_on_one_gpu_match_the_oracle():
             assert (ref["recv_count"][1] == 0).all()
     for r in range(world):
         np.testing.assert_array_equal(got[r][1], total[r])
+
+
+# ---------------------------------------------------------------------------
+# the other payloads: bf16 rows with sixteen slots, and FP8 with UE8M0 scales
+# ---------------------------------------------------------------------------
+
+def _cases():
+    from workloads import Workload
+    return {"bf16_k16": Workload("sll_c", R=2, T=140, H=256, E=32, K=16, masked_frac=0.05,
+                                 seed=62),
+            "ue8m0": Workload("sll_d", R=2, T=70, H=384, E=16, K=4, seed=63)}
+
+
+def _worker_formats(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    torch.cuda.set_device(0)
+    try:
+        import oracle
+        from combine_get_dispatch_06_b200.shard import ShardedBuffer
+        from tests.helpers import to_dev, to_host
+        from workloads import make
+
+        results = {}
+        for name, w in _cases().items():
+            inp = make(w)
+            x, idx, wts = inp["x"], inp["topk_idx"], inp["topk_weights"]
+            buf = ShardedBuffer(dist.group.WORLD, w.T, w.H, w.K, w.E)
+            bf16 = name == "bf16_k16"
+            buf.enable_low_latency(use_fp8=not bf16, use_ue8m0=not bf16)
+            out = buf.ll_dispatch(to_dev(x[rank]), to_dev(idx[rank]), round_scale=not bf16)
+            torch.cuda.synchronize()
+            res = {k: to_host(out[k]) for k in ("ll_pos", "recv_count", "layout_range",
+                                                "recv_src_info", "recv_x")}
+            res["recv_scales"] = None if bf16 else to_host(out["recv_scales"])
+            if bf16:  # experts return the received rows; combine reads them back
+                ref = oracle.ll_layout(idx, w.E)
+                rq, _ = oracle.ll_dispatch_rows(x, idx, ref["ll_pos"], w.E, use_fp8=False)
+                out["expert_outputs"].copy_(to_dev(rq[rank]))
+                co = buf.ll_combine(to_dev(idx[rank]), to_dev(wts[rank]))
+                torch.cuda.synchronize()
+                res["combined"] = to_host(co)
+            res["status"] = int(buf.status.item())
+            buf.close()
+            results[name] = res
+        q.put((rank, results, None))
+    except Exception:  # report instead of hanging the parent
+        import traceback
+        q.put((rank, None, traceback.format_exc()))
+        raise
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_low_latency_bf16_k16_and_ue8m0_match_the_oracle():
+    sys.path.insert(0, ROOT)
+    import oracle
+    from workloads import make
+
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_formats, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in procs:
+        rank, results, err = q.get(timeout=600)
+        assert err is None, f"rank {rank}:\n{err}"
+        got[rank] = results
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+
+    for name, w in _cases().items():
+        inp = make(w)
+        x, idx, wts = inp["x"], inp["topk_idx"], inp["topk_weights"]
+        ref = oracle.ll_layout(idx, w.E)
+        El = w.E // world
+        bf16 = name == "bf16_k16"
+        if bf16:
+            rq, _ = oracle.ll_dispatch_rows(x, idx, ref["ll_pos"], w.E, use_fp8=False)
+            co = oracle.ll_combine(rq, idx, wts, ref["ll_pos"])
+        for r in range(world):
+            res = got[r][name]
+            assert res["status"] == 0, name
+            np.testing.assert_array_equal(res["ll_pos"], ref["ll_pos"][r])
+            np.testing.assert_array_equal(res["recv_count"], ref["recv_count"][r])
+            np.testing.assert_array_equal(res["layout_range"], ref["layout_range"][r])
+            for j in range(El):
+                n = int(ref["recv_count"][r, j])
+                np.testing.assert_array_equal(res["recv_src_info"][j, :n],
+                                              ref["recv_src_info"][r, j, :n])
+                if bf16:
+                    np.testing.assert_array_equal(res["recv_x"][j, :n], rq[r, j, :n])
+            if bf16:
+                np.testing.assert_array_equal(res["combined"], co[r])
+        if not bf16:  # every slab row against the oracle's quantiser, row by row
+            for s in range(world):
+                for t in range(w.T):
+                    qr, _, ur = oracle.quantize_row_ex(x[s, t], round_scale=True)
+                    for k in range(w.K):
+                        e = int(idx[s, t, k])
+                        if e < 0:
+                            continue
+                        p = int(ref["ll_pos"][s, t, k])
+                        d, j = divmod(e, El)
+                        np.testing.assert_array_equal(got[d][name]["recv_x"][j, p], qr)
+                        np.testing.assert_array_equal(got[d][name]["recv_scales"][j, p], ur)
