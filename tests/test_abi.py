@@ -95,3 +95,46 @@ def test_dispatch_rejects_misaligned_and_missing(lib):
     assert call(idx=None) == 1            # neither topk_idx nor is_token_in_rank
     assert call(align=0) == 1
     assert call(cap=-1) == 1
+
+
+def test_sharded_low_latency_argument_checks(lib):
+    """The sharded low-latency entry points refuse bad arguments on the host:
+    a rank outside [0, R), experts that do not divide over the ranks, FP8
+    flag combinations that do not exist, a short workspace, missing tables."""
+    P, I, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.ep_shard_ll_counts.restype = I
+    lib.ep_shard_ll_counts.argtypes = [P, P, I, I, I, I, I, P, P, P]
+    lib.ep_shard_ll_workspace_bytes.restype = Z
+    lib.ep_shard_ll_workspace_bytes.argtypes = [I, I, I]
+    lib.ep_shard_ll_dispatch.restype = I
+    lib.ep_shard_ll_dispatch.argtypes = [P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, P, P,
+                                         P, Z, P, P]
+    lib.ep_shard_ll_combine.restype = I
+    lib.ep_shard_ll_combine.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P]
+    f = ctypes.c_void_p(256)
+    # counts: rank out of range, E % R != 0, K > 16
+    assert lib.ep_shard_ll_counts(f, None, 2, 2, 8, 4, 16, f, None, None) == 1
+    assert lib.ep_shard_ll_counts(f, None, -1, 2, 8, 4, 16, f, None, None) == 1
+    assert lib.ep_shard_ll_counts(f, None, 0, 3, 8, 4, 16, f, None, None) == 1
+    assert lib.ep_shard_ll_counts(f, None, 0, 2, 8, 17, 16, f, None, None) == 1
+    need = lib.ep_shard_ll_workspace_bytes(2, 8, 16)
+    assert need >= lib.ep_ll_workspace_bytes(1, 8, 16) + 16 * 4
+    ok = dict(x=f, idx=f, mask=None, counts=f, rank=0, R=2, T=8, H=256, K=4, E=16, flags=1,
+              rx=f, rs=f, rsi=f, lr=f, rc=f, pos=f, stats=None, ws=f, wsb=need)
+
+    def disp(**kw):
+        a = dict(ok, **kw)
+        return lib.ep_shard_ll_dispatch(a["x"], a["idx"], a["mask"], a["counts"], a["rank"],
+                                        a["R"], a["T"], a["H"], a["K"], a["E"], a["flags"],
+                                        a["rx"], a["rs"], a["rsi"], a["lr"], a["rc"], a["pos"],
+                                        a["stats"], a["ws"], a["wsb"], None, None)
+
+    assert disp(rank=2) == 1                 # rank outside [0, R)
+    assert disp(flags=4) == 1                # UE8M0 without round_scale
+    assert disp(flags=2) == 1                # round_scale without FP8
+    assert disp(H=200) == 1                  # FP8 needs H % 128 == 0
+    assert disp(wsb=need - 16) == 1          # short workspace
+    assert disp(rs=None) == 1                # FP8 without a scales table
+    assert disp(counts=None) == 1            # no gathered counts
+    assert lib.ep_shard_ll_combine(f, f, f, f, None, 2, 2, 8, 256, 4, 16, f, None, None) == 1
+    assert lib.ep_shard_ll_combine(None, f, f, f, None, 0, 2, 8, 256, 4, 16, f, None, None) == 1
