@@ -7,8 +7,8 @@
 // with the check against x * sum of masked weights):
 //   - one slab row per (token, expert); rows of expert e ordered by source
 //     rank, then token: row = exclusive prefix over the flattened (s, t) order
-//     of "token has e", computed here by the same decoupled look-back scan as
-//     normal dispatch, with experts as the columns;
+//     of "token has e", computed here by a tile scan that looks back over the
+//     earlier tiles' counts, as in normal dispatch, with experts as columns;
 //   - per 128-channel block: amax' = max(max|x|, 1e-4), inv = 448 / amax'
 //     (IEEE division), q = e4m3(x * inv) rounded to nearest even and
 //     saturated (cvt.rn.satfinite), scale = amax' / 448;
@@ -27,6 +27,10 @@
 //                       position
 //   ll_combine_kernel   one warp per (token, channel segment), up to 8 rows
 //                       in flight per lane
+// One rank per GPU (ep_shard_ll_*): ll_count_kernel counts the rank's rows
+// per expert, shard_ll_prefix_kernel turns every rank's counts into its row
+// offsets, its layout_range entries and its experts' receive counts, and the
+// three kernels above run in their peer-table forms.
 #include <algorithm>
 
 #include "ep_scan.cuh"
