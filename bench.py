@@ -564,8 +564,11 @@ def run_ours(args) -> None:
     # ---- timed region: exactly K steps, device-resident inputs ------------
     # The steps run back to back with no event between their kernels, since an
     # event between two programmatically chained launches keeps the second
-    # from starting early.  A second pass of K steps records events around
-    # each phase; the per-kernel times (and the roofline) come from it.
+    # from starting early.  A second pass of K steps runs the same sequence
+    # with the library's full-grid phase timers on (%globaltimer, earliest
+    # block start to last block end of each phase): phases_ms.  A third
+    # records CUDA events around each phase (phases_event_ms); the roofline's
+    # kernel time comes from those events.
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -585,8 +588,20 @@ def run_ours(args) -> None:
     sampler.start()
     time.sleep(0.3)
     ms_local = timed_pass(False)
+    timers = torch.zeros(24, dtype=torch.int64, device=device)
+    ep.ep_set_phase_timers(timers)
+    ms_timers = timed_pass(False)
+    ep.ep_set_phase_timers(None)
     ms_phased = timed_pass(True)
     clocks = sampler.stop()
+    pt = ep.phase_timer_ms(timers)
+    for ph in ep.PHASES:
+        if pt[ph]["launches"] != args.steps:
+            raise RuntimeError(f"phase timer {ph}: {pt[ph]['launches']} of {args.steps} steps")
+    phases_dev = {"dispatch_notify_with_layout": pt["notify"]["ms"],
+                  "dispatch_copy": pt["copy"]["ms"], "combine": pt["combine"]["ms"]}
+    phases_dev["dispatch"] = phases_dev["dispatch_notify_with_layout"] + phases_dev["dispatch_copy"]
+    phases_dev["step_with_phase_timers"] = ms_timers
     notify_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     copy_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     comb_ms = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
@@ -690,9 +705,14 @@ def run_ours(args) -> None:
         "config": workload_config(T, ws),
         "tokens_per_s": agg["tokens_per_s"],
         "pct_of_8TBps": 100.0 * agg["gbs"] / (SPEC_HBM_GBS * ws),
-        "phases_ms": {"dispatch": disp_ms, "dispatch_notify_with_layout": notify_ms,
-                      "dispatch_copy": copy_ms, "combine": comb_ms,
-                      "step_with_phase_events": ms_phased},
+        "phases_ms": phases_dev,
+        "phases_method": "device full-grid timers: %globaltimer from the earliest block start "
+                         "(after the launch's wait for the previous grid) of a phase's first "
+                         "kernel to the last block end of its last kernel, mean of K steps of "
+                         "the timed sequence with no events between kernels",
+        "phases_event_ms": {"dispatch": disp_ms, "dispatch_notify_with_layout": notify_ms,
+                            "dispatch_copy": copy_ms, "combine": comb_ms,
+                            "step_with_phase_events": ms_phased},
         "phases_graph_replay_ms": phases_graph,
         "bytes_per_step": {"dispatch": bytes_d, "combine": bytes_c, "copies": N},
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,

@@ -110,14 +110,16 @@ int ctas_per_sm(const void *func, int threads, size_t smem) {
 
 namespace {
 
+template <bool kTimed>
 __global__ void __launch_bounds__(256) zero_prefetch_kernel(uint4 *a, long a16, int32_t *b,
                                                             long b_words, const char *pf,
-                                                            long pf_bytes) {
+                                                            long pf_bytes, PhaseTimer *begin) {
   const long nthr = static_cast<long>(gridDim.x) * blockDim.x;
   const long me = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
   for (long off = me * 128; off < pf_bytes; off += nthr * 128)
     asm volatile("prefetch.global.L2 [%0];" ::"l"(pf + off));
   pdl_wait();
+  if constexpr (kTimed) timer_begin(begin);
   pdl_trigger();  // the next kernel's CTAs may start; they wait for this grid to complete
   for (long i = me; i < a16; i += nthr) a[i] = make_uint4(0u, 0u, 0u, 0u);
   for (long i = me; i < b_words; i += nthr) b[i] = 0;
@@ -126,22 +128,34 @@ __global__ void __launch_bounds__(256) zero_prefetch_kernel(uint4 *a, long a16, 
 }  // namespace
 
 int zero_prefetch(void *a, size_t a_bytes, int32_t *b, long b_words, const void *pf,
-                  long pf_bytes, cudaStream_t stream) {
+                  long pf_bytes, cudaStream_t stream, PhaseTimer *begin) {
   if ((reinterpret_cast<uintptr_t>(a) & 15u) != 0 || (a_bytes & 15u) != 0) {
     if (a_bytes > 0 && cudaMemsetAsync(a, 0, a_bytes, stream) != cudaSuccess) return EP_ERR_CUDA;
     if (b_words > 0 &&
         cudaMemsetAsync(b, 0, sizeof(int32_t) * static_cast<size_t>(b_words), stream) !=
             cudaSuccess)
       return EP_ERR_CUDA;
-    return EP_OK;
+    if (begin == nullptr) return EP_OK;
+    a_bytes = 0;  // the kernel only starts the timer
+    b_words = 0;
   }
   const long a16 = static_cast<long>(a_bytes / 16);
   if (pf == nullptr) pf_bytes = 0;
   const long want = (std::max({a16, b_words, (pf_bytes + 127) / 128}) + 255) / 256;
   const long grid = std::max(1L, std::min<long>(want, num_sms()));
-  return launch_status(launch_pdl(zero_prefetch_kernel, dim3(static_cast<unsigned>(grid)),
-                                  dim3(256), 0, stream, static_cast<uint4 *>(a), a16, b, b_words,
-                                  static_cast<const char *>(pf), pf_bytes));
+  auto *kernel = begin != nullptr ? zero_prefetch_kernel<true> : zero_prefetch_kernel<false>;
+  return launch_status(launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(256), 0, stream,
+                                  static_cast<uint4 *>(a), a16, b, b_words,
+                                  static_cast<const char *>(pf), pf_bytes, begin));
+}
+
+namespace {
+std::atomic<PhaseTimer *> g_phase_timers{nullptr};
+}  // namespace
+
+PhaseTimer *phase_timer(int phase) {
+  PhaseTimer *t = g_phase_timers.load(std::memory_order_relaxed);
+  return t != nullptr ? t + phase : nullptr;
 }
 
 }  // namespace ep
@@ -159,6 +173,12 @@ EP_API const char *ep_status_string(int code) {
 }
 
 EP_API int ep_version(void) { return 100; }
+
+EP_API int ep_set_phase_timers(unsigned long long *timers) {
+  if ((reinterpret_cast<uintptr_t>(timers) & 7u) != 0) return EP_ERR_INVALID_ARG;
+  ep::g_phase_timers.store(reinterpret_cast<ep::PhaseTimer *>(timers), std::memory_order_relaxed);
+  return EP_OK;
+}
 
 EP_API int ep_set_wait_timeout_ns(long long ns) {
   if (ns < 0) return EP_ERR_INVALID_ARG;

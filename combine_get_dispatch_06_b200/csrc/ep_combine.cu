@@ -47,16 +47,18 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float (&a)[8]) {
 // at once; kMinCtas: CTAs per SM the registers are sized for.  Two shapes:
 // 8 rows at 2 CTAs per SM, and -- when no token can have more than 6
 // copies -- 6 rows at 3 CTAs per SM, where the extra warps put more loads in
-// flight than the rows of one token can.
-template <bool kTab, int kBatch, int kMinCtas>
+// flight than the rows of one token can.  kTimed: the kernel is the combine
+// phase of the phase timers (tm); the untimed form never reads tm.
+template <bool kTab, int kBatch, int kMinCtas, bool kTimed>
 __global__ void __launch_bounds__(kCombineWarps * 32, kMinCtas)
     combine_kernel(const uint8_t *__restrict__ y, const float *__restrict__ recv_w,
                    const uint8_t *const *y_tab, const float *const *w_tab,
                    const int32_t *__restrict__ send_pos, const uint8_t *__restrict__ bias0,
                    const uint8_t *__restrict__ bias1, int R, long num_tok, int H, int K,
                    int cap, bool want_w, uint8_t *__restrict__ out, float *__restrict__ out_w,
-                   int32_t *status) {
+                   int32_t *status, PhaseTimer *tm) {
   pdl_wait();
+  if constexpr (kTimed) timer_begin(tm);
   // per warp: [R] row pointers of y, then [R] row pointers of recv_w
   extern __shared__ __align__(16) const uint8_t *s_ptr[];
   const int lane = threadIdx.x & 31;
@@ -136,6 +138,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32, kMinCtas)
     }
     __syncwarp();
   }
+  if constexpr (kTimed) timer_end(tm);
 }
 
 // Launch of one instantiation (arguments already checked).
@@ -147,7 +150,9 @@ int combine_launch_as(const void *y, const float *recv_w, const uint8_t *const *
                       cudaStream_t stream) {
   const int threads = kCombineWarps * 32;
   const size_t smem = static_cast<size_t>(kCombineWarps) * 2 * R * sizeof(void *);
-  auto *kernel = combine_kernel<kTab, kBatch, kMinCtas>;
+  PhaseTimer *const tm = kTab ? nullptr : phase_timer(kPhaseCombine);
+  auto *kernel = tm != nullptr ? combine_kernel<kTab, kBatch, kMinCtas, !kTab>
+                               : combine_kernel<kTab, kBatch, kMinCtas, false>;
   const void *fn = reinterpret_cast<const void *>(kernel);
   if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
   const long want = (num_tok + kCombineWarps - 1) / kCombineWarps;
@@ -157,7 +162,7 @@ int combine_launch_as(const void *y, const float *recv_w, const uint8_t *const *
       kernel, dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream,
       static_cast<const uint8_t *>(y), recv_w, y_tab, w_tab, send_pos,
       static_cast<const uint8_t *>(bias_0), static_cast<const uint8_t *>(bias_1), R, num_tok, H,
-      K, cap, combined_w != nullptr, static_cast<uint8_t *>(combined_x), combined_w, status);
+      K, cap, combined_w != nullptr, static_cast<uint8_t *>(combined_x), combined_w, status, tm);
   return launch_status(launched);
 }
 

@@ -28,6 +28,29 @@ WaitConfig wait_config();
 // Number of SMs of the current device (cached per device).
 int num_sms();
 
+// Opt-in full-grid timers of the single-GPU normal path (the "Notify
+// full-kernel duration" timer of the DeepEP PR #720 page, widened to a phase
+// of one or more chained kernels): the earliest block start of the phase's
+// first kernel, taken after its programmatic-dependency wait, to the last
+// block end of its last kernel, both by %globaltimer.  Blocks publish their
+// start as ~t with atomicMax (so the largest complement is the earliest
+// start); the last block of the last kernel to finish adds the interval to
+// the cumulative sum and clears the working slots for the next launch.
+// Layout and use: ep_set_phase_timers in ep.h.
+struct PhaseTimer {
+  unsigned long long start_c;    // ~earliest block start of the launch in progress (0: none)
+  unsigned long long done;       // blocks of the last kernel that have finished
+  unsigned long long sum_ns;     // cumulative phase duration
+  unsigned long long launches;   // phases timed
+  unsigned long long last_start, last_end;
+  unsigned long long reserved[2];
+};
+enum : int { kPhaseNotify = 0, kPhaseCopy = 1, kPhaseCombine = 2, kNumPhases = 3 };
+
+// Host: the timer of `phase` for kernels launched now, or nullptr while the
+// timers are off.
+PhaseTimer *phase_timer(int phase);
+
 // EP_OK for a launch that returned cudaSuccess, else EP_ERR_CUDA.  The
 // launch's own return value is used, not cudaGetLastError(), which would
 // also report (and clear) an error some other code left behind.
@@ -80,8 +103,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // and lets the next one start.  Before that wait it asks L2 for
 // pf[0, pf_bytes) (a hint only; pf may be nullptr).  Falls back to memsets
 // where `a` is not 16-byte aligned or a_bytes not a multiple of 16.
+// `begin`: a phase timer this kernel starts (nullptr: none).
 int zero_prefetch(void *a, size_t a_bytes, int32_t *b, long b_words, const void *pf,
-                  long pf_bytes, cudaStream_t stream);
+                  long pf_bytes, cudaStream_t stream, PhaseTimer *begin = nullptr);
 
 __device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -119,6 +143,32 @@ __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
+}
+
+// Phase timers (see PhaseTimer).  timer_begin: thread 0 of each block of the
+// phase's first kernel, after pdl_wait().  timer_end: every thread of each
+// block of the phase's last kernel, at its end (t is uniform); one atomic per
+// block counts the blocks done.
+__device__ __forceinline__ void timer_begin(PhaseTimer *t) {
+  if (t != nullptr && threadIdx.x == 0) atomicMax(&t->start_c, ~globaltimer());
+}
+
+__device__ __forceinline__ void timer_end(PhaseTimer *t) {
+  if (t == nullptr) return;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  __threadfence();
+  const unsigned long long blocks =
+      static_cast<unsigned long long>(gridDim.x) * gridDim.y * gridDim.z;
+  if (atomicAdd(&t->done, 1ull) + 1ull != blocks) return;
+  __threadfence();
+  const unsigned long long end = globaltimer();
+  const unsigned long long start = ~atomicExch(&t->start_c, 0ull);
+  t->sum_ns += end - start;
+  t->launches += 1ull;
+  t->last_start = start;
+  t->last_end = end;
+  atomicExch(&t->done, 0ull);
 }
 
 __device__ __forceinline__ uint64_t ld_relaxed_gpu(const uint64_t *p) {

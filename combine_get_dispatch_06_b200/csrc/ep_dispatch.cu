@@ -506,15 +506,17 @@ constexpr int kCopyMaxCtasPerSm = 2;
 //
 // kTab: the destinations' receive buffers are given by a table of R pointers
 // (one rank of a sharded job: peers' memory); else they are slices d * cap of
-// recv_x.
-template <int S, bool kTab>
+// recv_x.  kTimed: the kernel is the row-copy phase of the phase timers (tm);
+// the untimed form never reads tm.
+template <int S, bool kTab, bool kTimed>
 __global__ void __launch_bounds__(kMaxRanks)
     dispatch_copy_rows_kernel(const uint8_t *__restrict__ x, const int32_t *__restrict__ send_pos,
                          uint8_t *__restrict__ recv_x, uint8_t *const *recv_tab, int R,
                          long num_tok, int row_bytes, int chunk_bytes, int nchunks,
                          int stage_stride, int cap, int32_t *status,
-                         unsigned long long timeout_ns) {
+                         unsigned long long timeout_ns, PhaseTimer *tm) {
   pdl_wait();
+  if constexpr (kTimed) timer_begin(tm);
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
   uint8_t *buf = smem + 128;
@@ -611,6 +613,7 @@ __global__ void __launch_bounds__(kMaxRanks)
         (void)mbar_wait_bounded(&bars[k % S], static_cast<uint32_t>((k / S) & 1), timeout_ns);
     }
   }
+  if constexpr (kTimed) timer_end(tm);
 }
 
 
@@ -634,11 +637,13 @@ struct CopyArgs {
   int nblk, sc_mode, sc_store_bulk;
   int32_t *status;
   unsigned long long timeout_ns;
+  PhaseTimer *tm;  // the row-copy phase timer (or nullptr)
 };
 
 template <int S, bool kScales>
 __global__ void __launch_bounds__(kMaxRanks) dispatch_copy_planes_kernel(CopyArgs a) {
   pdl_wait();
+  timer_begin(a.tm);
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
   uint8_t *buf = smem + 128;
@@ -768,6 +773,7 @@ __global__ void __launch_bounds__(kMaxRanks) dispatch_copy_planes_kernel(CopyArg
         (void)mbar_wait_bounded(&bars[k % S], static_cast<uint32_t>((k / S) & 1), a.timeout_ns);
     }
   }
+  timer_end(a.tm);
 }
 
 }  // namespace
@@ -801,8 +807,10 @@ struct NotifyFinishParams {
   const int32_t *P;
   int R, E, align;
   int32_t *nrte, *ntpe_out, *ntpr_out;
+  PhaseTimer *tm;  // ends the notify phase timer (or nullptr)
 };
 
+template <bool kTimed>
 __global__ void __launch_bounds__(256) notify_finish_kernel(NotifyFinishParams f) {
   pdl_wait();
   pdl_trigger();
@@ -838,6 +846,7 @@ __global__ void __launch_bounds__(256) notify_finish_kernel(NotifyFinishParams f
   if (f.ntpr_out != nullptr)
     for (long i = me; i < static_cast<long>(f.R) * f.R; i += nthr)
       f.ntpr_out[i] = __ldcg(&f.P[i]) - (i >= f.R ? __ldcg(&f.P[i - f.R]) : 0);
+  if constexpr (kTimed) timer_end(f.tm);
 }
 
 // 32-byte stores need rows that are whole multiples of 32 bytes and a
@@ -880,8 +889,10 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   const int Ectr = topk_idx != nullptr ? E : 0;
   const size_t need = ep_dispatch_workspace_bytes(R, T, Ectr);
   // zeroed by a kernel chained to the scan, which first asks L2 for the ids
+  PhaseTimer *const tm = phase_timer(kPhaseNotify);
   if (zero_prefetch(workspace, need, nullptr, 0, topk_idx,
-                    topk_idx != nullptr ? static_cast<long>(R) * T * K * 8 : 0L, stream) != EP_OK)
+                    topk_idx != nullptr ? static_cast<long>(R) * T * K * 8 : 0L, stream,
+                    tm) != EP_OK)
     return EP_ERR_CUDA;
 
   const int tiles_per_src = (T + kScanTile - 1) / kScanTile;
@@ -954,10 +965,13 @@ int notify_impl(const int64_t *topk_idx, const float *topk_weights,
   f.nrte = num_recv_tokens_per_expert;
   f.ntpe_out = ntpe_out;
   f.ntpr_out = ntpr_out;
+  f.tm = tm;
   const long words = f.recv_idx != nullptr ? static_cast<long>(cap) * K / ((K & 1) == 0 ? 2 : 1)
                                            : 0L;
   const int bx = static_cast<int>(std::max<long>(1L, std::min<long>((words + 255) / 256, 64)));
-  launched = launch_pdl(notify_finish_kernel, dim3(bx, R), dim3(256), 0, stream, f);
+  launched = tm != nullptr
+                 ? launch_pdl(notify_finish_kernel<true>, dim3(bx, R), dim3(256), 0, stream, f)
+                 : launch_pdl(notify_finish_kernel<false>, dim3(bx, R), dim3(256), 0, stream, f);
   return launch_status(launched);
 }
 
@@ -997,6 +1011,7 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
   a.stage_stride = (std::max(a.chunk_bytes, sc_bytes) + 127) & ~127;
   a.status = status;
   a.timeout_ns = wait_config().timeout_ns;
+  a.tm = recv_tab == nullptr ? phase_timer(kPhaseCopy) : nullptr;
   const int stages = short_rows ? kCopyStagesShort : kCopyStages;
   // at most kCopyMaxCtasPerSm CTAs on an SM, also when scheduled early
   const size_t smem =
@@ -1008,12 +1023,16 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
                     : reinterpret_cast<const void *>(dispatch_copy_planes_kernel<kCopyStages, true>);
   else if (recv_tab != nullptr)
     fn = short_rows
-             ? reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStagesShort, true>)
-             : reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStages, true>);
+             ? reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStagesShort, true, false>)
+             : reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStages, true, false>);
+  else if (a.tm != nullptr)
+    fn = short_rows
+             ? reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStagesShort, false, true>)
+             : reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStages, false, true>);
   else
     fn = short_rows
-             ? reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStagesShort, false>)
-             : reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStages, false>);
+             ? reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStagesShort, false, false>)
+             : reinterpret_cast<const void *>(dispatch_copy_rows_kernel<kCopyStages, false, false>);
   if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
   const long grid = std::min<long>(
       a.num_tok,
@@ -1032,21 +1051,29 @@ int copy_impl(const void *x, const float *xs, int col_major, int nblk, const int
   } else {
     auto *tab = reinterpret_cast<uint8_t *const *>(recv_tab);
     if (recv_tab != nullptr && short_rows)
-      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStagesShort, true>, g, b, smem, stream,
+      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStagesShort, true, false>, g, b, smem, stream,
           a.x, a.send_pos, a.recv_x, tab, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
-          a.stage_stride, a.cap, a.status, a.timeout_ns);
+          a.stage_stride, a.cap, a.status, a.timeout_ns, a.tm);
     else if (recv_tab != nullptr)
-      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStages, true>, g, b, smem, stream,
+      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStages, true, false>, g, b, smem, stream,
           a.x, a.send_pos, a.recv_x, tab, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
-          a.stage_stride, a.cap, a.status, a.timeout_ns);
-    else if (short_rows)
-      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStagesShort, false>, g, b, smem,
+          a.stage_stride, a.cap, a.status, a.timeout_ns, a.tm);
+    else if (short_rows && a.tm != nullptr)
+      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStagesShort, false, true>, g, b, smem,
           stream, a.x, a.send_pos, a.recv_x, tab, a.R, a.num_tok, a.row_bytes, a.chunk_bytes,
-          a.nchunks, a.stage_stride, a.cap, a.status, a.timeout_ns);
+          a.nchunks, a.stage_stride, a.cap, a.status, a.timeout_ns, a.tm);
+    else if (short_rows)
+      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStagesShort, false, false>, g, b, smem,
+          stream, a.x, a.send_pos, a.recv_x, tab, a.R, a.num_tok, a.row_bytes, a.chunk_bytes,
+          a.nchunks, a.stage_stride, a.cap, a.status, a.timeout_ns, a.tm);
+    else if (a.tm != nullptr)
+      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStages, false, true>, g, b, smem,
+          stream, a.x, a.send_pos, a.recv_x, tab, a.R, a.num_tok, a.row_bytes, a.chunk_bytes,
+          a.nchunks, a.stage_stride, a.cap, a.status, a.timeout_ns, a.tm);
     else
-      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStages, false>, g, b, smem, stream,
-          a.x, a.send_pos, a.recv_x, tab, a.R, a.num_tok, a.row_bytes, a.chunk_bytes, a.nchunks,
-          a.stage_stride, a.cap, a.status, a.timeout_ns);
+      launched = launch_pdl(dispatch_copy_rows_kernel<kCopyStages, false, false>, g, b, smem,
+          stream, a.x, a.send_pos, a.recv_x, tab, a.R, a.num_tok, a.row_bytes, a.chunk_bytes,
+          a.nchunks, a.stage_stride, a.cap, a.status, a.timeout_ns, a.tm);
   }
   return launch_status(launched);
 }
@@ -1364,7 +1391,7 @@ extern "C" EP_API int ep_shard_notify(
     f.recv_idx = recv_topk_idx;
     const long words = static_cast<long>(cap) * K / ((K & 1) == 0 ? 2 : 1);
     const int bx = static_cast<int>(std::min<long>((words + 255) / 256, 64));
-    launched = launch_pdl(notify_finish_kernel, dim3(bx, 1), dim3(256), 0, stream, f);
+    launched = launch_pdl(notify_finish_kernel<false>, dim3(bx, 1), dim3(256), 0, stream, f);
     return launch_status(launched);
   }
   return EP_OK;

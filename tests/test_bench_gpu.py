@@ -27,7 +27,7 @@ def test_bench_line_carries_the_contract():
     d = json.loads(lines[0])
     for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
               "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
-              "roofline", "e2e", "gpu_launches", "clocks", "phases_ms",
+              "roofline", "e2e", "gpu_launches", "clocks", "phases_ms", "phases_event_ms",
               "phases_graph_replay_ms", "bytes_per_step"):
         assert k in d, k
     assert d["n_gpus"] == 1 and d["steps"] == 3 and d["warmup"] >= 3
@@ -44,6 +44,11 @@ def test_bench_line_carries_the_contract():
     assert d["gpu_launches"] == 5 * d["steps"]
     for ph in ("dispatch_notify_with_layout", "dispatch_copy", "combine"):
         assert d["phases_ms"][ph] > 0 and d["phases_graph_replay_ms"][ph] > 0
+        assert d["phases_event_ms"][ph] > 0
+    # device-timed phases are disjoint spans inside the step that ran them
+    dev = d["phases_ms"]
+    spans = dev["dispatch_notify_with_layout"] + dev["dispatch_copy"] + dev["combine"]
+    assert 0.85 * dev["step_with_phase_timers"] < spans <= 1.001 * dev["step_with_phase_timers"]
     # the three phases alone add up to about one step
     alone = sum(d["phases_graph_replay_ms"].values())
     assert 0.8 * d["ms_per_step"] < alone < 1.2 * d["ms_per_step"]

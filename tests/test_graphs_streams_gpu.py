@@ -185,3 +185,61 @@ def test_independent_calls_on_two_streams():
         check_dispatch(out, ref, w.R, w.K)
         np.testing.assert_array_equal(to_host(cx), ref["combined_x"])
         np.testing.assert_array_equal(to_host(cw), ref["combined_topk_weights"])
+
+
+def test_phase_timers_time_each_phase_of_each_step():
+    """The opt-in full-grid timers (DeepEP PR #720 page, "Notify full-kernel
+    duration"): one timed phase per call, in stream order and disjoint; the
+    results stay the oracle's; a captured graph times its replays; turned
+    off, nothing more is counted."""
+    w = Workload("pt", R=8, T=300, H=256, E=64, K=8, masked_frac=0.05, seed=23)
+    inp, xd, idd, wd = _normal_inputs(w)
+    ref = oracle.normal_path(inp["x"], inp["topk_idx"], inp["topk_weights"], w.E)
+    dev = xd.device
+    out, cx, cw, ws = _normal_buffers(w, dev)
+    st = ep.new_status(dev)
+    timers = torch.zeros(24, dtype=torch.int64, device=dev)
+    ep.ep_set_phase_timers(timers)
+    try:
+        steps = 3
+        for _ in range(steps):
+            _normal_step(w, xd, idd, wd, out, cx, cw, ws, st)
+        torch.cuda.synchronize()
+        v = timers.cpu().tolist()
+        for p in range(3):
+            assert v[8 * p + 0] == 0 and v[8 * p + 1] == 0  # working slots cleared
+            assert v[8 * p + 3] == steps
+            assert v[8 * p + 2] > 0
+            assert 0 < v[8 * p + 4] < v[8 * p + 5]
+        # last step: notify, then copy, then combine, no overlap
+        assert v[5] <= v[8 + 4] and v[8 + 5] <= v[16 + 4]
+        pt = ep.phase_timer_ms(timers)
+        assert all(pt[ph]["launches"] == steps and pt[ph]["ms"] > 0 for ph in ep.PHASES)
+
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            _normal_step(w, xd, idd, wd, out, cx, cw, ws, st)
+        torch.cuda.current_stream(dev).wait_stream(s)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            _normal_step(w, xd, idd, wd, out, cx, cw, ws, st)
+        before = timers.cpu().tolist()
+        g.replay()
+        g.replay()
+        torch.cuda.synchronize()
+        after = timers.cpu().tolist()
+        for p in range(3):
+            assert after[8 * p + 3] == before[8 * p + 3] + 2
+        del g
+    finally:
+        ep.ep_set_phase_timers(None)
+    _scramble(list(out.values()) + [cx, cw])
+    _normal_step(w, xd, idd, wd, out, cx, cw, ws, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    check_dispatch(out, ref, w.R, w.K)
+    np.testing.assert_array_equal(to_host(cx), ref["combined_x"])
+    np.testing.assert_array_equal(to_host(cw), ref["combined_topk_weights"])
+    assert timers.cpu().tolist() == after  # off: nothing more counted
