@@ -138,3 +138,26 @@ def test_sharded_low_latency_argument_checks(lib):
     assert disp(counts=None) == 1            # no gathered counts
     assert lib.ep_shard_ll_combine(f, f, f, f, None, 2, 2, 8, 256, 4, 16, f, None, None) == 1
     assert lib.ep_shard_ll_combine(None, f, f, f, None, 0, 2, 8, 256, 4, 16, f, None, None) == 1
+
+
+def test_phase_timer_switch_checks(lib):
+    """ep_set_phase_timers only records a pointer: an unaligned one is
+    refused, NULL turns the timers off; the binding wants a CUDA int64 tensor
+    of at least 3 x 8 words and reads the mean duration of each phase."""
+    lib.ep_set_phase_timers.argtypes = [ctypes.c_void_p]
+    assert lib.ep_set_phase_timers(ctypes.c_void_p(0x1004)) == 1  # EP_ERR_INVALID_ARG
+    assert lib.ep_set_phase_timers(None) == 0
+    import torch
+
+    import combine_get_dispatch_06_b200 as ep
+    for bad in (torch.zeros(24), torch.zeros(24, dtype=torch.int64)):
+        with pytest.raises(ValueError):
+            ep.ep_set_phase_timers(bad)  # float, or not on a CUDA device
+    ep.ep_set_phase_timers(None)
+    v = torch.zeros(24, dtype=torch.int64)
+    v[2], v[3] = 3_000_000, 2          # notify: 3 ms over 2 phases
+    v[8 + 2], v[8 + 3] = 5_000, 1      # copy: 5 us once
+    pt = ep.phase_timer_ms(v)
+    assert pt["notify"] == {"ms": 1.5, "launches": 2}
+    assert pt["copy"] == {"ms": 0.005, "launches": 1}
+    assert pt["combine"] == {"ms": None, "launches": 0}
