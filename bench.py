@@ -308,16 +308,22 @@ KERNEL_SOURCES = {
 
 
 def kernel_source_hash(kernel: str) -> str:
-    """sha1 of the CUDA sources of `kernel`, to tell whether recorded counters
-    still describe the kernel that runs."""
+    """sha1 of the code of the CUDA sources of `kernel` (comments and blank
+    lines removed, so that an edit of a comment keeps it), to tell whether
+    recorded counters still describe the kernel that runs."""
     import hashlib
+    import re
 
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "combine_get_dispatch_06_b200", "csrc")
     for f in KERNEL_SOURCES[kernel]:
         h.update(f.encode())
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f)) as fh:
+            text = re.sub(r"/\*.*?\*/", "", fh.read(), flags=re.S)
+        for line in text.splitlines():
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                h.update(code.encode() + b"\n")
     return h.hexdigest()
 
 

@@ -1,5 +1,7 @@
 // ep_api.cu -- host-side helpers of the C ABI: status text, version, the
-// process-wide limits of the bounded device waits, device properties.
+// process-wide limits of the bounded device waits and the phase-timer switch,
+// device properties, and the zeroing kernel chained ahead of a notify or an
+// LL dispatch.
 #include <algorithm>
 #include <atomic>
 #include <cstring>

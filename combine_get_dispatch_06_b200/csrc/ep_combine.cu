@@ -11,7 +11,8 @@
 // then each lane owns 16-byte chunks (8 channels) of the hidden row: it issues
 // the loads of two chunks from up to 8 rows at once (16 loads in flight per
 // lane), accumulates in fp32 in list order and writes 16 bytes back.
-// HBM-bound: N*H*2 bytes read, R*T*H*2 bytes written.
+// HBM-bound: N*H*2 bytes read, R*T*H*2 bytes written.  With the phase timers
+// on (ep_set_phase_timers) the single-GPU form runs its timed instance.
 #include <algorithm>
 
 #include "ep_common.cuh"

@@ -7,18 +7,25 @@
 // flattened (s, t) order, of is_token_in_rank[.][.][d]; its value at the end
 // of source rank s is the rank prefix matrix P[s][d].
 //
-// Two kernels:
+// Kernels:
 //   dispatch_scan_kernel  one CTA per 128-token tile: routing bits -> warp
-//                         ballots -> per-rank tile counts -> decoupled
-//                         look-back -> send_pos, recv_src_idx, received
-//                         top-k metadata, P, recv_count; expert counts are
-//                         reduced with shared + global atomics and finalised
-//                         by the last CTA.  Small (a few MB of traffic).
+//                         ballots -> per-rank tile counts -> look-back ->
+//                         send_pos, recv_src_idx, received top-k metadata, P,
+//                         recv_count; expert counts are reduced with shared +
+//                         global atomics.  Small (a few MB of traffic).
+//   notify_finish_kernel  after the scan: -1 padding of the received ids past
+//                         each rank's count, and the gathered counts turned
+//                         into the outputs over the whole grid.
+//   shard_prefix_kernel   one rank of a sharded job: P, its destination bases
+//                         and receive counts from the all-gathered counts.
 //   dispatch_copy_rows_kernel  the data movement: each token row is read ONCE from
 //                         HBM into shared memory by a bulk (TMA) copy and
 //                         written to each destination by bulk shared->global
 //                         copies, S stages deep.  HBM-bound: R*T*H*2 bytes
 //                         read, N*H*2 bytes written (N = number of copies).
+//   dispatch_copy_planes_kernel  the same for e4m3 rows plus their scales.
+// With the phase timers on (ep_set_phase_timers), the notify's finish kernel
+// and the bf16 row copy run their timed instances (template flag kTimed).
 #include <algorithm>
 #include <mutex>
 
