@@ -459,11 +459,28 @@ def extra_configs(device, ep) -> dict:
 
     ms_d = timeit(ll_d, iters=50)
     ms_c = timeit(ll_c, iters=50)
+    # the same back-to-back calls with the full-grid phase timers on: each
+    # call's span from its zeroing kernel's earliest block (after the wait for
+    # the previous call) to its last block, without the hand-off between calls
+    timers = torch.zeros(8 * len(ep.PHASES), dtype=torch.int64, device=device)
+    ep.ep_set_phase_timers(timers)
+    try:
+        timeit(ll_d, iters=50)
+        timeit(ll_c, iters=50)
+    finally:
+        ep.ep_set_phase_timers(None)
+    pt = ep.phase_timer_ms(timers)
+    span_d, span_c = pt["ll_dispatch"]["ms"], pt["ll_combine"]["ms"]
     C = int(cnt.sum())
     out["low_latency"] = {
         "dispatch_us": ms_d * 1e3, "combine_us": ms_c * 1e3,
         "dispatch_gbs": ll_dispatch_bytes(R, T, H, K, C) / (ms_d * 1e-3) / 1e9,
         "combine_gbs": ll_combine_bytes(R, T, H, K, C) / (ms_c * 1e-3) / 1e9,
+        "dispatch_span_us": span_d * 1e3, "combine_span_us": span_c * 1e3,
+        "dispatch_span_gbs": ll_dispatch_bytes(R, T, H, K, C) / (span_d * 1e-3) / 1e9,
+        "combine_span_gbs": ll_combine_bytes(R, T, H, K, C) / (span_c * 1e-3) / 1e9,
+        "span_method": "full-grid phase timers (%globaltimer), mean over the timed calls; "
+                       "dispatch_us / combine_us: CUDA-graph replay time per call",
         "copies": C, "tokens_per_s": R * T / ((ms_d + ms_c) * 1e-3)}
     del x, idx, wt, y, d, out_c
     torch.cuda.empty_cache()
@@ -601,7 +618,7 @@ def run_ours(args) -> None:
     ms_phased = timed_pass(True)
     clocks = sampler.stop()
     pt = ep.phase_timer_ms(timers)
-    for ph in ep.PHASES:
+    for ph in ("notify", "copy", "combine"):
         if pt[ph]["launches"] != args.steps:
             raise RuntimeError(f"phase timer {ph}: {pt[ph]['launches']} of {args.steps} steps")
     phases_dev = {"dispatch_notify_with_layout": pt["notify"]["ms"],

@@ -38,7 +38,7 @@ _SIGS = {
     "ep_version": (_I, []),
     "ep_set_wait_timeout_ns": (_I, [ctypes.c_longlong]),
     "ep_set_debug_flags": (_I, [ctypes.c_uint]),
-    "ep_set_phase_timers": (_I, [_P]),
+    "ep_set_phase_timers": (_I, [_P, ctypes.c_int]),
     "ep_get_dispatch_layout": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
     "ep_dispatch_workspace_bytes": (_Z, [_I, _I, _I]),
     "ep_dispatch": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
@@ -150,25 +150,28 @@ def ep_set_debug_flags(flags: int) -> None:
     _check(_lib.ep_set_debug_flags(int(flags)), "ep_set_debug_flags")
 
 
-PHASES = ("notify", "copy", "combine")
+PHASES = ("notify", "copy", "combine", "ll_dispatch", "ll_combine")
 
 
 def ep_set_phase_timers(timers: Optional[torch.Tensor]) -> None:
-    """Turn the full-grid phase timers on (a zeroed int64 CUDA tensor of
-    3 x 8 words) or off (None); see phase_timer_ms."""
+    """Turn the full-grid phase timers on (a zeroed int64 CUDA tensor of 8
+    words per phase, in PHASES order; a shorter tensor times the first
+    phases only) or off (None); see phase_timer_ms."""
+    n = 0
     if timers is not None:
-        if timers.dtype != torch.int64 or not timers.is_cuda or timers.numel() < 24 \
+        if timers.dtype != torch.int64 or not timers.is_cuda or timers.numel() < 8 \
                 or not timers.is_contiguous():
-            raise ValueError("timers must be a contiguous CUDA int64 tensor of >= 24 words")
-    _check(_lib.ep_set_phase_timers(_ptr(timers)), "ep_set_phase_timers")
+            raise ValueError("timers must be a contiguous CUDA int64 tensor of >= 8 words")
+        n = min(timers.numel() // 8, len(PHASES))
+    _check(_lib.ep_set_phase_timers(_ptr(timers), n), "ep_set_phase_timers")
 
 
 def phase_timer_ms(timers: torch.Tensor) -> dict:
     """Mean duration in ms (and count) of each phase timed into `timers`."""
-    v = timers.view(-1)[:24].cpu().tolist()
+    v = timers.view(-1).cpu().tolist()
     out = {}
     for i, name in enumerate(PHASES):
-        n = v[8 * i + 3]
+        n = v[8 * i + 3] if 8 * i + 8 <= len(v) else 0
         out[name] = {"ms": (v[8 * i + 2] / n / 1e6) if n else None, "launches": n}
     return out
 

@@ -153,11 +153,14 @@ int zero_prefetch(void *a, size_t a_bytes, int32_t *b, long b_words, const void 
 
 namespace {
 std::atomic<PhaseTimer *> g_phase_timers{nullptr};
+std::atomic<int> g_phase_count{0};
 }  // namespace
 
 PhaseTimer *phase_timer(int phase) {
   PhaseTimer *t = g_phase_timers.load(std::memory_order_relaxed);
-  return t != nullptr ? t + phase : nullptr;
+  if (t == nullptr || phase < 0 || phase >= g_phase_count.load(std::memory_order_relaxed))
+    return nullptr;
+  return t + phase;
 }
 
 }  // namespace ep
@@ -176,8 +179,17 @@ EP_API const char *ep_status_string(int code) {
 
 EP_API int ep_version(void) { return 100; }
 
-EP_API int ep_set_phase_timers(unsigned long long *timers) {
-  if ((reinterpret_cast<uintptr_t>(timers) & 7u) != 0) return EP_ERR_INVALID_ARG;
+EP_API int ep_set_phase_timers(unsigned long long *timers, int num_phases) {
+  if (timers == nullptr) {
+    ep::g_phase_timers.store(nullptr, std::memory_order_relaxed);
+    ep::g_phase_count.store(0, std::memory_order_relaxed);
+    return EP_OK;
+  }
+  if ((reinterpret_cast<uintptr_t>(timers) & 7u) != 0 || num_phases < 1 ||
+      num_phases > ep::kNumPhases)
+    return EP_ERR_INVALID_ARG;
+  ep::g_phase_timers.store(nullptr, std::memory_order_relaxed);
+  ep::g_phase_count.store(num_phases, std::memory_order_relaxed);
   ep::g_phase_timers.store(reinterpret_cast<ep::PhaseTimer *>(timers), std::memory_order_relaxed);
   return EP_OK;
 }

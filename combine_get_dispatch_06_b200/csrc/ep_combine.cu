@@ -59,7 +59,8 @@ __global__ void __launch_bounds__(kCombineWarps * 32, kMinCtas)
                    int cap, bool want_w, uint8_t *__restrict__ out, float *__restrict__ out_w,
                    int32_t *status, PhaseTimer *tm) {
   pdl_wait();
-  if constexpr (kTimed) timer_begin(tm);
+  unsigned long long begun = 0ull;
+  if constexpr (kTimed) begun = timer_begin(tm);
   // per warp: [R] row pointers of y, then [R] row pointers of recv_w
   extern __shared__ __align__(16) const uint8_t *s_ptr[];
   const int lane = threadIdx.x & 31;
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32, kMinCtas)
     }
     __syncwarp();
   }
-  if constexpr (kTimed) timer_end(tm);
+  if constexpr (kTimed) timer_end(tm, begun);
 }
 
 // Launch of one instantiation (arguments already checked).

@@ -28,7 +28,7 @@ WaitConfig wait_config();
 // Number of SMs of the current device (cached per device).
 int num_sms();
 
-// Opt-in full-grid timers of the single-GPU normal path (the "Notify
+// Opt-in full-grid timers of the single-GPU entry points (the "Notify
 // full-kernel duration" timer of the DeepEP PR #720 page, widened to a phase
 // of one or more chained kernels): the earliest block start of the phase's
 // first kernel, taken after its programmatic-dependency wait, to the last
@@ -45,10 +45,17 @@ struct PhaseTimer {
   unsigned long long last_start, last_end;
   unsigned long long reserved[2];
 };
-enum : int { kPhaseNotify = 0, kPhaseCopy = 1, kPhaseCombine = 2, kNumPhases = 3 };
+enum : int {
+  kPhaseNotify = 0,
+  kPhaseCopy = 1,
+  kPhaseCombine = 2,
+  kPhaseLLDispatch = 3,
+  kPhaseLLCombine = 4,
+  kNumPhases = 5
+};
 
 // Host: the timer of `phase` for kernels launched now, or nullptr while the
-// timers are off.
+// timers are off or the caller's array has no room for that phase.
 PhaseTimer *phase_timer(int phase);
 
 // EP_OK for a launch that returned cudaSuccess, else EP_ERR_CUDA.  The
@@ -146,22 +153,31 @@ __device__ __forceinline__ uint64_t globaltimer() {
 }
 
 // Phase timers (see PhaseTimer).  timer_begin: thread 0 of each block of the
-// phase's first kernel, after pdl_wait().  timer_end: every thread of each
-// block of the phase's last kernel, at its end (t is uniform); one atomic per
-// block counts the blocks done.
-__device__ __forceinline__ void timer_begin(PhaseTimer *t) {
-  if (t != nullptr && threadIdx.x == 0) atomicMax(&t->start_c, ~globaltimer());
+// phase's first kernel, after pdl_wait(); it returns the stamp's old value.
+// timer_end: every thread of each block of the phase's last kernel, at its
+// end (t is uniform); one atomic per block counts the blocks done.  When the
+// stamp was taken in the same kernel, thread 0 passes the value timer_begin
+// returned: it stores that value before it counts the block, so the stamp
+// (whose result it is) has been performed before the count is issued -- no
+// fence, which delayed every block's exit.  A stamp taken in an earlier
+// kernel of the stream is complete when this kernel passes pdl_wait (pass
+// 0).  The last block reads only the timer's own words, through atomics.
+__device__ __forceinline__ unsigned long long timer_begin(PhaseTimer *t) {
+  if (t == nullptr || threadIdx.x != 0) return 0ull;
+  return atomicMax(&t->start_c, ~globaltimer());
 }
 
-__device__ __forceinline__ void timer_end(PhaseTimer *t) {
+__device__ __forceinline__ void timer_end(PhaseTimer *t, unsigned long long begun) {
+  __shared__ unsigned long long s_begun;
   if (t == nullptr) return;
   __syncthreads();
   if (threadIdx.x != 0) return;
-  __threadfence();
+  asm volatile("st.volatile.shared.u64 [%0], %1;" ::"r"(static_cast<uint32_t>(
+                   __cvta_generic_to_shared(&s_begun))), "l"(begun)
+               : "memory");
   const unsigned long long blocks =
       static_cast<unsigned long long>(gridDim.x) * gridDim.y * gridDim.z;
   if (atomicAdd(&t->done, 1ull) + 1ull != blocks) return;
-  __threadfence();
   const unsigned long long end = globaltimer();
   const unsigned long long start = ~atomicExch(&t->start_c, 0ull);
   t->sum_ns += end - start;

@@ -523,7 +523,8 @@ __global__ void __launch_bounds__(kMaxRanks)
                          int stage_stride, int cap, int32_t *status,
                          unsigned long long timeout_ns, PhaseTimer *tm) {
   pdl_wait();
-  if constexpr (kTimed) timer_begin(tm);
+  unsigned long long begun = 0ull;
+  if constexpr (kTimed) begun = timer_begin(tm);
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
   uint8_t *buf = smem + 128;
@@ -620,7 +621,7 @@ __global__ void __launch_bounds__(kMaxRanks)
         (void)mbar_wait_bounded(&bars[k % S], static_cast<uint32_t>((k / S) & 1), timeout_ns);
     }
   }
-  if constexpr (kTimed) timer_end(tm);
+  if constexpr (kTimed) timer_end(tm, begun);
 }
 
 
@@ -650,7 +651,7 @@ struct CopyArgs {
 template <int S, bool kScales>
 __global__ void __launch_bounds__(kMaxRanks) dispatch_copy_planes_kernel(CopyArgs a) {
   pdl_wait();
-  timer_begin(a.tm);
+  const unsigned long long begun = timer_begin(a.tm);
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem);
   uint8_t *buf = smem + 128;
@@ -780,7 +781,7 @@ __global__ void __launch_bounds__(kMaxRanks) dispatch_copy_planes_kernel(CopyArg
         (void)mbar_wait_bounded(&bars[k % S], static_cast<uint32_t>((k / S) & 1), a.timeout_ns);
     }
   }
-  timer_end(a.tm);
+  timer_end(a.tm, begun);
 }
 
 }  // namespace
@@ -853,7 +854,7 @@ __global__ void __launch_bounds__(256) notify_finish_kernel(NotifyFinishParams f
   if (f.ntpr_out != nullptr)
     for (long i = me; i < static_cast<long>(f.R) * f.R; i += nthr)
       f.ntpr_out[i] = __ldcg(&f.P[i]) - (i >= f.R ? __ldcg(&f.P[i - f.R]) : 0);
-  if constexpr (kTimed) timer_end(f.tm);
+  if constexpr (kTimed) timer_end(f.tm, 0ull);  // begun by the zeroing kernel
 }
 
 // 32-byte stores need rows that are whole multiples of 32 bytes and a

@@ -424,14 +424,14 @@ __host__ __device__ inline LLSmem ll_smem_plan(int H) {
 // kTab: one rank of a sharded job; the slabs of destination d are recv_tab[d]
 // ([El][cap] rows) and scales_tab[d] in peer memory, and warp 0 turns each
 // slot's row into the two row pointers.
-template <bool kFP8, bool kTab>
+template <bool kFP8, bool kTab, bool kTimed>
 __global__ void __launch_bounds__(kLLThreads)
     ll_dispatch_kernel(const uint8_t *__restrict__ x, const int64_t *__restrict__ topk_idx,
                        const int32_t *pos_mirror, long num_tok, int H, int K, int E, int cap,
                        int round_scale, int ue8m0, LLSmem plan, uint8_t *__restrict__ recv,
                        void *__restrict__ scales_out, uint32_t *claim, int32_t *status,
                        unsigned long long timeout_ns, uint8_t *const *recv_tab,
-                       uint8_t *const *scales_tab, int El) {
+                       uint8_t *const *scales_tab, int El, PhaseTimer *tm) {
   pdl_trigger();  // the next kernel may take the room this grid leaves
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ long s_tok[kLLMaxStages];  // token in each input stage, -1 = none
@@ -672,6 +672,7 @@ __global__ void __launch_bounds__(kLLThreads)
   if constexpr (kTab) __threadfence_system();  // rows stored into peers' memory
   // the scan grid completes before this one does
   pdl_wait();
+  if constexpr (kTimed) timer_end(tm, 0ull);  // begun by the zeroing kernel
 }
 
 // ---------------------------------------------------------------------------
@@ -748,13 +749,17 @@ constexpr int kLLCombineWarps = 8;
 // a sharded job (its tokens are source rank s0's); expert e's rows are in
 // destination e / El's slab y_tab[e / El] in peer memory, read with plain
 // loads.  Otherwise y holds every destination's slabs and s0 = 0.
+template <bool kTimed>
 __global__ void __launch_bounds__(kLLCombineWarps * 32)
     ll_combine_kernel(const uint8_t *__restrict__ y, const uint8_t *const *y_tab, int s0,
                       const int64_t *__restrict__ topk_idx,
                       const float *__restrict__ topk_w, const int32_t *__restrict__ ll_pos,
                       const int32_t *__restrict__ mask, long num_tok, int T, int H, int K, int E,
-                      int cap, int nseg, uint8_t *__restrict__ out, int32_t *status) {
+                      int cap, int nseg, uint8_t *__restrict__ out, int32_t *status,
+                      PhaseTimer *tm) {
   pdl_wait();
+  unsigned long long begun = 0ull;
+  if constexpr (kTimed) begun = timer_begin(tm);
   __shared__ const uint8_t *s_row[kLLCombineWarps][kMaxTopk];
   __shared__ float s_w[kLLCombineWarps][kMaxTopk];
   const int lane = threadIdx.x & 31;
@@ -834,6 +839,7 @@ __global__ void __launch_bounds__(kLLCombineWarps * 32)
     }
     __syncwarp();
   }
+  if constexpr (kTimed) timer_end(tm, begun);
 }
 
 }  // namespace
@@ -853,9 +859,11 @@ size_t ll_mirror_offset(long tiles, int E) {  // 16-byte aligned
 int ll_combine_launch(const uint8_t *y, const uint8_t *const *y_tab, int s0,
                       const int64_t *topk_idx, const float *topk_weights, const int32_t *ll_pos,
                       const int32_t *rank_mask, long num_tok, int T, int H, int K, int E,
-                      long cap, void *out, int32_t *status, cudaStream_t stream) {
+                      long cap, void *out, int32_t *status, cudaStream_t stream,
+                      PhaseTimer *tm = nullptr) {
   const int threads = kLLCombineWarps * 32;
-  const void *fn = reinterpret_cast<const void *>(ll_combine_kernel);
+  auto *kernel = tm != nullptr ? ll_combine_kernel<true> : ll_combine_kernel<false>;
+  const void *fn = reinterpret_cast<const void *>(kernel);
   const long resident = static_cast<long>(ctas_per_sm(fn, threads, 0)) * num_sms();
   // split rows into segments until there are >= 4 work items per resident warp
   const int nvec = H / 8;
@@ -863,10 +871,10 @@ int ll_combine_launch(const uint8_t *y, const uint8_t *const *y_tab, int s0,
   nseg = std::max(1, std::min(nseg, std::max(1, nvec / 32)));
   const long items = num_tok * nseg;
   const long grid = std::min<long>((items + kLLCombineWarps - 1) / kLLCombineWarps, resident);
-  const cudaError_t launched = launch_pdl(ll_combine_kernel,
+  const cudaError_t launched = launch_pdl(kernel,
       dim3(static_cast<unsigned>(grid)), dim3(threads), 0, stream, y, y_tab, s0, topk_idx,
       topk_weights, ll_pos, rank_mask, num_tok, T, H, K, E, static_cast<int>(cap), nseg,
-      static_cast<uint8_t *>(out), status);
+      static_cast<uint8_t *>(out), status, tm);
   return launch_status(launched);
 }
 
@@ -877,7 +885,7 @@ int ll_combine_launch(const uint8_t *y, const uint8_t *const *y_tab, int s0,
 int ll_scan_and_dispatch(const LLScanParams &p, const void *x, int H, int use_fp8,
                          int round_scale, int ue8m0, const LLSmem &plan, void *recv_x,
                          void *recv_scales, uint8_t *const *recv_tab, uint8_t *const *scales_tab,
-                         long num_tok, cudaStream_t stream) {
+                         long num_tok, cudaStream_t stream, PhaseTimer *tm = nullptr) {
   cudaError_t launched;
   const dim3 sg(static_cast<unsigned>(p.num_tiles)), sb(kLLScanThreads);
   const bool shard = p.rsi_tab != nullptr;
@@ -890,12 +898,15 @@ int ll_scan_and_dispatch(const LLScanParams &p, const void *x, int H, int use_fp
   if (launch_status(launched) != EP_OK) return EP_ERR_CUDA;
 
   const bool tab = recv_tab != nullptr;
+  if (tab) tm = nullptr;  // the sharded form is never timed
   const size_t smem = spread_smem(static_cast<size_t>(plan.bytes), kLLMaxCtasPerSm);
   const void *fn =
-      use_fp8 ? (tab ? reinterpret_cast<const void *>(ll_dispatch_kernel<true, true>)
-                     : reinterpret_cast<const void *>(ll_dispatch_kernel<true, false>))
-              : (tab ? reinterpret_cast<const void *>(ll_dispatch_kernel<false, true>)
-                     : reinterpret_cast<const void *>(ll_dispatch_kernel<false, false>));
+      use_fp8 ? (tab  ? reinterpret_cast<const void *>(ll_dispatch_kernel<true, true, false>)
+                 : tm ? reinterpret_cast<const void *>(ll_dispatch_kernel<true, false, true>)
+                      : reinterpret_cast<const void *>(ll_dispatch_kernel<true, false, false>))
+              : (tab  ? reinterpret_cast<const void *>(ll_dispatch_kernel<false, true, false>)
+                 : tm ? reinterpret_cast<const void *>(ll_dispatch_kernel<false, false, true>)
+                      : reinterpret_cast<const void *>(ll_dispatch_kernel<false, false, false>));
   if (ensure_dynamic_smem(fn, smem) != EP_OK) return EP_ERR_CUDA;
   const long grid = std::min<long>(
       num_tok,
@@ -906,27 +917,37 @@ int ll_scan_and_dispatch(const LLScanParams &p, const void *x, int H, int use_fp
   uint8_t *rx = static_cast<uint8_t *>(recv_x);
   uint32_t *claim = &p.head->claim;
   const unsigned long long to = p.timeout_ns;
+  uint8_t *const *no_tab = nullptr;
   if (use_fp8 && tab)
-    launched = launch_pdl(ll_dispatch_kernel<true, true>, g, b, smem, stream, xb, p.topk_idx,
-                          p.pos_mirror, num_tok, H, p.K, p.E, p.cap, round_scale, ue8m0, plan,
-                          rx, recv_scales, claim, p.status, to, recv_tab, scales_tab, p.El);
+    launched = launch_pdl(ll_dispatch_kernel<true, true, false>, g, b, smem, stream, xb,
+                          p.topk_idx, p.pos_mirror, num_tok, H, p.K, p.E, p.cap, round_scale,
+                          ue8m0, plan, rx, recv_scales, claim, p.status, to, recv_tab,
+                          scales_tab, p.El, tm);
+  else if (use_fp8 && tm != nullptr)
+    launched = launch_pdl(ll_dispatch_kernel<true, false, true>, g, b, smem, stream, xb,
+                          p.topk_idx, p.pos_mirror, num_tok, H, p.K, p.E, p.cap, round_scale,
+                          ue8m0, plan, rx, recv_scales, claim, p.status, to, no_tab, no_tab,
+                          p.El, tm);
   else if (use_fp8)
-    launched = launch_pdl(ll_dispatch_kernel<true, false>, g, b, smem, stream, xb, p.topk_idx,
-                          p.pos_mirror, num_tok, H, p.K, p.E, p.cap, round_scale, ue8m0, plan,
-                          rx, recv_scales, claim, p.status, to,
-                          static_cast<uint8_t *const *>(nullptr),
-                          static_cast<uint8_t *const *>(nullptr), p.El);
+    launched = launch_pdl(ll_dispatch_kernel<true, false, false>, g, b, smem, stream, xb,
+                          p.topk_idx, p.pos_mirror, num_tok, H, p.K, p.E, p.cap, round_scale,
+                          ue8m0, plan, rx, recv_scales, claim, p.status, to, no_tab, no_tab,
+                          p.El, tm);
   else if (tab)
-    launched = launch_pdl(ll_dispatch_kernel<false, true>, g, b, smem, stream, xb, p.topk_idx,
-                          p.pos_mirror, num_tok, H, p.K, p.E, p.cap, 0, 0, plan, rx,
-                          static_cast<void *>(nullptr), claim, p.status, to, recv_tab,
-                          static_cast<uint8_t *const *>(nullptr), p.El);
+    launched = launch_pdl(ll_dispatch_kernel<false, true, false>, g, b, smem, stream, xb,
+                          p.topk_idx, p.pos_mirror, num_tok, H, p.K, p.E, p.cap, 0, 0, plan, rx,
+                          static_cast<void *>(nullptr), claim, p.status, to, recv_tab, no_tab,
+                          p.El, tm);
+  else if (tm != nullptr)
+    launched = launch_pdl(ll_dispatch_kernel<false, false, true>, g, b, smem, stream, xb,
+                          p.topk_idx, p.pos_mirror, num_tok, H, p.K, p.E, p.cap, 0, 0, plan, rx,
+                          static_cast<void *>(nullptr), claim, p.status, to, no_tab, no_tab,
+                          p.El, tm);
   else
-    launched = launch_pdl(ll_dispatch_kernel<false, false>, g, b, smem, stream, xb, p.topk_idx,
-                          p.pos_mirror, num_tok, H, p.K, p.E, p.cap, 0, 0, plan, rx,
-                          static_cast<void *>(nullptr), claim, p.status, to,
-                          static_cast<uint8_t *const *>(nullptr),
-                          static_cast<uint8_t *const *>(nullptr), p.El);
+    launched = launch_pdl(ll_dispatch_kernel<false, false, false>, g, b, smem, stream, xb,
+                          p.topk_idx, p.pos_mirror, num_tok, H, p.K, p.E, p.cap, 0, 0, plan, rx,
+                          static_cast<void *>(nullptr), claim, p.status, to, no_tab, no_tab,
+                          p.El, tm);
   return launch_status(launched);
 }
 }  // namespace
@@ -992,9 +1013,10 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   // the call's first kernel zeroes them (the workspace is at least
   // ep_ll_workspace_bytes, a multiple of 256 bytes past `used`, so whole
   // 16-byte words stay inside it), prefetching the ids the scan reads first
+  PhaseTimer *const tm = phase_timer(kPhaseLLDispatch);
   if (zero_prefetch(workspace, (used + 15) & ~static_cast<size_t>(15), layout_range,
                     tiles_per_src > 1 ? 2L * E * R : 0L, topk_idx,
-                    static_cast<long>(R) * T * K * 8, stream) != EP_OK)
+                    static_cast<long>(R) * T * K * 8, stream, tm) != EP_OK)
     return EP_ERR_CUDA;
 
   uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1025,7 +1047,7 @@ extern "C" EP_API int ep_ll_dispatch(const void *x, const int64_t *topk_idx,
   p.timeout_ns = wc.timeout_ns;
   p.flags = wc.flags;
   return ll_scan_and_dispatch(p, x, H, use_fp8, round_scale, ue8m0, plan, recv_x, recv_scales,
-                              nullptr, nullptr, static_cast<long>(R) * T, stream);
+                              nullptr, nullptr, static_cast<long>(R) * T, stream, tm);
 }
 
 extern "C" EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
@@ -1048,7 +1070,7 @@ extern "C" EP_API int ep_ll_combine(const void *y, const int64_t *topk_idx,
   if (cap > 0x7fffffffL) return EP_ERR_UNSUPPORTED;
   return ll_combine_launch(static_cast<const uint8_t *>(y), nullptr, 0, topk_idx, topk_weights,
                            ll_pos, rank_mask, static_cast<long>(R) * T, T, H, K, E, cap, out,
-                           status, stream);
+                           status, stream, phase_timer(kPhaseLLCombine));
 }
 
 // ---------------------------------------------------------------------------

@@ -98,7 +98,7 @@ EP_API int ep_set_wait_timeout_ns(long long ns);
 EP_API int ep_set_debug_flags(unsigned flags);
 
 /*
- * Opt-in full-grid phase timers of the single-GPU normal path.
+ * Opt-in full-grid phase timers of the single-GPU entry points.
  * Passage: DeepEP PR #720 page, "Notify full-kernel duration": thread 0 of
  * every block publishes its %globaltimer at entry, a complemented atomicMax
  * keeps the earliest block start, and the last block to complete records the
@@ -107,28 +107,33 @@ EP_API int ep_set_debug_flags(unsigned flags);
  * its first kernel (after that kernel's wait for the previous grid in the
  * stream) and ends at the last block of its last kernel.
  *
- *   timers   device memory, 8-byte aligned, 3 x 8 uint64 (zeroed by the
- *            caller before the first timed launch), or NULL to turn the
- *            timers off.  Phase p in 0..2 owns timers[8p .. 8p+7]:
- *              p = 0  notify (ep_notify_dispatch, and the notify half of
- *                     ep_dispatch / ep_dispatch_noalloc): zeroing, scan and
- *                     finish kernels;
- *              p = 1  row copy (ep_dispatch_cached, ep_dispatch_fp8, the copy
- *                     half of ep_dispatch / ep_dispatch_noalloc);
- *              p = 2  combine (ep_combine);
- *            [8p+0] and [8p+1] are working slots (the complemented earliest
- *            start and the finished-block count of the launch in progress;
- *            each launch returns them to 0), [8p+2] the cumulative duration
- *            in ns, [8p+3] the number of phases timed, [8p+4] and [8p+5] the
- *            last phase's start and end (%globaltimer ns).
+ *   timers      device memory, 8-byte aligned, num_phases x 8 uint64 (zeroed
+ *               by the caller before the first timed launch), or NULL to turn
+ *               the timers off.  Phase p owns timers[8p .. 8p+7]:
+ *                 p = 0  notify (ep_notify_dispatch, and the notify half of
+ *                        ep_dispatch / ep_dispatch_noalloc): zeroing, scan and
+ *                        finish kernels;
+ *                 p = 1  row copy (ep_dispatch_cached, ep_dispatch_cached_fp8,
+ *                        the copy half of ep_dispatch / ep_dispatch_noalloc);
+ *                 p = 2  combine (ep_combine);
+ *                 p = 3  LL dispatch (ep_ll_dispatch): zeroing, scan and the
+ *                        dispatch kernel that runs beside the scan;
+ *                 p = 4  LL combine (ep_ll_combine);
+ *               [8p+0] and [8p+1] are working slots (the complemented earliest
+ *               start and the finished-block count of the launch in progress;
+ *               each launch returns them to 0), [8p+2] the cumulative duration
+ *               in ns, [8p+3] the number of phases timed, [8p+4] and [8p+5] the
+ *               last phase's start and end (%globaltimer ns).
+ *   num_phases  1..5: phases p >= num_phases are not timed (ignored for NULL).
  *
  * Process-wide; read when a call launches its kernels, so it applies to the
- * calls issued after it.  The sharded (ep_shard_*) and low-latency entry
- * points never time.  Phases of one timer must not overlap: time one stream.
- * The memory must stay valid while calls that saw it may still run.
- * Returns EP_ERR_INVALID_ARG for a pointer that is not 8-byte aligned.
+ * calls issued after it (a CUDA graph keeps what its capture saw).  The
+ * sharded (ep_shard_*) entry points never time.  Phases of one timer must not
+ * overlap: time one stream.  The memory must stay valid while calls that saw
+ * it may still run.  Returns EP_ERR_INVALID_ARG for a pointer that is not
+ * 8-byte aligned or num_phases outside 1..5.
  */
-EP_API int ep_set_phase_timers(unsigned long long *timers);
+EP_API int ep_set_phase_timers(unsigned long long *timers, int num_phases);
 
 /*
  * A1: get_dispatch_layout.

@@ -144,9 +144,11 @@ def test_phase_timer_switch_checks(lib):
     """ep_set_phase_timers only records a pointer: an unaligned one is
     refused, NULL turns the timers off; the binding wants a CUDA int64 tensor
     of at least 3 x 8 words and reads the mean duration of each phase."""
-    lib.ep_set_phase_timers.argtypes = [ctypes.c_void_p]
-    assert lib.ep_set_phase_timers(ctypes.c_void_p(0x1004)) == 1  # EP_ERR_INVALID_ARG
-    assert lib.ep_set_phase_timers(None) == 0
+    lib.ep_set_phase_timers.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    assert lib.ep_set_phase_timers(ctypes.c_void_p(0x1004), 3) == 1  # EP_ERR_INVALID_ARG
+    assert lib.ep_set_phase_timers(ctypes.c_void_p(0x1000), 0) == 1  # no phase
+    assert lib.ep_set_phase_timers(ctypes.c_void_p(0x1000), 6) == 1  # past the last phase
+    assert lib.ep_set_phase_timers(None, 0) == 0
     import torch
 
     import combine_get_dispatch_06_b200 as ep
@@ -161,3 +163,4 @@ def test_phase_timer_switch_checks(lib):
     assert pt["notify"] == {"ms": 1.5, "launches": 2}
     assert pt["copy"] == {"ms": 0.005, "launches": 1}
     assert pt["combine"] == {"ms": None, "launches": 0}
+    assert pt["ll_dispatch"] == {"ms": None, "launches": 0}  # not in a 3-phase array

@@ -214,7 +214,8 @@ def test_phase_timers_time_each_phase_of_each_step():
         # last step: notify, then copy, then combine, no overlap
         assert v[5] <= v[8 + 4] and v[8 + 5] <= v[16 + 4]
         pt = ep.phase_timer_ms(timers)
-        assert all(pt[ph]["launches"] == steps and pt[ph]["ms"] > 0 for ph in ep.PHASES)
+        assert all(pt[ph]["launches"] == steps and pt[ph]["ms"] > 0
+                   for ph in ("notify", "copy", "combine"))
 
         g = torch.cuda.CUDAGraph()
         s = torch.cuda.Stream(dev)
@@ -243,3 +244,58 @@ def test_phase_timers_time_each_phase_of_each_step():
     np.testing.assert_array_equal(to_host(cx), ref["combined_x"])
     np.testing.assert_array_equal(to_host(cw), ref["combined_topk_weights"])
     assert timers.cpu().tolist() == after  # off: nothing more counted
+
+
+def test_phase_timers_time_the_low_latency_pair():
+    """Phases 3 and 4 of the full-grid timers: one LL dispatch span (zeroing,
+    scan and the dispatch kernel beside it) and one LL combine span per call,
+    disjoint and in stream order; results still the oracle's; a 3-phase array
+    leaves the LL calls untimed."""
+    w = Workload("plt", R=8, T=200, H=512, E=32, K=6, masked_frac=0.05, seed=24)
+    inp = make(w)
+    xd, idd, wd = to_dev(inp["x"]), to_dev(inp["topk_idx"]), to_dev(inp["topk_weights"])
+    ref = oracle.ll_layout(inp["topk_idx"], w.E)
+    rq, rs = oracle.ll_dispatch_rows(inp["x"], inp["topk_idx"], ref["ll_pos"], w.E, use_fp8=True)
+    yh = oracle.dequant_rows(rq, rs)
+    ro = oracle.ll_combine(yh, inp["topk_idx"], inp["topk_weights"], ref["ll_pos"])
+    dev = xd.device
+    ws = torch.empty(ep.ep_ll_workspace_bytes(w.R, w.T, w.E), dtype=torch.uint8, device=dev)
+    st = ep.new_status(dev)
+    y = to_dev(yh)
+    timers = torch.zeros(40, dtype=torch.int64, device=dev)
+    ep.ep_set_phase_timers(timers)
+    try:
+        steps = 3
+        for _ in range(steps):
+            d = ep.ep_ll_dispatch(xd, idd, w.E, use_fp8=True, workspace=ws, status=st)
+            co = ep.ep_ll_combine(y, idd, wd, d["ll_pos"], status=st)
+        torch.cuda.synchronize()
+        v = timers.cpu().tolist()
+    finally:
+        ep.ep_set_phase_timers(None)
+    assert int(st.item()) == 0
+    for p in (3, 4):
+        assert v[8 * p + 0] == 0 and v[8 * p + 1] == 0
+        assert v[8 * p + 3] == steps and v[8 * p + 2] > 0
+        assert 0 < v[8 * p + 4] < v[8 * p + 5]
+    assert v[24 + 5] <= v[32 + 4]  # last dispatch ends before the last combine starts
+    assert all(v[8 * p + 3] == 0 for p in range(3))  # no normal-path call was made
+    np.testing.assert_array_equal(to_host(d["ll_pos"]), ref["ll_pos"])
+    np.testing.assert_array_equal(to_host(d["recv_count"]), ref["recv_count"])
+    np.testing.assert_array_equal(to_host(co), ro)
+    q, sc = to_host(d["recv_x"]), to_host(d["recv_scales"])
+    for r in range(w.R):
+        for j in range(w.E // w.R):
+            n = ref["recv_count"][r, j]
+            np.testing.assert_array_equal(q[r, j, :n], rq[r, j, :n])
+            np.testing.assert_array_equal(sc[r, j, :n], rs[r, j, :n])
+    # an array with room for the three normal-path phases only
+    short = torch.zeros(24, dtype=torch.int64, device=dev)
+    ep.ep_set_phase_timers(short)
+    try:
+        ep.ep_ll_dispatch(xd, idd, w.E, use_fp8=True, out=d, workspace=ws, status=st)
+        ep.ep_ll_combine(y, idd, wd, d["ll_pos"], out=co, status=st)
+        torch.cuda.synchronize()
+    finally:
+        ep.ep_set_phase_timers(None)
+    assert int(st.item()) == 0 and short.cpu().tolist() == [0] * 24
